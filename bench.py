@@ -1,0 +1,404 @@
+#!/usr/bin/env python3
+"""Benchmark: shifted-window attention forward + backward on B200.
+
+One step = one pass of the whole path (pad, shift, partition, masked window
+attention with relative-position bias, reverse, unshift; then the backward with
+dq, dk, dv and the bias-table gradient) over one batch of the synthetic
+1/12-degree-shaped workload (256 x 544 tokens, 16 heads x 64, 8 x 8 windows,
+shift 4, bf16), inputs resident in HBM. Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  (N > 1: launched by torch.distributed.run, one process per GPU; every rank
+  runs its own batch -- windows and batches are independent, so there is no
+  data-path collective; scaling is weak.)
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the pages ship no runnable implementation).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from shifted_window_attention_pad_b200 import WORKLOADS, BENCH_WORKLOAD  # noqa: E402
+from shifted_window_attention_pad_b200.synth import make_inputs  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+METRIC = "shifted-window attn fwd+bwd tokens/s"
+DOMINANT = "bwd_kernel<64,64> (fused backward: S, dP, dV, dQ, dK, dT)"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0,
+                    help="CPU seconds for the oracle baseline sample")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def init_dist(world, backend):
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (identity without a group)."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(wl, rank):
+    """Each rank draws its own batch of the same shape."""
+    return wl.seed + 1000 * rank
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", FALLBACK_BF16_TFLOPS)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in ("shifted_window_attention_pad_b200/csrc/fast_sm100.cu",
+                "shifted_window_attention_pad_b200/csrc/sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when absent or taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[workload]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only) on a thread."""
+
+    def __init__(self, device, period_s=0.02):
+        self.period, self.samples, self.ok = period_s, [], False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:
+                uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device.index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        nv = self.nv
+        names = {"hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+                 "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+                 "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+                 "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4)}
+        seen = set()
+        for _, rs in self.samples:
+            for n, bit in names.items():
+                if rs & bit:
+                    seen.add(n)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(seen),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs (baseline and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample_step(wl, rows, inp_np):
+    """One oracle forward + backward on the sample: head 0 of the workload's
+    first `rows` grid rows of image 0 (a problem of the same window, shift and
+    head size). Returns (tokens of the full workload the work stands for, s)."""
+    import oracle
+    s = oracle.make_shape(1, rows, wl.W, wl.win, wl.shift, 1, wl.head_dim)
+    q, k, v, do, T = inp_np
+    t0 = time.perf_counter()
+    oracle.forward(s, q[:, :rows], k[:, :rows], v[:, :rows], T)
+    oracle.backward(s, q[:, :rows], k[:, :rows], v[:, :rows], T, do[:, :rows])
+    dt = time.perf_counter() - t0
+    # work is uniform per (token, head): the sample stands for rows*W tokens of one head
+    return rows * wl.W / wl.heads, dt
+
+
+def oracle_inputs(wl, rows):
+    inp = make_inputs(wl)
+    f = lambda t: np.ascontiguousarray(t[:1, :rows, :, :1].to(torch.float64).numpy())
+    return (f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["dout"]),
+            np.ascontiguousarray(inp["table"][:, :1].to(torch.float64).numpy()))
+
+
+def pick_rows(wl, budget_s):
+    """Largest multiple of the window (<= H) whose oracle step fits the budget,
+    from a calibration step on one window row."""
+    import oracle
+    rows0 = min(wl.win, wl.H)
+    inp = oracle_inputs(wl, wl.H)
+    _, dt = oracle_sample_step(wl, rows0, inp)
+    per_row = dt / rows0
+    rows = int(budget_s / max(per_row, 1e-9)) // wl.win * wl.win
+    return max(rows0, min(wl.H, rows)), inp, oracle.num_threads()
+
+
+def cpu_baseline(wl, budget_s):
+    rows, inp, cores = pick_rows(wl, budget_s)
+    tok, dt = oracle_sample_step(wl, rows, inp)
+    return {"value": tok / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "fp64 oracle fwd+bwd on head 0 of grid rows 0..%d (x %d cols) of image 0; "
+                      "%.1f s; scaled to tokens/s of the full %d-head workload" %
+                      (rows - 1, wl.W, dt, wl.heads)}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    steps, warmup = args.steps, args.warmup
+    per_step = max(0.5, min(20.0, 150.0 / max(1, steps + warmup)))
+    rows, inp, cores = pick_rows(wl, per_step)
+    for _ in range(warmup):
+        oracle_sample_step(wl, rows, inp)
+    tok_total, t_total = 0.0, 0.0
+    for _ in range(steps):
+        tok, dt = oracle_sample_step(wl, rows, inp)
+        tok_total += tok
+        t_total += dt
+    value = tok_total / t_total
+    sample = ("fp64 oracle fwd+bwd per step on head 0 of grid rows 0..%d (x %d cols) of image 0, "
+              "scaled to tokens/s of the full %d-head workload" % (rows - 1, wl.W, wl.heads))
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": warmup, "ms_per_step": 1e3 * t_total / max(1, steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "grid": [wl.B, wl.H, wl.W], "window": wl.win,
+                       "shift": wl.shift, "heads": wl.heads, "head_dim": wl.head_dim},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    from shifted_window_attention_pad_b200 import binding as sb
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    wl = WORKLOADS[args.workload]
+    desc = sb.desc_for(wl)
+    inp = make_inputs(wl, seed=rank_seed(wl, rank))
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "dout"))
+    T = inp["table"].to(dev)
+    out, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    dT = torch.empty_like(T)
+    ws = sb.new_workspace(desc, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sb.swin_wattn_fwd(desc, q, k, v, T, out, None, ws, stream)
+        sb.swin_wattn_bwd(desc, q, k, v, T, do, dq, dk, dv, dT, ws, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if sb.swin_wattn_poll_status(ws) != 0:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = sb.swin_wattn_launch_count()
+    with ClockSampler(dev) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            sb.swin_wattn_fwd(desc, q, k, v, T, out, None, ws, stream)
+            ev[i][1].record(stream)
+            sb.swin_wattn_bwd(desc, q, k, v, T, do, dq, dk, dv, dT, ws, stream)
+            ev[i][2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    launches = sb.swin_wattn_launch_count() - launches0
+    ms = max_over_ranks(start.elapsed_time(end), dev)
+    if sb.swin_wattn_poll_status(ws) != 0:
+        raise RuntimeError("device-side timeout in the timed region")
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+
+    secs = ms / 1e3
+    tokens = wl.tokens * K * world
+    value = tokens / secs
+    tflops = wl.flops_fwd_bwd() * K * world / secs / 1e12
+    hbm, _, peak_src = measured_peaks()
+    bwd_bytes = wl.alg_bytes_bwd()
+    achieved = bwd_bytes / (bwd_ms / 1e3) / 1e9
+    fwd_achieved = wl.alg_bytes_fwd() / (fwd_ms / 1e3) / 1e9
+    step_gbs = (wl.alg_bytes_fwd() + wl.alg_bytes_bwd()) * K / secs / 1e9
+
+    # end to end through the public API with pinned host buffers
+    hq, hk, hv, hdo = (inp[n].pin_memory() for n in ("q", "k", "v", "dout"))
+    hT = inp["table"].pin_memory()
+    ho, hdq, hdk, hdv = (torch.empty_like(hq).pin_memory() for _ in range(4))
+    hdT = torch.empty_like(hT).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True); do.copy_(hdo, non_blocking=True)
+        T.copy_(hT, non_blocking=True)
+        sb.swin_wattn_fwd(desc, q, k, v, T, out, None, ws, stream)
+        sb.swin_wattn_bwd(desc, q, k, v, T, do, dq, dk, dv, dT, ws, stream)
+        ho.copy_(out, non_blocking=True); hdq.copy_(dq, non_blocking=True)
+        hdk.copy_(dk, non_blocking=True); hdv.copy_(dv, non_blocking=True)
+        hdT.copy_(dT, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    E = max(1, args.e2e_steps)
+    if world > 1:
+        dist.barrier()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo, hT))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdk, hdv, hdT))
+
+    clk = clocks.summary()
+    if world > 1:
+        allc = [None] * world
+        dist.all_gather_object(allc, clk)
+        clk["reasons"] = sorted(set(r for c in allc for r in (c["reasons"] or [])))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_budget_s)
+
+    if rank == 0:
+        traffic = recorded_traffic(wl.name)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "grid": [wl.B, wl.H, wl.W], "window": wl.win,
+                       "shift": wl.shift, "heads": wl.heads, "head_dim": wl.head_dim,
+                       "tokens_per_rank_step": wl.tokens, "parallelism": "dp%d" % world,
+                       "l2": "inputs larger than L2 (q,k,v,dO = %.2f GB per step)" %
+                             (4 * wl.tokens * wl.heads * wl.head_dim * 2 / 1e9)},
+            "tflops": tflops,
+            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+            "hbm_gbs_step": step_gbs, "hbm_gbs_fwd": fwd_achieved,
+            "roofline": {"bound": "hbm", "kernel": DOMINANT, "achieved": achieved,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "peak_source": peak_src, "traffic": traffic,
+                         "alg_bytes_per_launch": bwd_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": wl.tokens * E * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

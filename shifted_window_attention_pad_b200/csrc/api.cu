@@ -1,0 +1,148 @@
+// api.cu -- the C ABI of libswinwattn.so (declared in include/swin_wattn.h).
+//
+// Host-side checks, workspace sizing and the choice between the tcgen05/TMA
+// kernels (bf16 shapes they cover) and the portable per-token kernels. No
+// device memory is allocated here and no stream is synchronised except by
+// swin_wattn_poll_status.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/swin_wattn.h"
+#include "kernels.h"
+
+namespace swin {
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static int check_desc(const swin_wattn_desc* d) {
+  if (!d) return SWIN_ERR_INVALID_ARG;
+  if (d->B < 1 || d->H < 1 || d->W < 1) return SWIN_ERR_INVALID_ARG;
+  if (d->win_h < 1 || d->win_w < 1 || d->win_h > 64 || d->win_w > 64) return SWIN_ERR_INVALID_ARG;
+  if (d->shift_h < 0 || d->shift_h >= d->win_h) return SWIN_ERR_INVALID_ARG;
+  if (d->shift_w < 0 || d->shift_w >= d->win_w) return SWIN_ERR_INVALID_ARG;
+  if (d->heads < 1 || d->head_dim < 8 || d->head_dim > 256 || (d->head_dim & 7))
+    return SWIN_ERR_INVALID_ARG;
+  if (d->dtype != SWIN_DTYPE_F32 && d->dtype != SWIN_DTYPE_BF16) return SWIN_ERR_UNSUPPORTED;
+  const long long Hp = (d->H + d->win_h - 1) / d->win_h * (long long)d->win_h;
+  const long long Wp = (d->W + d->win_w - 1) / d->win_w * (long long)d->win_w;
+  // Token ids of the index map are int32; grid offsets stay far inside int64.
+  if ((long long)d->B * Hp * Wp > 0x7fffffffLL) return SWIN_ERR_INVALID_ARG;
+  if ((long long)d->B * Hp * Wp * d->heads * d->head_dim > (1LL << 40)) return SWIN_ERR_INVALID_ARG;
+  return SWIN_OK;
+}
+
+static bool use_fast(const swin_wattn_desc* d, const Geo& g) {
+  return !(d->flags & SWIN_FLAG_FORCE_GENERIC) && fast_supported(g, d->dtype);
+}
+
+static int cuda_status(cudaError_t e) { return e == cudaSuccess ? SWIN_OK : SWIN_ERR_CUDA; }
+
+static size_t need_workspace(const swin_wattn_desc* d, const Geo& g) {
+  return use_fast(d, g) ? fast_workspace(g) : generic_workspace(g);
+}
+
+static int check_ws(const swin_wattn_desc* d, const Geo& g, void* ws, size_t bytes) {
+  if (!ws || ((uintptr_t)ws & 255u)) return SWIN_ERR_WORKSPACE;
+  if (bytes < need_workspace(d, g)) return SWIN_ERR_WORKSPACE;
+  return SWIN_OK;
+}
+
+}  // namespace swin
+
+using namespace swin;
+
+extern "C" {
+
+int swin_wattn_path(const swin_wattn_desc* desc) {
+  const int rc = check_desc(desc);
+  if (rc) return rc;
+  return use_fast(desc, make_geo(*desc)) ? 1 : 0;
+}
+
+int swin_wattn_workspace_size(const swin_wattn_desc* desc, size_t* bytes) {
+  const int rc = check_desc(desc);
+  if (rc) return rc;
+  if (!bytes) return SWIN_ERR_INVALID_ARG;
+  *bytes = need_workspace(desc, make_geo(*desc));
+  return SWIN_OK;
+}
+
+int swin_wattn_fwd(const swin_wattn_desc* desc, const void* q, const void* k, const void* v,
+                   const float* bias_table, void* out, float* lse, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  int rc = check_desc(desc);
+  if (rc) return rc;
+  if (!q || !k || !v || !bias_table || !out) return SWIN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(bias_table) || (lse && !aligned16(lse)))
+    return SWIN_ERR_INVALID_ARG;
+  const Geo g = make_geo(*desc);
+  rc = check_ws(desc, g, workspace, workspace_bytes);
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (use_fast(desc, g))
+    return cuda_status(fast_forward(g, q, k, v, bias_table, out, lse, workspace, desc->flags, st));
+  return cuda_status(
+      generic_forward(g, desc->dtype, q, k, v, bias_table, out, lse, workspace, st));
+}
+
+int swin_wattn_bwd(const swin_wattn_desc* desc, const void* q, const void* k, const void* v,
+                   const float* bias_table, const void* dout, void* dq, void* dk, void* dv,
+                   float* dbias_table, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_desc(desc);
+  if (rc) return rc;
+  if (!q || !k || !v || !bias_table || !dout || !dq || !dk || !dv || !dbias_table)
+    return SWIN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, bias_table, dout, dq, dk, dv, dbias_table};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return SWIN_ERR_INVALID_ARG;
+  const Geo g = make_geo(*desc);
+  rc = check_ws(desc, g, workspace, workspace_bytes);
+  if (rc) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (use_fast(desc, g))
+    return cuda_status(fast_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
+                                     workspace, desc->flags, st));
+  return cuda_status(generic_backward(g, desc->dtype, q, k, v, bias_table, dout, dq, dk, dv,
+                                      dbias_table, workspace, st));
+}
+
+int swin_wattn_index_map(const swin_wattn_desc* desc, int32_t* map, void* stream) {
+  const int rc = check_desc(desc);
+  if (rc) return rc;
+  if (!map) return SWIN_ERR_INVALID_ARG;
+  return cuda_status(index_map(make_geo(*desc), map, (cudaStream_t)stream));
+}
+
+int swin_wattn_poll_status(void* workspace, int* device_status, void* stream) {
+  if (!workspace || !device_status) return SWIN_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SWIN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SWIN_ERR_CUDA;
+  *device_status = v;
+  if (v != 0 && cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) return SWIN_ERR_CUDA;
+  return SWIN_OK;
+}
+
+const char* swin_wattn_strerror(int status) {
+  switch (status) {
+    case SWIN_OK: return "ok";
+    case SWIN_ERR_INVALID_ARG: return "invalid argument (null pointer, shape or alignment)";
+    case SWIN_ERR_UNSUPPORTED: return "unsupported dtype/size combination or device";
+    case SWIN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SWIN_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case SWIN_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+    default: return "unknown status";
+  }
+}
+
+uint64_t swin_wattn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,900 @@
+// fast_sm100.cu -- tcgen05 / TMA kernels for shifted-window attention on B200.
+//
+// What they compute: shifted-window multi-head self-attention over a padded
+// token grid (TERRA page, Abstract: window-based Swin Transformer with
+// "shifted-window execution" over ragged window layouts; Table I: the padded
+// resolution H^ x W^), read as the published Swin scheme -- pad, cyclic shift,
+// window partition, softmax(q k^T / sqrt(d) + relative-position bias + shift
+// mask) v, window reverse, reverse shift -- forward and backward, including the
+// gradient of the relative-position bias table.
+//
+// How, on sm_100a:
+//  * Layout stage folded into TMA addressing. Each window is one 5-D TMA box
+//    [head_dim, 1 head, win_w, win_h, 1 image] of the [B, H, W, heads, hd] tensor,
+//    started at its source position (y0 + s) -- the cyclic shift is a coordinate
+//    offset, the zero padding is the TMA out-of-bounds fill. A window on the wrap
+//    seam is split into up to 2 x 2 sub-boxes (heights win_h - s_h and s_h,
+//    widths likewise); their rows land back to back in shared memory and every
+//    consumer knows the resulting slot order. No permuted copy ever exists.
+//  * A tile is 128 rows = G = 128 / N windows of one head (N = win_h * win_w).
+//    S = Q K^T and O = P V (forward) and S, dP = dO V^T, dV = P^T dO, dQ = dS K,
+//    dK = dS^T Q (backward) are tcgen05.mma kind::f16, M = 128, fp32 in TMEM.
+//    Entries of S that pair different windows are never read; the P and dS
+//    tiles keep zeros there, so they contribute nothing.
+//  * One warpgroup reads S (and dP) from TMEM one row per thread, adds the bias
+//    from a table row in shared memory, applies the pad and shift-region mask
+//    from per-slot coordinates (no mask tensor), runs the softmax in registers
+//    (a whole window row is in the tile, so no running rescale is needed), writes
+//    P (and dS) to shared memory for the next MMAs, and stores outputs straight
+//    to their grid rows. The bias-table gradient is summed per warp in shared
+//    memory (lanes of a warp always hit distinct entries), folded per tile in a
+//    fixed order and per CTA, then reduced over CTAs by a second kernel: the sum
+//    order never depends on timing.
+//  * Warp roles: warps 0-3 softmax/epilogue, warp 4 TMA producer, warp 5 MMA
+//    issuer and TMEM owner. Persistent grid of one CTA per SM; tiles go
+//    round-robin, head fastest, so the SMs stream neighbouring bytes together.
+//  * Every mbarrier wait is bounded (%globaltimer); a wait that runs out records
+//    a timeout in the workspace status word and the kernel drains and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace swin {
+namespace {
+
+using namespace ptx;
+
+constexpr int kRows = 128;        // tile rows = TMEM lanes = UMMA M
+constexpr int kWg = 128;          // softmax / epilogue threads (warps 0-3)
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kThreads = 192;
+constexpr int kMaxMaps = 9;       // box shapes: {full, seam part 1, seam part 2}^2
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kTestLimitNs = 1000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct FastParams {
+  CUtensorMap maps[4][kMaxMaps];  // [q, k, v, dout][ky * 3 + kx]
+  Geo g;
+  long long n_groups;             // tiles per head: ceil(n_win / G)
+  long long n_tiles;              // n_groups * heads
+  int bins_pad;
+  int acc_in_smem;                // bias-gradient accumulation per CTA in shared memory
+  float scale_log2;               // head_dim^-1/2 * log2(e)
+  const float* bias_t;            // [heads][bins_pad], times log2(e)
+  void* out0;                     // forward: out;  backward: dq
+  void* out1;                     // backward: dk
+  void* out2;                     // backward: dv
+  float* lse;                     // forward, optional
+  float* partial;                 // backward: bias-gradient partials [unit][heads][bins_pad]
+  int* status;                    // device status word (workspace header)
+  int test_timeout;
+};
+
+// ---- shared-memory layout (same arithmetic on host and device) ------------------
+struct Layout {
+  uint32_t tiles, ptile, bias, colinfo, bins_w, acc, bars, misc, total;
+};
+
+template <int HD, int NS, int NTEN, int NPT>
+__host__ __device__ inline Layout make_layout(int bins_pad, int heads, int acc_in_smem) {
+  constexpr uint32_t tile_bytes = kRows * HD * 2;
+  Layout L;
+  L.tiles = 0;
+  L.ptile = L.tiles + NS * NTEN * tile_bytes;                 // P (and dS) tiles, 32 KB each
+  L.bias = L.ptile + NPT * 32768;
+  L.colinfo = L.bias + ((NS * bins_pad * 4 + 15) & ~15);
+  L.bins_w = L.colinfo + 2 * kRows * 4;
+  L.acc = L.bins_w + 4 * bins_pad * 4;
+  L.bars = (L.acc + (acc_in_smem ? heads * bins_pad * 4 : 0) + 7) & ~7u;
+  L.misc = L.bars + 8 * 32;
+  L.total = L.misc + 16;
+  return L;
+}
+
+// Rows of the 128-row tile are windows g = row / N; inside a window the rows
+// follow the sub-boxes in order (y segment, x segment), each row-major.
+struct SubBox {
+  int y, x, rows, cols, map_id, row_off;
+};
+
+__device__ inline void window_coords(const Geo& g, long long win, int& b, int& wy, int& wx) {
+  const long long per_b = (long long)g.nWy * g.nWx;
+  b = (int)(win / per_b);
+  const int r = (int)(win - (long long)b * per_b);
+  wy = r / g.nWx;
+  wx = r - wy * g.nWx;
+}
+
+// Sub-boxes of window (wy, wx): source start, size, box-shape id, first row.
+__device__ inline int plan_window(const Geo& g, int wy, int wx, SubBox* sb) {
+  const bool wrap_y = g.sh > 0 && wy == g.nWy - 1;
+  const bool wrap_x = g.sw > 0 && wx == g.nWx - 1;
+  int ys[2], yl[2], yk[2], xs[2], xl[2], xk[2];
+  const int ny = wrap_y ? 2 : 1, nx = wrap_x ? 2 : 1;
+  if (wrap_y) {
+    ys[0] = 0; yl[0] = g.wh - g.sh; yk[0] = 1;
+    ys[1] = g.wh - g.sh; yl[1] = g.sh; yk[1] = 2;
+  } else {
+    ys[0] = 0; yl[0] = g.wh; yk[0] = 0;
+  }
+  if (wrap_x) {
+    xs[0] = 0; xl[0] = g.ww - g.sw; xk[0] = 1;
+    xs[1] = g.ww - g.sw; xl[1] = g.sw; xk[1] = 2;
+  } else {
+    xs[0] = 0; xl[0] = g.ww; xk[0] = 0;
+  }
+  int n = 0, off = 0;
+  for (int a = 0; a < ny; ++a)
+    for (int c = 0; c < nx; ++c) {
+      sb[n].y = (wy * g.wh + ys[a] + g.sh) % g.Hp;
+      sb[n].x = (wx * g.ww + xs[c] + g.sw) % g.Wp;
+      sb[n].rows = yl[a];
+      sb[n].cols = xl[c];
+      sb[n].map_id = yk[a] * 3 + xk[c];
+      sb[n].row_off = off;
+      off += yl[a] * xl[c];
+      ++n;
+    }
+  return n;
+}
+
+// Slot coordinates (iy, ix) of row r (0..N-1) of window (wy, wx) in sub-box order.
+__device__ inline void row_slot(const Geo& g, int wy, int wx, int r, int& iy, int& ix) {
+  const bool wrap_y = g.sh > 0 && wy == g.nWy - 1;
+  const bool wrap_x = g.sw > 0 && wx == g.nWx - 1;
+  const int h0 = wrap_y ? g.wh - g.sh : g.wh;
+  const int w0 = wrap_x ? g.ww - g.sw : g.ww;
+  const int top = h0 * g.ww;
+  const int yseg = r >= top;
+  const int rr = yseg ? r - top : r;
+  const int yh = yseg ? g.wh - h0 : h0;
+  const int xseg = rr >= yh * w0;
+  const int r2 = xseg ? rr - yh * w0 : rr;
+  const int wseg = xseg ? g.ww - w0 : w0;
+  const int ly = r2 / wseg;
+  iy = (yseg ? h0 : 0) + ly;
+  ix = (xseg ? w0 : 0) + (r2 - ly * wseg);
+}
+
+// Everything the softmax warpgroup needs to know about its own row.
+struct RowInfo {
+  bool valid;
+  int label;        // shift region 0..8
+  int bias_base;    // (iy + wh - 1)(2 ww - 1) + ix + ww - 1
+  int key_off;      // iy (2 ww - 1) + ix : subtract from a query's base to index the table
+  long long token;  // (b H + y) W + x
+};
+
+__device__ inline RowInfo row_info(const Geo& g, long long win, int r) {
+  RowInfo ri;
+  ri.valid = false;
+  ri.label = 15;
+  ri.bias_base = 0;
+  ri.key_off = 0;
+  ri.token = 0;
+  if (win >= g.n_win) return ri;
+  int b, wy, wx, iy, ix;
+  window_coords(g, win, b, wy, wx);
+  row_slot(g, wy, wx, r, iy, ix);
+  const int yr = wy * g.wh + iy, xr = wx * g.ww + ix;
+  const int y = (yr + g.sh) % g.Hp, x = (xr + g.sw) % g.Wp;
+  ri.valid = y < g.H && x < g.W;
+  ri.label = 3 * region_1d(yr, g.Hp, g.wh, g.sh) + region_1d(xr, g.Wp, g.ww, g.sw);
+  ri.bias_base = (iy + g.wh - 1) * (2 * g.ww - 1) + ix + g.ww - 1;
+  ri.key_off = iy * (2 * g.ww - 1) + ix;
+  ri.token = ((long long)b * g.H + y) * g.W + x;
+  return ri;
+}
+
+// Packed per-key info: low 16 bits key offset into the bias table, bits 16-19
+// region label, or 15 for a pad key (never equal to a query's label).
+__device__ inline uint32_t key_word(const RowInfo& ri) {
+  return (uint32_t)ri.key_off | ((uint32_t)(ri.valid ? ri.label : 15) << 16);
+}
+
+// Producer: one elected thread issues every TMA copy of tile `t` into `stage`.
+template <int HD, int NTEN>
+__device__ inline void issue_tile_loads(const FastParams& p, long long t, uint8_t* tiles,
+                                        float* bias_dst, uint64_t* full) {
+  const Geo& g = p.g;
+  const int G = kRows / g.N;
+  const long long group = t / g.heads;
+  const int h = (int)(t - group * g.heads);
+  constexpr uint32_t row_bytes = HD * 2;
+  constexpr uint32_t tile_bytes = kRows * row_bytes;
+  for (int gw = 0; gw < G; ++gw) {
+    const long long win = group * G + gw;
+    const uint32_t row0 = gw * g.N;
+    if (win < g.n_win) {
+      int b, wy, wx;
+      window_coords(g, win, b, wy, wx);
+      SubBox sb[4];
+      const int n = plan_window(g, wy, wx, sb);
+      for (int i = 0; i < n; ++i)
+        for (int tt = 0; tt < NTEN; ++tt)
+          tma_load_5d(tiles + tt * tile_bytes + (row0 + sb[i].row_off) * row_bytes,
+                      &p.maps[tt][sb[i].map_id], full, 0, h, sb[i].x, sb[i].y, b);
+    } else {
+      // No such window: a box wholly above the grid reads zeros and keeps the
+      // transaction count uniform.
+      for (int tt = 0; tt < NTEN; ++tt)
+        tma_load_5d(tiles + tt * tile_bytes + row0 * row_bytes, &p.maps[tt][0], full, 0, h, 0,
+                    -g.wh, 0);
+    }
+  }
+  bulk_load(bias_dst, p.bias_t + (size_t)h * p.bins_pad, p.bins_pad * 4, full);
+}
+
+// K-major operand, rows of HD bf16 (128-byte swizzle for HD = 64, 64-byte for 32),
+// advanced by k16 steps of 16 elements along K.
+template <int HD>
+__device__ inline uint64_t desc_kmajor_tile(uint32_t base, int k16) {
+  constexpr uint32_t row_bytes = HD * 2;
+  constexpr uint32_t sw = HD == 64 ? kSwizzle128 : kSwizzle64;
+  return smem_desc(base + k16 * 32, 16, 8 * row_bytes, sw);
+}
+// MN-major operand (the HD columns are N), K = tile rows, 16 rows per step.
+template <int HD>
+__device__ inline uint64_t desc_mnmajor_tile(uint32_t base, int k16) {
+  constexpr uint32_t row_bytes = HD * 2;
+  constexpr uint32_t sw = HD == 64 ? kSwizzle128 : kSwizzle64;
+  return smem_desc(base + k16 * 16 * row_bytes, 8 * row_bytes, 8 * row_bytes, sw);
+}
+// P / dS tile: 128 rows x 128 columns bf16 as two 16 KB regions of 64 columns,
+// 128-byte swizzle. As K-major A (M = rows, K = columns):
+__device__ inline uint64_t desc_p_kmajor(uint32_t base, int k16) {
+  return smem_desc(base + (k16 >> 2) * 16384 + (k16 & 3) * 32, 16, 1024, kSwizzle128);
+}
+// As MN-major A of the transpose (M = columns, K = rows): region stride 16 KB
+// between the two 64-column atoms, 8-row groups 1 KB apart.
+__device__ inline uint64_t desc_p_mnmajor(uint32_t base, int k16) {
+  return smem_desc(base + k16 * 2048, 16384, 1024, kSwizzle128);
+}
+
+// Writes this thread's row of a P-style tile: columns [col0, col0 + NCOL) from
+// `vals` (already scaled), rounded to bf16, 128-byte swizzled.
+template <int NCOL>
+__device__ inline void store_p_row(uint32_t base, int row, int col0, const float* vals) {
+#pragma unroll
+  for (int c = 0; c < NCOL / 8; ++c) {
+    const int col = col0 + c * 8;
+    const uint32_t addr = base + (col >> 6) * 16384 + row * 128 + ((((col >> 3) & 7) ^ (row & 7)) << 4);
+    st_shared_v4(addr, pack_bf16(vals[c * 8 + 0], vals[c * 8 + 1]),
+                 pack_bf16(vals[c * 8 + 2], vals[c * 8 + 3]),
+                 pack_bf16(vals[c * 8 + 4], vals[c * 8 + 5]),
+                 pack_bf16(vals[c * 8 + 6], vals[c * 8 + 7]));
+  }
+}
+
+template <int HD>
+__device__ inline void store_row_bf16(void* dst, const float* v, float mul) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int c = 0; c < HD / 8; ++c)
+    st_global_v4(d + c, pack_bf16(v[c * 8 + 0] * mul, v[c * 8 + 1] * mul),
+                 pack_bf16(v[c * 8 + 2] * mul, v[c * 8 + 3] * mul),
+                 pack_bf16(v[c * 8 + 4] * mul, v[c * 8 + 5] * mul),
+                 pack_bf16(v[c * 8 + 6] * mul, v[c * 8 + 7] * mul));
+}
+
+template <int NCOL>
+__device__ inline void tmem_load_cols(uint32_t taddr, float* v) {
+#pragma unroll
+  for (int c = 0; c < NCOL / 32; ++c) tmem_ld32(taddr + c * 32, v + c * 32);
+}
+
+// ================================================================================
+// Forward
+// ================================================================================
+constexpr int kFwdStages = 3;
+constexpr int kFwdSlots = 2;   // TMEM slots of 128 columns (S, then O in its first HD)
+
+template <int HD, int N>
+__global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FastParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  constexpr int NS = kFwdStages, NT = kFwdSlots, G = kRows / N;
+  constexpr uint32_t tile_bytes = kRows * HD * 2;
+  const Geo& g = p.g;
+  const Layout L = make_layout<HD, NS, 3, NT>(p.bins_pad, g.heads, 0);
+  uint8_t* tiles = smem + L.tiles;
+  uint8_t* ptile = smem + L.ptile;
+  float* bias = (float*)(smem + L.bias);
+  uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
+  uint64_t* bars = (uint64_t*)(smem + L.bars);
+  uint64_t* full = bars;
+  uint64_t* empty = full + NS;
+  uint64_t* s_full = empty + NS;
+  uint64_t* p_full = s_full + NT;
+  uint64_t* o_full = p_full + NT;
+  uint64_t* t_empty = o_full + NT;
+  uint64_t* drain = t_empty + NT;
+  uint64_t* never = drain + 1;
+  uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
+  volatile int* abort = (volatile int*)(smem + L.misc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < NT; ++i) {
+      mbar_init(&s_full[i], 1); mbar_init(&p_full[i], kWg);
+      mbar_init(&o_full[i], 1); mbar_init(&t_empty[i], kWg);
+    }
+    mbar_init(drain, 1);
+    mbar_init(never, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarp && lane == 0)
+    for (int tt = 0; tt < 3; ++tt)
+      for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
+  // P tiles start at zero: rows never write the columns of other windows.
+  for (uint32_t i = threadIdx.x; i < NT * 32768 / 16; i += kThreads)
+    reinterpret_cast<uint4*>(ptile)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async();
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, NT * 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      long long k = 0;
+      for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
+        const int s = (int)(k % NS);
+        const uint32_t ph = (uint32_t)((k / NS) & 1);
+        if (!mbar_wait(&empty[s], ph ^ 1, abort, p.status, kWaitLimitNs)) break;
+        mbar_arrive_expect_tx(&full[s], 3 * tile_bytes + p.bins_pad * 4);
+        issue_tile_loads<HD, 3>(p, t, tiles + s * 3 * tile_bytes, bias + s * p.bins_pad, &full[s]);
+      }
+      if (*abort) {  // let copies already in flight land before the CTA leaves
+        const long long first = k > NS ? k - NS : 0;
+        for (long long j = first; j < k; ++j)
+          mbar_drain(&full[j % NS], (uint32_t)((j / NS) & 1), kTestLimitNs * 100);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16(kRows, HD, 0, 1);
+      long long k = 0;
+      for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
+        const int s = (int)(k % NS), sl = (int)(k % NT);
+        const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
+        if (!mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs)) break;
+        if (!mbar_wait(&t_empty[sl], pht ^ 1, abort, p.status, kWaitLimitNs)) break;
+        tc_fence_after();
+        const uint32_t q_s = smem_u32(tiles + (s * 3 + 0) * tile_bytes);
+        const uint32_t k_s = smem_u32(tiles + (s * 3 + 1) * tile_bytes);
+        const uint32_t v_s = smem_u32(tiles + (s * 3 + 2) * tile_bytes);
+        const uint32_t d = tmem + sl * 128;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          umma_ss(d, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk), idesc_s, kk);
+        umma_commit(&s_full[sl]);
+        if (!mbar_wait(&p_full[sl], pht, abort, p.status, kWaitLimitNs)) break;
+        tc_fence_after();
+        const uint32_t p_s = smem_u32(ptile + sl * 32768);
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          umma_ss(d, desc_p_kmajor(p_s, kk), desc_mnmajor_tile<HD>(v_s, kk), idesc_o, kk);
+        umma_commit(&o_full[sl]);
+        umma_commit(&empty[s]);
+      }
+      if (*abort) {
+        umma_commit(drain);
+        mbar_drain(drain, 0, kTestLimitNs * 100);
+      }
+    }
+  } else {
+    // Softmax / epilogue warpgroup: thread = tile row = TMEM lane.
+    const int row = threadIdx.x;
+    const int gw = row / N;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    long long k = 0;
+    for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
+      const int s = (int)(k % NS), sl = (int)(k % NT);
+      const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
+      const long long group = t / g.heads;
+      const int h = (int)(t - group * g.heads);
+      const RowInfo me = row_info(g, group * G + gw, row - gw * N);
+      uint32_t* ci = colinfo + (k & 1) * kRows;
+      ci[row] = key_word(me);
+      if (named_sync_or(1, kWg, *abort)) break;
+      if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
+      mbar_wait(&s_full[sl], pht, abort, p.status, kWaitLimitNs);
+      mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
+      tc_fence_after();
+      float x[N];
+      tmem_load_cols<N>(tmem + lane_base + sl * 128 + gw * N, x);
+      tmem_wait_ld();
+      const float* brow = bias + s * p.bins_pad;
+      const uint32_t* cw = ci + gw * N;
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const uint32_t w = cw[j];
+        const bool ok = (int)(w >> 16) == me.label;
+        x[j] = ok ? fmaf(x[j], p.scale_log2, brow[me.bias_base - (int)(w & 0xFFFF)]) : -INFINITY;
+        m = fmaxf(m, x[j]);
+      }
+      float l = 0.f;
+      if (me.valid) {
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          x[j] = ex2(x[j] - m);
+          l += x[j];
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < N; ++j) x[j] = 0.f;
+        l = 1.f;
+      }
+      store_p_row<N>(smem_u32(ptile + sl * 32768), row, gw * N, x);
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(&p_full[sl]);
+      mbar_wait(&o_full[sl], pht, abort, p.status, kWaitLimitNs);
+      tc_fence_after();
+      float o[HD];
+      tmem_load_cols<HD>(tmem + lane_base + sl * 128, o);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&t_empty[sl]);
+      if (me.valid) {
+        const float inv = 1.f / l;
+        store_row_bf16<HD>((__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD, o, inv);
+        if (p.lse) p.lse[me.token * g.heads + h] = (m + __log2f(l)) * 0.69314718055994531f;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, NT * 128);
+  }
+}
+
+// ================================================================================
+// Backward
+// ================================================================================
+constexpr int kBwdStages = 2;
+constexpr int kBwdSlots = 2;   // TMEM slots of 256 columns: S | dP, then dV | dQ | dK
+
+template <int HD, int N>
+__global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ FastParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  constexpr int NS = kBwdStages, NT = kBwdSlots, G = kRows / N;
+  constexpr uint32_t tile_bytes = kRows * HD * 2;
+  const Geo& g = p.g;
+  const Layout L = make_layout<HD, NS, 4, 2>(p.bins_pad, g.heads, p.acc_in_smem);
+  uint8_t* tiles = smem + L.tiles;
+  uint8_t* ptile = smem + L.ptile;            // P
+  uint8_t* dstile = ptile + 32768;            // dS * scale
+  float* bias = (float*)(smem + L.bias);
+  uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
+  float* bins_w = (float*)(smem + L.bins_w);  // [4 warps][bins_pad]
+  float* acc = (float*)(smem + L.acc);        // [heads][bins_pad] when acc_in_smem
+  uint64_t* bars = (uint64_t*)(smem + L.bars);
+  uint64_t* full = bars;
+  uint64_t* empty = full + NS;
+  uint64_t* sdp_full = empty + NS;
+  uint64_t* pds_full = sdp_full + NT;
+  uint64_t* grad_full = pds_full + NT;
+  uint64_t* t_empty = grad_full + NT;
+  uint64_t* drain = t_empty + NT;
+  uint64_t* never = drain + 1;
+  uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
+  volatile int* abort = (volatile int*)(smem + L.misc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bp = p.bins_pad;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < NT; ++i) {
+      mbar_init(&sdp_full[i], 1); mbar_init(&pds_full[i], kWg);
+      mbar_init(&grad_full[i], 1); mbar_init(&t_empty[i], kWg);
+    }
+    mbar_init(drain, 1);
+    mbar_init(never, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarp && lane == 0)
+    for (int tt = 0; tt < 4; ++tt)
+      for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
+  for (uint32_t i = threadIdx.x; i < 2 * 32768 / 16; i += kThreads)
+    reinterpret_cast<uint4*>(ptile)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = threadIdx.x; i < 4 * bp; i += kThreads) bins_w[i] = 0.f;
+  if (p.acc_in_smem)
+    for (int i = threadIdx.x; i < g.heads * bp; i += kThreads) acc[i] = 0.f;
+  fence_proxy_async();
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, NT * 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      long long k = 0;
+      for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
+        const int s = (int)(k % NS);
+        const uint32_t ph = (uint32_t)((k / NS) & 1);
+        if (!mbar_wait(&empty[s], ph ^ 1, abort, p.status, kWaitLimitNs)) break;
+        mbar_arrive_expect_tx(&full[s], 4 * tile_bytes + bp * 4);
+        issue_tile_loads<HD, 4>(p, t, tiles + s * 4 * tile_bytes, bias + s * bp, &full[s]);
+      }
+      if (*abort) {
+        const long long first = k > NS ? k - NS : 0;
+        for (long long j = first; j < k; ++j)
+          mbar_drain(&full[j % NS], (uint32_t)((j / NS) & 1), kTestLimitNs * 100);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);      // S, dP
+      constexpr uint32_t idesc_t = idesc_bf16(kRows, HD, 1, 1);         // dV, dK: A = X^T
+      constexpr uint32_t idesc_q = idesc_bf16(kRows, HD, 0, 1);         // dQ
+      long long k = 0;
+      for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
+        const int s = (int)(k % NS), sl = (int)(k % NT);
+        const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
+        if (!mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs)) break;
+        if (!mbar_wait(&t_empty[sl], pht ^ 1, abort, p.status, kWaitLimitNs)) break;
+        tc_fence_after();
+        const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
+        const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
+        const uint32_t v_s = smem_u32(tiles + (s * 4 + 2) * tile_bytes);
+        const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
+        const uint32_t d = tmem + sl * 256;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          umma_ss(d, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk), idesc_s, kk);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          umma_ss(d + 128, desc_kmajor_tile<HD>(do_s, kk), desc_kmajor_tile<HD>(v_s, kk), idesc_s,
+                  kk);
+        umma_commit(&sdp_full[sl]);
+        if (!mbar_wait(&pds_full[sl], pht, abort, p.status, kWaitLimitNs)) break;
+        tc_fence_after();
+        const uint32_t p_s = smem_u32(ptile), ds_s = smem_u32(dstile);
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)  // dV = P^T dO
+          umma_ss(d + 0, desc_p_mnmajor(p_s, kk), desc_mnmajor_tile<HD>(do_s, kk), idesc_t, kk);
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)  // dQ = dS K
+          umma_ss(d + 64, desc_p_kmajor(ds_s, kk), desc_mnmajor_tile<HD>(k_s, kk), idesc_q, kk);
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)  // dK = dS^T Q
+          umma_ss(d + 128, desc_p_mnmajor(ds_s, kk), desc_mnmajor_tile<HD>(q_s, kk), idesc_t, kk);
+        umma_commit(&grad_full[sl]);
+        umma_commit(&empty[s]);
+      }
+      if (*abort) {
+        umma_commit(drain);
+        mbar_drain(drain, 0, kTestLimitNs * 100);
+      }
+    }
+  } else {
+    const int row = threadIdx.x;
+    const int gw = row / N;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float dscale = p.scale_log2 * (1.0f / kLog2e);  // head_dim^-1/2
+    float* my_bins = bins_w + warp * bp;
+    long long k = 0;
+    for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
+      const int s = (int)(k % NS), sl = (int)(k % NT);
+      const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
+      const long long group = t / g.heads;
+      const int h = (int)(t - group * g.heads);
+      const RowInfo me = row_info(g, group * G + gw, row - gw * N);
+      uint32_t* ci = colinfo + (k & 1) * kRows;
+      ci[row] = key_word(me);
+      if (named_sync_or(1, kWg, *abort)) break;
+      if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
+      mbar_wait(&sdp_full[sl], pht, abort, p.status, kWaitLimitNs);
+      mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
+      tc_fence_after();
+      float x[N], dp[N];
+      tmem_load_cols<N>(tmem + lane_base + sl * 256 + gw * N, x);
+      tmem_load_cols<N>(tmem + lane_base + sl * 256 + 128 + gw * N, dp);
+      tmem_wait_ld();
+      const float* brow = bias + s * bp;
+      const uint32_t* cw = ci + gw * N;
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        const uint32_t w = cw[j];
+        const bool ok = (int)(w >> 16) == me.label;
+        x[j] = ok ? fmaf(x[j], p.scale_log2, brow[me.bias_base - (int)(w & 0xFFFF)]) : -INFINITY;
+        m = fmaxf(m, x[j]);
+      }
+      if (me.valid) {
+        float l = 0.f;
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          x[j] = ex2(x[j] - m);
+          l += x[j];
+        }
+        const float inv = 1.f / l;
+        float D = 0.f;
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          x[j] *= inv;
+          D = fmaf(x[j], dp[j], D);
+        }
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          const float ds = x[j] * (dp[j] - D);
+          const uint32_t w = cw[j];
+          if ((int)(w >> 16) == me.label) {
+            float* bin = my_bins + me.bias_base - (int)(w & 0xFFFF);
+            *bin += ds;
+          }
+          dp[j] = ds * dscale;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < N; ++j) x[j] = dp[j] = 0.f;
+      }
+      store_p_row<N>(smem_u32(ptile), row, gw * N, x);
+      store_p_row<N>(smem_u32(dstile), row, gw * N, dp);
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(&pds_full[sl]);
+      // Fold the four warps' bias-gradient bins of this tile, in warp order.
+      named_sync(2, kWg);
+      for (int b = row; b < g.bins; b += kWg) {
+        const float v4 = bins_w[b] + bins_w[bp + b] + bins_w[2 * bp + b] + bins_w[3 * bp + b];
+        bins_w[b] = bins_w[bp + b] = bins_w[2 * bp + b] = bins_w[3 * bp + b] = 0.f;
+        if (p.acc_in_smem)
+          acc[h * bp + b] += v4;
+        else
+          p.partial[(group * g.heads + h) * bp + b] = v4;
+      }
+      mbar_wait(&grad_full[sl], pht, abort, p.status, kWaitLimitNs);
+      tc_fence_after();
+      float o[HD];
+      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 0, o);      // dV
+      tmem_wait_ld();
+      if (me.valid) store_row_bf16<HD>((__nv_bfloat16*)p.out2 + (me.token * g.heads + h) * HD, o, 1.f);
+      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 64, o);     // dQ
+      tmem_wait_ld();
+      if (me.valid) store_row_bf16<HD>((__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD, o, 1.f);
+      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 128, o);    // dK
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&t_empty[sl]);
+      if (me.valid) store_row_bf16<HD>((__nv_bfloat16*)p.out1 + (me.token * g.heads + h) * HD, o, 1.f);
+    }
+    if (p.acc_in_smem) {
+      named_sync(2, kWg);
+      for (int i = row; i < g.heads * bp; i += kWg) p.partial[(long long)blockIdx.x * g.heads * bp + i] = acc[i];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, NT * 256);
+  }
+}
+
+// Bias table transposed to [heads][bins_pad] and scaled by log2(e).
+__global__ void bias_prep_kernel(const float* __restrict__ table, int bins, int heads,
+                                 int bins_pad, float* __restrict__ out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= heads * bins_pad) return;
+  const int h = i / bins_pad, b = i - h * bins_pad;
+  out[i] = b < bins ? table[b * heads + h] * kLog2e : 0.f;
+}
+
+// ================================================================================
+// Host side
+// ================================================================================
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+
+int box_len(int kind, int w, int s) { return kind == 0 ? w : (kind == 1 ? w - s : s); }
+
+// The 5-D map [hd, heads, W, H, B] of one tensor with box [hd, 1, bx, by, 1].
+bool encode_map(CUtensorMap* m, const void* base, const Geo& g, int by, int bx) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[5] = {(cuuint64_t)g.hd, (cuuint64_t)g.heads, (cuuint64_t)g.W,
+                              (cuuint64_t)g.H, (cuuint64_t)g.B};
+  const cuuint64_t es = 2;
+  const cuuint64_t strides[4] = {g.hd * es, (cuuint64_t)g.heads * g.hd * es,
+                                 (cuuint64_t)g.W * g.heads * g.hd * es,
+                                 (cuuint64_t)g.H * g.W * g.heads * g.hd * es};
+  const cuuint32_t box[5] = {(cuuint32_t)g.hd, 1, (cuuint32_t)bx, (cuuint32_t)by, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUtensorMapSwizzle sw =
+      g.hd == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_maps(FastParams& p, int which, const void* base) {
+  const Geo& g = p.g;
+  for (int ky = 0; ky < 3; ++ky)
+    for (int kx = 0; kx < 3; ++kx) {
+      int by = box_len(ky, g.wh, g.sh), bx = box_len(kx, g.ww, g.sw);
+      if (by <= 0) by = g.wh;  // shape unused when the axis has no shift
+      if (bx <= 0) bx = g.ww;
+      if (!encode_map(&p.maps[which][ky * 3 + kx], base, g, by, bx)) return false;
+    }
+  return true;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+constexpr size_t kSmemLimit = 227 * 1024;
+
+
+template <int HD>
+size_t fwd_smem(const Geo& g) {
+  return make_layout<HD, kFwdStages, 3, kFwdSlots>(bins_padded(g.bins), g.heads, 0).total + 1024;
+}
+template <int HD>
+size_t bwd_smem(const Geo& g, int acc_in_smem) {
+  return make_layout<HD, kBwdStages, 4, 2>(bins_padded(g.bins), g.heads, acc_in_smem).total + 1024;
+}
+
+bool smem_ok(const Geo& g) {
+  const size_t f = g.hd == 64 ? fwd_smem<64>(g) : fwd_smem<32>(g);
+  const size_t b = g.hd == 64 ? bwd_smem<64>(g, 0) : bwd_smem<32>(g, 0);
+  return f <= kSmemLimit && b <= kSmemLimit;
+}
+
+int acc_mode(const Geo& g) {
+  const size_t b = g.hd == 64 ? bwd_smem<64>(g, 1) : bwd_smem<32>(g, 1);
+  return b <= kSmemLimit ? 1 : 0;
+}
+
+void fill_common(FastParams& p, const Geo& g, const float* bias_t, int* status, int flags) {
+  memset(&p, 0, sizeof(p));
+  p.g = g;
+  const int G = kRows / g.N;
+  p.n_groups = (g.n_win + G - 1) / G;
+  p.n_tiles = p.n_groups * g.heads;
+  p.bins_pad = bins_padded(g.bins);
+  p.scale_log2 = kLog2e / sqrtf((float)g.hd);
+  p.bias_t = bias_t;
+  p.status = status;
+  p.test_timeout = (flags & SWIN_FLAG_TEST_TIMEOUT) ? 1 : 0;
+}
+
+template <typename K>
+cudaError_t launch(K kernel, const FastParams& p, size_t smem, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
+  kernel<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t prep_bias(const Geo& g, const float* table, float* bias_t, cudaStream_t st) {
+  const int n = g.heads * bins_padded(g.bins);
+  bias_prep_kernel<<<(n + 255) / 256, 256, 0, st>>>(table, g.bins, g.heads, bins_padded(g.bins),
+                                                    bias_t);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool fast_supported(const Geo& g, int dtype) {
+  if (dtype != SWIN_DTYPE_BF16) return false;
+  if (g.hd != 64 && g.hd != 32) return false;
+  if (g.N != 64 && g.N != 32) return false;
+  // Every sub-box must be a whole number of 8-row swizzle atoms.
+  const int ylen[3] = {g.wh, g.wh - g.sh, g.sh};
+  const int xlen[3] = {g.ww, g.ww - g.sw, g.sw};
+  for (int a = 0; a < 3; ++a)
+    for (int c = 0; c < 3; ++c) {
+      if ((a > 0 && g.sh == 0) || (c > 0 && g.sw == 0)) continue;
+      if ((ylen[a] * xlen[c]) % 8) return false;
+    }
+  if (g.bins > 0xFFFF) return false;
+  return smem_ok(g);
+}
+
+size_t fast_workspace(const Geo& g) {
+  const int bp = bins_padded(g.bins);
+  const int G = kRows / g.N;
+  const long long groups = (g.n_win + G - 1) / G;
+  const size_t per_tile = (size_t)groups * g.heads * bp * 4;
+  const size_t per_cta = (size_t)1024 * g.heads * bp * 4;  // any grid up to 1024 CTAs
+  return kWsHeader + align256((size_t)g.heads * bp * 4) + align256(per_tile > per_cta ? per_tile : per_cta);
+}
+
+cudaError_t fast_forward(const Geo& g, const void* q, const void* k, const void* v,
+                         const float* table, void* out, float* lse, void* ws, int flags,
+                         cudaStream_t st) {
+  float* bias_t = (float*)((char*)ws + kWsHeader);
+  static thread_local FastParams p;
+  fill_common(p, g, bias_t, (int*)ws, flags);
+  p.out0 = out;
+  p.lse = lse;
+  if (!encode_maps(p, 0, q) || !encode_maps(p, 1, k) || !encode_maps(p, 2, v))
+    return cudaErrorInvalidValue;
+  cudaError_t e = prep_bias(g, table, bias_t, st);
+  if (e != cudaSuccess) return e;
+  if (g.hd == 64)
+    return g.N == 64 ? launch(fwd_kernel<64, 64>, p, fwd_smem<64>(g), st)
+                     : launch(fwd_kernel<64, 32>, p, fwd_smem<64>(g), st);
+  return g.N == 64 ? launch(fwd_kernel<32, 64>, p, fwd_smem<32>(g), st)
+                   : launch(fwd_kernel<32, 32>, p, fwd_smem<32>(g), st);
+}
+
+cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void* v,
+                          const float* table, const void* dout, void* dq, void* dk, void* dv,
+                          float* dtable, void* ws, int flags, cudaStream_t st) {
+  float* bias_t = (float*)((char*)ws + kWsHeader);
+  float* partial = (float*)((char*)ws + kWsHeader + align256((size_t)g.heads * bins_padded(g.bins) * 4));
+  static thread_local FastParams p;
+  fill_common(p, g, bias_t, (int*)ws, flags);
+  p.out0 = dq;
+  p.out1 = dk;
+  p.out2 = dv;
+  p.partial = partial;
+  p.acc_in_smem = acc_mode(g);
+  if (!encode_maps(p, 0, q) || !encode_maps(p, 1, k) || !encode_maps(p, 2, v) ||
+      !encode_maps(p, 3, dout))
+    return cudaErrorInvalidValue;
+  cudaError_t e = prep_bias(g, table, bias_t, st);
+  if (e != cudaSuccess) return e;
+  const size_t smem = g.hd == 64 ? bwd_smem<64>(g, p.acc_in_smem) : bwd_smem<32>(g, p.acc_in_smem);
+  if (g.hd == 64)
+    e = g.N == 64 ? launch(bwd_kernel<64, 64>, p, smem, st) : launch(bwd_kernel<64, 32>, p, smem, st);
+  else
+    e = g.N == 64 ? launch(bwd_kernel<32, 64>, p, smem, st) : launch(bwd_kernel<32, 32>, p, smem, st);
+  if (e != cudaSuccess) return e;
+  const long long grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
+  return dbias_reduce(g, partial, p.acc_in_smem ? grid : p.n_groups, dtable, st);
+}
+
+}  // namespace swin

@@ -1,0 +1,97 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function that
+include/swin_wattn.h declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from shifted_window_attention_pad_b200 import WORKLOADS, binding as sb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(swin_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    from shifted_window_attention_pad_b200 import build
+    build.build()
+    return sb.lib()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("swin_wattn_fwd", "swin_wattn_bwd", "swin_wattn_workspace_size",
+              "swin_wattn_index_map", "swin_wattn_strerror"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+        assert ctypes.cast(getattr(L, n), ctypes.c_void_p).value
+
+
+def test_fast_path_covers_the_bf16_window64_workloads(L):
+    expect = {"tiny-16x16-w4": 0, "ragged-90x180-w8": 1, "twelfth-degree-256x544-w8": 1,
+              "downsampled-128x272-w16": 0, "small-patch-2x512x1088-w8": 1}
+    for name, want in expect.items():
+        assert sb.swin_wattn_path(sb.desc_for(WORKLOADS[name])) == want, name
+    d = sb.desc_for(WORKLOADS["twelfth-degree-256x544-w8"], flags=sb.SWIN_FLAG_FORCE_GENERIC)
+    assert sb.swin_wattn_path(d) == 0
+
+
+@pytest.mark.parametrize("field,value", [("shift_h", 8), ("shift_w", -1), ("win_h", 0),
+                                         ("head_dim", 12), ("heads", 0), ("B", 0), ("H", 0),
+                                         ("win_w", 65), ("head_dim", 264)])
+def test_bad_descriptions_are_rejected_on_the_host(L, field, value):
+    d = sb.desc_for(WORKLOADS["twelfth-degree-256x544-w8"])
+    setattr(d, field, value)
+    assert L.swin_wattn_path(ctypes.byref(d)) == -1
+    n = ctypes.c_size_t(0)
+    assert L.swin_wattn_workspace_size(ctypes.byref(d), ctypes.byref(n)) == -1
+
+
+def test_bad_dtype_is_unsupported(L):
+    d = sb.desc_for(WORKLOADS["tiny-16x16-w4"])
+    d.dtype = 7
+    assert L.swin_wattn_path(ctypes.byref(d)) == -2
+
+
+def test_null_and_misaligned_pointers_are_rejected_before_any_cuda_call(L):
+    d = sb.desc_for(WORKLOADS["ragged-90x180-w8"])
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    assert L.swin_wattn_fwd(ctypes.byref(d), None, good, good, good, good, None, good, 1 << 30,
+                            None) == -1
+    assert L.swin_wattn_fwd(ctypes.byref(d), P((1 << 20) + 2), good, good, good, good, None,
+                            good, 1 << 30, None) == -1
+    assert L.swin_wattn_bwd(ctypes.byref(d), good, good, good, good, good, good, good, None,
+                            good, good, 1 << 30, None) == -1
+    # workspace: too small, misaligned
+    assert L.swin_wattn_fwd(ctypes.byref(d), good, good, good, good, good, None, good, 16,
+                            None) == -3
+    assert L.swin_wattn_fwd(ctypes.byref(d), good, good, good, good, good, None, P((1 << 20) + 16),
+                            1 << 30, None) == -3
+    assert L.swin_wattn_index_map(ctypes.byref(d), None, None) == -1
+
+
+def test_workspace_sizes_are_modest(L):
+    for wl in WORKLOADS.values():
+        n = sb.swin_wattn_workspace_size(sb.desc_for(wl))
+        assert 256 <= n < 512 * 2**20, (wl.name, n)
+
+
+def test_strerror_covers_every_status(L):
+    for s in range(-5, 1):
+        assert sb.swin_wattn_strerror(s) != "unknown status"

@@ -1,0 +1,217 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, element by element, plus bit-exact layout checks and
+invariants. Acceptance bar: index and layout work bit-exact; fp32 max relative
+error <= 1e-5 (normwise); bf16 max|gpu - ref| / RMS(ref) <= 2e-2 per tensor."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from shifted_window_attention_pad_b200 import WORKLOADS, binding as sb
+from shifted_window_attention_pad_b200.synth import make_inputs, as_f64
+from shifted_window_attention_pad_b200.workloads import Workload
+
+from gpu_helpers import BF16_TOL, F32_TOL, compare, oracle_shape, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from shifted_window_attention_pad_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+def tol(dtype):
+    return F32_TOL if dtype == "f32" else BF16_TOL
+
+
+# ---------------------------------------------------------------------------
+# Layout stage: bit-exact
+# ---------------------------------------------------------------------------
+SWEEP = [(H, W, w, s) for (H, W) in [(1, 1), (5, 7), (16, 16), (17, 40), (40, 3), (90, 180)]
+         for (w, s) in [(1, 0), (2, 1), (4, 2), (7, 3), (8, 4), (8, 0)]]
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_index_map_bit_exact_on_workload_shapes(name):
+    wl = WORKLOADS[name]
+    d = sb.desc_for(wl)
+    gpu = sb.swin_wattn_index_map(d).cpu().numpy().reshape(wl.B, -1, wl.win * wl.win)
+    ref = oracle.index_map(oracle_shape(d))
+    assert np.array_equal(gpu.astype(np.int64), ref)
+
+
+@pytest.mark.parametrize("H,W,w,s", SWEEP)
+def test_index_map_bit_exact_sweep(H, W, w, s):
+    d = sb.make_desc(2, H, W, w, s, 1, 8, "f32")
+    gpu = sb.swin_wattn_index_map(d).cpu().numpy().reshape(2, -1, w * w)
+    assert np.array_equal(gpu.astype(np.int64), oracle.index_map(oracle_shape(d)))
+
+
+# ---------------------------------------------------------------------------
+# Parity on the five workloads
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["tiny-16x16-w4", "ragged-90x180-w8",
+                                  "twelfth-degree-256x544-w8", "downsampled-128x272-w16"])
+def test_parity_full(name):
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    gpu = run_gpu(d, inp)
+    ref = run_oracle(d, inp)
+    errs = compare(gpu, ref, wl.dtype)
+    print(name, "path", sb.swin_wattn_path(d), errs)
+    assert set(errs) == {"o", "lse", "dq", "dk", "dv", "dT"}
+    for n, e in errs.items():
+        assert e <= tol(wl.dtype), (name, n, e)
+
+
+def test_parity_small_patch_two_heads():
+    """Batch 2 x 512 x 1088, 12 heads: the whole problem runs on the GPU; heads 0
+    and 7 (heads are independent) are checked against the oracle in full."""
+    wl = WORKLOADS["small-patch-2x512x1088-w8"]
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    gpu = run_gpu(d, inp, want_lse=False)
+    for h in (0, 7):
+        sub = {n: inp[n][:, :, :, h:h + 1].contiguous() for n in ("q", "k", "v", "dout")}
+        sub["table"] = inp["table"][:, h:h + 1].contiguous()
+        ds = sb.make_desc(wl.B, wl.H, wl.W, wl.win, wl.shift, 1, wl.head_dim, wl.dtype)
+        ref = run_oracle(ds, sub)
+        g = {n: gpu[n][:, :, :, h:h + 1] for n in ("o", "dq", "dk", "dv")}
+        g["dT"] = gpu["dT"][:, h:h + 1]
+        errs = compare(g, ref, wl.dtype)
+        print("head", h, errs)
+        for n, e in errs.items():
+            assert e <= BF16_TOL, (h, n, e)
+
+
+def test_generic_kernels_bf16_parity():
+    wl = WORKLOADS["ragged-90x180-w8"]
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl, flags=sb.SWIN_FLAG_FORCE_GENERIC)
+    assert sb.swin_wattn_path(d) == 0
+    errs = compare(run_gpu(d, inp), run_oracle(d, inp), "bf16")
+    for n, e in errs.items():
+        assert e <= BF16_TOL, (n, e)
+
+
+# Shapes that exercise the fast path's edges: non-square windows, head_dim 32,
+# a grid smaller than one window, no shift, an odd window count (half-empty
+# tile), batch > 1.
+EDGE = [
+    Workload("edge-a", 2, 20, 28, 8, 4, 3, 64, "bf16", 11),
+    Workload("edge-b", 1, 5, 6, 8, 4, 2, 64, "bf16", 12),
+    Workload("edge-c", 1, 24, 40, 8, 0, 2, 32, "bf16", 13),
+    Workload("edge-d", 3, 9, 17, 8, 4, 1, 32, "bf16", 14),
+]
+
+
+@pytest.mark.parametrize("wl", EDGE, ids=lambda w: w.name)
+def test_fast_path_edges(wl):
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    assert sb.swin_wattn_path(d) == 1
+    errs = compare(run_gpu(d, inp), run_oracle(d, inp), "bf16")
+    print(wl.name, errs)
+    for n, e in errs.items():
+        assert e <= BF16_TOL, (wl.name, n, e)
+
+
+@pytest.mark.parametrize("win,shift", [((4, 8), (2, 4)), ((8, 4), (4, 2)), ((4, 16), (2, 8))])
+def test_fast_path_non_square_windows(win, shift):
+    B, H, W, heads, hd = 1, 18, 30, 2, 64
+    d = sb.make_desc(B, H, W, win, shift, heads, hd, "bf16")
+    wl = Workload("ns", B, H, W, win[0], shift[0], heads, hd, "bf16", 21)
+    inp = make_inputs(wl, shape_override=(B, H, W, heads, hd))
+    nb = (2 * win[0] - 1) * (2 * win[1] - 1)
+    inp["table"] = torch.from_numpy(
+        np.random.Generator(np.random.PCG64(5)).standard_normal((nb, heads)).astype(np.float32) * 0.02)
+    assert sb.swin_wattn_path(d) == 1
+    errs = compare(run_gpu(d, inp), run_oracle(d, inp), "bf16")
+    for n, e in errs.items():
+        assert e <= BF16_TOL, (win, n, e)
+
+
+# ---------------------------------------------------------------------------
+# Exact cases and invariants
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_hand_example_isolated_tokens_exact_on_gpu(dtype):
+    """4x4 grid, 2x2 windows, shift 1: the corner window's four tokens each sit
+    in their own region, so o = v, dq = dk = 0 and dv = dO exactly."""
+    wl = Workload("hand", 1, 4, 4, 2, 1, 3, 8, dtype, 3)
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    gpu = run_gpu(d, inp)
+    for tok in (15, 12, 3, 0):
+        y, x = divmod(tok, 4)
+        assert torch.equal(gpu["o"][0, y, x].cpu(), inp["v"][0, y, x])
+        assert torch.all(gpu["dq"][0, y, x] == 0) and torch.all(gpu["dk"][0, y, x] == 0)
+        assert torch.equal(gpu["dv"][0, y, x].cpu(), inp["dout"][0, y, x])
+
+
+def test_other_region_keys_do_not_reach_a_query_bit_exact():
+    """Seam window of the 1/12-degree shape: change k and v of one token of region
+    A; queries of the other regions in that window keep identical bits."""
+    wl = WORKLOADS["ragged-90x180-w8"]
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    s = oracle_shape(d)
+    m = oracle.index_map(s)[0]
+    lab = oracle.region_labels(s)
+    win = m.shape[0] - 1                       # bottom-right corner window
+    src, labels = m[win], lab[win]
+    tgt = next(i for i in range(len(src)) if src[i] >= 0)
+    others = [src[i] for i in range(len(src)) if src[i] >= 0 and labels[i] != labels[tgt]]
+    same = [src[i] for i in range(len(src)) if src[i] >= 0 and labels[i] == labels[tgt]
+            and i != tgt]
+    assert others and same
+    o1 = run_gpu(d, inp, backward=False)["o"].reshape(-1, wl.heads, wl.head_dim).cpu()
+    inp2 = dict(inp)
+    for n in ("k", "v"):
+        t = inp[n].clone().reshape(-1, wl.heads, wl.head_dim)
+        t[src[tgt]] += 3.0
+        inp2[n] = t.reshape(inp[n].shape)
+    o2 = run_gpu(d, inp2, backward=False)["o"].reshape(-1, wl.heads, wl.head_dim).cpu()
+    assert torch.equal(o1[others], o2[others])
+    assert not torch.equal(o1[same], o2[same])
+
+
+def test_bias_gradient_sums_to_zero_and_backward_is_deterministic():
+    wl = WORKLOADS["twelfth-degree-256x544-w8"]
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    a = run_gpu(d, inp, want_lse=False)
+    b = run_gpu(d, inp, want_lse=False)
+    for n in ("o", "dq", "dk", "dv", "dT"):
+        assert torch.equal(a[n], b[n]), n
+    dT = as_f64(a["dT"])
+    assert np.all(np.abs(dT.sum(axis=0)) <= 1e-3 * np.abs(dT).sum(axis=0) + 1e-6)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait on a barrier that nothing arrives on runs out after ~1 ms: the call
+    reports SWIN_ERR_TIMEOUT through the workspace status word, and the next
+    call on the same context works."""
+    wl = WORKLOADS["ragged-90x180-w8"]
+    inp = make_inputs(wl)
+    dev = "cuda"
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "dout"))
+    T = inp["table"].to(dev)
+    d = sb.desc_for(wl, flags=sb.SWIN_FLAG_TEST_TIMEOUT)
+    ws = sb.new_workspace(d)
+    out = torch.empty_like(q)
+    sb.swin_wattn_fwd(d, q, k, v, T, out, None, ws)
+    assert sb.swin_wattn_poll_status(ws) == sb.SWIN_ERR_TIMEOUT
+    dq, dk, dv, dT = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(T)
+    sb.swin_wattn_bwd(d, q, k, v, T, do, dq, dk, dv, dT, ws)
+    assert sb.swin_wattn_poll_status(ws) == sb.SWIN_ERR_TIMEOUT
+    assert sb.swin_wattn_poll_status(ws) == 0
+    d_ok = sb.desc_for(wl)
+    gpu = run_gpu(d_ok, inp)
+    ref = run_oracle(d_ok, inp)
+    for n, e in compare(gpu, ref, "bf16").items():
+        assert e <= BF16_TOL, (n, e)
