@@ -67,7 +67,7 @@ struct FastParams {
   long long n_groups;             // tiles per head: ceil(n_win / G)
   long long n_tiles;              // n_groups * heads
   int bins_pad;
-  int acc_in_smem;                // bias-gradient accumulation per CTA in shared memory
+  int acc_local;                  // bias-gradient accumulation per CTA in thread-local memory
   float scale_log2;               // head_dim^-1/2 * log2(e)
   const float* bias_t;            // [heads][bins_pad], times log2(e)
   void* out0;                     // forward: out;  backward: dq
@@ -81,20 +81,22 @@ struct FastParams {
 
 // ---- shared-memory layout (same arithmetic on host and device) ------------------
 struct Layout {
-  uint32_t tiles, ptile, bias, colinfo, bins_w, acc, bars, misc, total;
+  uint32_t tiles, ptile, bias, colinfo, bins_w, bars, misc, total;
 };
 
-template <int HD, int NS, int NTEN, int NPT>
-__host__ __device__ inline Layout make_layout(int bins_pad, int heads, int acc_in_smem) {
+// NS stages of NTEN input tiles, then PBYTES of P / dS operand blocks, the
+// bias rows of the stages, the key words, per-warp bias-gradient bins,
+// mbarriers and two words (TMEM base, abort flag).
+template <int HD, int NS, int NTEN, uint32_t PBYTES>
+__host__ __device__ inline Layout make_layout(int bins_pad) {
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   Layout L;
   L.tiles = 0;
-  L.ptile = L.tiles + NS * NTEN * tile_bytes;                 // P (and dS) tiles, 32 KB each
-  L.bias = L.ptile + NPT * 32768;
+  L.ptile = L.tiles + NS * NTEN * tile_bytes;
+  L.bias = L.ptile + PBYTES;
   L.colinfo = L.bias + ((NS * bins_pad * 4 + 15) & ~15);
   L.bins_w = L.colinfo + 2 * kRows * 4;
-  L.acc = L.bins_w + 4 * bins_pad * 4;
-  L.bars = (L.acc + (acc_in_smem ? heads * bins_pad * 4 : 0) + 7) & ~7u;
+  L.bars = (L.bins_w + 4 * bins_pad * 4 + 7) & ~7u;
   L.misc = L.bars + 8 * 32;
   L.total = L.misc + 16;
   return L;
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   constexpr int NS = kFwdStages, NT = kFwdSlots, G = kRows / N;
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   const Geo& g = p.g;
-  const Layout L = make_layout<HD, NS, 3, NT>(p.bins_pad, g.heads, 0);
+  const Layout L = make_layout<HD, NS, 3, NT * 32768>(p.bins_pad);
   uint8_t* tiles = smem + L.tiles;
   uint8_t* ptile = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
@@ -472,24 +474,63 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 // ================================================================================
 // Backward
 // ================================================================================
+// P and scale*dS feed the dV, dQ and dK products. Rounded to bf16 alone they
+// would cost up to 2.5% of the output RMS on the largest gradients, so each is
+// split into bf16 hi + lo parts (x = hi + lo to ~2^-17 relative) and both parts
+// are accumulated in TMEM. The two windows of a tile never mix: each operand is
+// two 64 x 64 blocks (8 KB, 128-byte swizzle, 128-byte rows) plus shared zero
+// blocks Z1, Z2, in this order:
+//   [P0h][P0l][dS0h][Z1][dS1h][dS0l][Z2][dS1l][P1h][P1l]
+// As a K-major A (dQ = dS K: rows = queries, K = keys) the key half 0 of dS is
+// the 16 KB run [dS0 | Z] and the key half 1 is [Z | dS1]. As an MN-major A
+// (dV = P^T dO, dK = dS^T Q: M = keys, K = queries) the second 64-key atom is
+// addressed through the leading byte offset, so the query half 0 reads
+// (X0, Z) and the query half 1 reads (Z, X1) for any X0 < Z < X1.
 constexpr int kBwdStages = 2;
 constexpr int kBwdSlots = 2;   // TMEM slots of 256 columns: S | dP, then dV | dQ | dK
+constexpr uint32_t kBlk = 8192;
+enum { kP0h = 0, kP0l, kS0h, kZ1, kS1h, kS0l, kZ2, kS1l, kP1h, kP1l, kNumBlk };
+constexpr int kAccMax = 64;    // thread-local bias-gradient accumulators
 
-template <int HD, int N>
+__device__ inline uint64_t desc_blk_kmajor(uint32_t base, int blk0, int blk1, int k16) {
+  // keys [0,64) read the run starting at blk0, keys [64,128) the run at blk1
+  const uint32_t start = base + (k16 < 4 ? blk0 : blk1) * kBlk + (k16 & 3) * 32;
+  return smem_desc(start, 16, 1024, kSwizzle128);
+}
+__device__ inline uint64_t desc_blk_mnmajor(uint32_t base, int x0, int z, int x1, int k16) {
+  // query half 0: atoms (x0, z); query half 1: atoms (z, x1)
+  const int first = k16 < 4 ? x0 : z, second = k16 < 4 ? z : x1;
+  const uint32_t start = base + first * kBlk + (k16 & 3) * 2048;
+  return smem_desc(start, (uint32_t)(second - first) * kBlk, 1024, kSwizzle128);
+}
+
+// Row `lr` (0..63) of one 64 x 64 block, from 64 fp32 values.
+__device__ inline void store_blk_row(uint32_t blk, int lr, const float* v) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    st_shared_v4(blk + lr * 128 + ((c ^ (lr & 7)) << 4), pack_bf16(v[c * 8 + 0], v[c * 8 + 1]),
+                 pack_bf16(v[c * 8 + 2], v[c * 8 + 3]), pack_bf16(v[c * 8 + 4], v[c * 8 + 5]),
+                 pack_bf16(v[c * 8 + 6], v[c * 8 + 7]));
+}
+
+__device__ inline float bf16_round(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+template <int HD>
 __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ FastParams p) {
+  constexpr int N = 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   constexpr int NS = kBwdStages, NT = kBwdSlots, G = kRows / N;
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   const Geo& g = p.g;
-  const Layout L = make_layout<HD, NS, 4, 2>(p.bins_pad, g.heads, p.acc_in_smem);
+  const Layout L = make_layout<HD, NS, 4, kNumBlk * kBlk>(p.bins_pad);
   uint8_t* tiles = smem + L.tiles;
-  uint8_t* ptile = smem + L.ptile;            // P
-  uint8_t* dstile = ptile + 32768;            // dS * scale
+  uint8_t* blocks = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
   uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
   float* bins_w = (float*)(smem + L.bins_w);  // [4 warps][bins_pad]
-  float* acc = (float*)(smem + L.acc);        // [heads][bins_pad] when acc_in_smem
   uint64_t* bars = (uint64_t*)(smem + L.bars);
   uint64_t* full = bars;
   uint64_t* empty = full + NS;
@@ -518,11 +559,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   if (warp == kProducerWarp && lane == 0)
     for (int tt = 0; tt < 4; ++tt)
       for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
-  for (uint32_t i = threadIdx.x; i < 2 * 32768 / 16; i += kThreads)
-    reinterpret_cast<uint4*>(ptile)[i] = make_uint4(0, 0, 0, 0);
+  for (uint32_t i = threadIdx.x; i < kBlk / 16; i += kThreads) {
+    reinterpret_cast<uint4*>(blocks + kZ1 * kBlk)[i] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(blocks + kZ2 * kBlk)[i] = make_uint4(0, 0, 0, 0);
+  }
   for (int i = threadIdx.x; i < 4 * bp; i += kThreads) bins_w[i] = 0.f;
-  if (p.acc_in_smem)
-    for (int i = threadIdx.x; i < g.heads * bp; i += kThreads) acc[i] = 0.f;
   fence_proxy_async();
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, NT * 256);
@@ -554,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);      // S, dP
       constexpr uint32_t idesc_t = idesc_bf16(kRows, HD, 1, 1);         // dV, dK: A = X^T
       constexpr uint32_t idesc_q = idesc_bf16(kRows, HD, 0, 1);         // dQ
+      const uint32_t bb = smem_u32(blocks);
       long long k = 0;
       for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
         const int s = (int)(k % NS), sl = (int)(k % NT);
@@ -576,16 +618,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         umma_commit(&sdp_full[sl]);
         if (!mbar_wait(&pds_full[sl], pht, abort, p.status, kWaitLimitNs)) break;
         tc_fence_after();
-        const uint32_t p_s = smem_u32(ptile), ds_s = smem_u32(dstile);
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)  // dV = P^T dO
-          umma_ss(d + 0, desc_p_mnmajor(p_s, kk), desc_mnmajor_tile<HD>(do_s, kk), idesc_t, kk);
+        for (int kk = 0; kk < kRows / 16; ++kk) {  // dV = P^T dO  (hi, then lo)
+          umma_ss(d + 0, desc_blk_mnmajor(bb, kP0h, kZ1, kP1h, kk),
+                  desc_mnmajor_tile<HD>(do_s, kk), idesc_t, kk);
+          umma_ss(d + 0, desc_blk_mnmajor(bb, kP0l, kZ1, kP1l, kk),
+                  desc_mnmajor_tile<HD>(do_s, kk), idesc_t, 1);
+        }
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)  // dQ = dS K
-          umma_ss(d + 64, desc_p_kmajor(ds_s, kk), desc_mnmajor_tile<HD>(k_s, kk), idesc_q, kk);
+        for (int kk = 0; kk < kRows / 16; ++kk) {  // dQ = dS K
+          umma_ss(d + 64, desc_blk_kmajor(bb, kS0h, kZ1, kk), desc_mnmajor_tile<HD>(k_s, kk),
+                  idesc_q, kk);
+          umma_ss(d + 64, desc_blk_kmajor(bb, kS0l, kZ2, kk), desc_mnmajor_tile<HD>(k_s, kk),
+                  idesc_q, 1);
+        }
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)  // dK = dS^T Q
-          umma_ss(d + 128, desc_p_mnmajor(ds_s, kk), desc_mnmajor_tile<HD>(q_s, kk), idesc_t, kk);
+        for (int kk = 0; kk < kRows / 16; ++kk) {  // dK = dS^T Q
+          umma_ss(d + 128, desc_blk_mnmajor(bb, kS0h, kZ1, kS1h, kk),
+                  desc_mnmajor_tile<HD>(q_s, kk), idesc_t, kk);
+          umma_ss(d + 128, desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, kk),
+                  desc_mnmajor_tile<HD>(q_s, kk), idesc_t, 1);
+        }
         umma_commit(&grad_full[sl]);
         umma_commit(&empty[s]);
       }
@@ -596,17 +649,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     }
   } else {
     const int row = threadIdx.x;
-    const int gw = row / N;
+    const int gw = row / N, lr = row - gw * N;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const float dscale = p.scale_log2 * (1.0f / kLog2e);  // head_dim^-1/2
+    const uint32_t bb = smem_u32(blocks);
+    const uint32_t blk_ph = bb + (gw ? kP1h : kP0h) * kBlk, blk_pl = bb + (gw ? kP1l : kP0l) * kBlk;
+    const uint32_t blk_sh = bb + (gw ? kS1h : kS0h) * kBlk, blk_sl = bb + (gw ? kS1l : kS0l) * kBlk;
     float* my_bins = bins_w + warp * bp;
+    const int nb = (g.bins + kWg - 1) / kWg;     // table entries owned by this thread
+    float acc[kAccMax];
+    if (p.acc_local)
+      for (int i = 0; i < kAccMax; ++i) acc[i] = 0.f;
     long long k = 0;
     for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
       const int s = (int)(k % NS), sl = (int)(k % NT);
       const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
       const long long group = t / g.heads;
       const int h = (int)(t - group * g.heads);
-      const RowInfo me = row_info(g, group * G + gw, row - gw * N);
+      const RowInfo me = row_info(g, group * G + gw, lr);
       uint32_t* ci = colinfo + (k & 1) * kRows;
       ci[row] = key_word(me);
       if (named_sync_or(1, kWg, *abort)) break;
@@ -656,18 +716,28 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 #pragma unroll
         for (int j = 0; j < N; ++j) x[j] = dp[j] = 0.f;
       }
-      store_p_row<N>(smem_u32(ptile), row, gw * N, x);
-      store_p_row<N>(smem_u32(dstile), row, gw * N, dp);
+      // hi parts, then the residuals as lo parts
+      store_blk_row(blk_ph, lr, x);
+      store_blk_row(blk_sh, lr, dp);
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        x[j] -= bf16_round(x[j]);
+        dp[j] -= bf16_round(dp[j]);
+      }
+      store_blk_row(blk_pl, lr, x);
+      store_blk_row(blk_sl, lr, dp);
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&pds_full[sl]);
       // Fold the four warps' bias-gradient bins of this tile, in warp order.
       named_sync(2, kWg);
-      for (int b = row; b < g.bins; b += kWg) {
+      for (int i = 0; i < nb; ++i) {
+        const int b = row + i * kWg;
+        if (b >= g.bins) break;
         const float v4 = bins_w[b] + bins_w[bp + b] + bins_w[2 * bp + b] + bins_w[3 * bp + b];
         bins_w[b] = bins_w[bp + b] = bins_w[2 * bp + b] = bins_w[3 * bp + b] = 0.f;
-        if (p.acc_in_smem)
-          acc[h * bp + b] += v4;
+        if (p.acc_local)
+          acc[h * nb + i] += v4;
         else
           p.partial[(group * g.heads + h) * bp + b] = v4;
       }
@@ -686,9 +756,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       mbar_arrive(&t_empty[sl]);
       if (me.valid) store_row_bf16<HD>((__nv_bfloat16*)p.out1 + (me.token * g.heads + h) * HD, o, 1.f);
     }
-    if (p.acc_in_smem) {
-      named_sync(2, kWg);
-      for (int i = row; i < g.heads * bp; i += kWg) p.partial[(long long)blockIdx.x * g.heads * bp + i] = acc[i];
+    if (p.acc_local) {
+      float* dst = p.partial + (long long)blockIdx.x * g.heads * bp;
+      for (int hh = 0; hh < g.heads; ++hh)
+        for (int i = 0; i < nb; ++i) {
+          const int b = row + i * kWg;
+          if (b < bp) dst[hh * bp + b] = b < g.bins ? acc[hh * nb + i] : 0.f;
+        }
     }
   }
   tc_fence_before();
@@ -775,22 +849,23 @@ constexpr size_t kSmemLimit = 227 * 1024;
 
 template <int HD>
 size_t fwd_smem(const Geo& g) {
-  return make_layout<HD, kFwdStages, 3, kFwdSlots>(bins_padded(g.bins), g.heads, 0).total + 1024;
+  return make_layout<HD, kFwdStages, 3, kFwdSlots * 32768>(bins_padded(g.bins)).total + 1024;
 }
 template <int HD>
-size_t bwd_smem(const Geo& g, int acc_in_smem) {
-  return make_layout<HD, kBwdStages, 4, 2>(bins_padded(g.bins), g.heads, acc_in_smem).total + 1024;
+size_t bwd_smem(const Geo& g) {
+  return make_layout<HD, kBwdStages, 4, kNumBlk * kBlk>(bins_padded(g.bins)).total + 1024;
 }
 
 bool smem_ok(const Geo& g) {
   const size_t f = g.hd == 64 ? fwd_smem<64>(g) : fwd_smem<32>(g);
-  const size_t b = g.hd == 64 ? bwd_smem<64>(g, 0) : bwd_smem<32>(g, 0);
+  const size_t b = g.hd == 64 ? bwd_smem<64>(g) : bwd_smem<32>(g);
   return f <= kSmemLimit && b <= kSmemLimit;
 }
 
+// Bias-gradient sums per CTA in thread-local memory when every thread's share
+// (its table entries for all heads) fits; per tile in the workspace otherwise.
 int acc_mode(const Geo& g) {
-  const size_t b = g.hd == 64 ? bwd_smem<64>(g, 1) : bwd_smem<32>(g, 1);
-  return b <= kSmemLimit ? 1 : 0;
+  return (long long)g.heads * ((g.bins + kWg - 1) / kWg) <= kAccMax ? 1 : 0;
 }
 
 void fill_common(FastParams& p, const Geo& g, const float* bias_t, int* status, int flags) {
@@ -829,7 +904,7 @@ cudaError_t prep_bias(const Geo& g, const float* table, float* bias_t, cudaStrea
 bool fast_supported(const Geo& g, int dtype) {
   if (dtype != SWIN_DTYPE_BF16) return false;
   if (g.hd != 64 && g.hd != 32) return false;
-  if (g.N != 64 && g.N != 32) return false;
+  if (g.N != 64) return false;
   // Every sub-box must be a whole number of 8-row swizzle atoms.
   const int ylen[3] = {g.wh, g.wh - g.sh, g.sh};
   const int xlen[3] = {g.ww, g.ww - g.sw, g.sw};
@@ -863,11 +938,8 @@ cudaError_t fast_forward(const Geo& g, const void* q, const void* k, const void*
     return cudaErrorInvalidValue;
   cudaError_t e = prep_bias(g, table, bias_t, st);
   if (e != cudaSuccess) return e;
-  if (g.hd == 64)
-    return g.N == 64 ? launch(fwd_kernel<64, 64>, p, fwd_smem<64>(g), st)
-                     : launch(fwd_kernel<64, 32>, p, fwd_smem<64>(g), st);
-  return g.N == 64 ? launch(fwd_kernel<32, 64>, p, fwd_smem<32>(g), st)
-                   : launch(fwd_kernel<32, 32>, p, fwd_smem<32>(g), st);
+  return g.hd == 64 ? launch(fwd_kernel<64, 64>, p, fwd_smem<64>(g), st)
+                    : launch(fwd_kernel<32, 64>, p, fwd_smem<32>(g), st);
 }
 
 cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void* v,
@@ -881,20 +953,17 @@ cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void
   p.out1 = dk;
   p.out2 = dv;
   p.partial = partial;
-  p.acc_in_smem = acc_mode(g);
+  p.acc_local = acc_mode(g);
   if (!encode_maps(p, 0, q) || !encode_maps(p, 1, k) || !encode_maps(p, 2, v) ||
       !encode_maps(p, 3, dout))
     return cudaErrorInvalidValue;
   cudaError_t e = prep_bias(g, table, bias_t, st);
   if (e != cudaSuccess) return e;
-  const size_t smem = g.hd == 64 ? bwd_smem<64>(g, p.acc_in_smem) : bwd_smem<32>(g, p.acc_in_smem);
-  if (g.hd == 64)
-    e = g.N == 64 ? launch(bwd_kernel<64, 64>, p, smem, st) : launch(bwd_kernel<64, 32>, p, smem, st);
-  else
-    e = g.N == 64 ? launch(bwd_kernel<32, 64>, p, smem, st) : launch(bwd_kernel<32, 32>, p, smem, st);
+  const size_t smem = g.hd == 64 ? bwd_smem<64>(g) : bwd_smem<32>(g);
+  e = g.hd == 64 ? launch(bwd_kernel<64>, p, smem, st) : launch(bwd_kernel<32>, p, smem, st);
   if (e != cudaSuccess) return e;
   const long long grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
-  return dbias_reduce(g, partial, p.acc_in_smem ? grid : p.n_groups, dtable, st);
+  return dbias_reduce(g, partial, p.acc_local ? grid : p.n_groups, dtable, st);
 }
 
 }  // namespace swin

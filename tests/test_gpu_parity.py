@@ -120,7 +120,7 @@ def test_fast_path_edges(wl):
         assert e <= BF16_TOL, (wl.name, n, e)
 
 
-@pytest.mark.parametrize("win,shift", [((4, 8), (2, 4)), ((8, 4), (4, 2)), ((4, 16), (2, 8))])
+@pytest.mark.parametrize("win,shift", [((4, 16), (2, 8)), ((16, 4), (8, 2)), ((2, 32), (1, 16))])
 def test_fast_path_non_square_windows(win, shift):
     B, H, W, heads, hd = 1, 18, 30, 2, 64
     d = sb.make_desc(B, H, W, win, shift, heads, hd, "bf16")
@@ -154,9 +154,10 @@ def test_hand_example_isolated_tokens_exact_on_gpu(dtype):
 
 
 def test_other_region_keys_do_not_reach_a_query_bit_exact():
-    """Seam window of the 1/12-degree shape: change k and v of one token of region
-    A; queries of the other regions in that window keep identical bits."""
-    wl = WORKLOADS["ragged-90x180-w8"]
+    """Corner window of an unpadded 32 x 48 grid (four 4 x 4 shift regions):
+    change k and v of one token of one region; queries of the other regions in
+    that window keep identical bits, those of its own region change."""
+    wl = Workload("iso", 1, 32, 48, 8, 4, 2, 64, "bf16", 7)
     inp = make_inputs(wl)
     d = sb.desc_for(wl)
     s = oracle_shape(d)

@@ -343,3 +343,28 @@ def test_backward_matches_finite_differences(H, W, win, shift):
             fd = (lp - lm) / (2 * eps)
             an = grad.reshape(-1)[i]
             assert abs(fd - an) <= 2e-8 + 2e-7 * abs(an), (name, i, fd, an)
+
+
+# ---------------------------------------------------------------------------
+# The bf16 error measure of the parity tests
+# ---------------------------------------------------------------------------
+def test_bf16_measure_charges_computation_not_storage_rounding():
+    """Rounding the exact result to bf16 costs (next to) nothing under the parity
+    measure (but up to 0.04 RMS under the raw max|d|/RMS), while a real
+    computational error of 3% of the RMS on one element is caught. (torch rounds
+    fp64 -> bf16 through fp32, a double rounding that can exceed half a bf16 ulp
+    by ~1e-8.)"""
+    import gpu_helpers as gh
+    from shifted_window_attention_pad_b200 import WORKLOADS
+    from shifted_window_attention_pad_b200.synth import make_inputs, as_f64
+    wl = WORKLOADS["ragged-90x180-w8"]
+    inp = make_inputs(wl)
+    s = oracle.make_shape(wl.B, wl.H, wl.W, wl.win, wl.shift, wl.heads, wl.head_dim)
+    o, _ = oracle.forward(s, *(as_f64(inp[n]) for n in ("q", "k", "v", "table")), want_lse=False)
+    rounded = torch.from_numpy(o).to(torch.bfloat16).double().numpy()
+    assert gh.err_bf16(rounded, o) < 1e-6
+    assert gh.err_bf16(rounded, o, storage_rounding=False) > gh.BF16_TOL
+    bad = rounded.copy()
+    rms = np.sqrt(np.mean(o * o))
+    bad.reshape(-1)[12345] += 0.03 * rms + gh.half_ulp_bf16(o.reshape(-1)[12345])
+    assert gh.err_bf16(bad, o) > gh.BF16_TOL
