@@ -26,10 +26,12 @@
 //    from per-slot coordinates (no mask tensor), runs the softmax in registers
 //    (a whole window row is in the tile, so no running rescale is needed), writes
 //    P (and dS) to shared memory for the next MMAs, and stores outputs straight
-//    to their grid rows. The bias-table gradient is summed per warp in shared
-//    memory (lanes of a warp always hit distinct entries), folded per tile in a
-//    fixed order and per CTA, then reduced over CTAs by a second kernel: the sum
-//    order never depends on timing.
+//    to their grid rows. The bias-table gradient is summed in fixed point: each
+//    dS, in units of 2^-24, is split into a high part (units of 2^-8) and a low
+//    part (units of 2^-24, |lo| <= 2^15) added with two native shared-memory
+//    int32 reductions, so the per-tile bins are exact sums whose value does not
+//    depend on the order in which threads land; per CTA they accumulate in
+//    int64, and a second kernel adds the CTAs in a fixed order.
 //  * Warp roles: warps 0-3 softmax/epilogue, warp 4 TMA producer, warp 5 MMA
 //    issuer and TMEM owner. Persistent grid of one CTA per SM; tiles go
 //    round-robin, head fastest, so the SMs stream neighbouring bytes together.
@@ -85,8 +87,8 @@ struct Layout {
 };
 
 // NS stages of NTEN input tiles, then PBYTES of P / dS operand blocks, the
-// bias rows of the stages, the key words, per-warp bias-gradient bins,
-// mbarriers and two words (TMEM base, abort flag).
+// bias rows of the stages, the key words, the tile's bias-gradient bins (two
+// fixed-point int32 parts), mbarriers and two words (TMEM base, abort flag).
 template <int HD, int NS, int NTEN, uint32_t PBYTES>
 __host__ __device__ inline Layout make_layout(int bins_pad) {
   constexpr uint32_t tile_bytes = kRows * HD * 2;
@@ -96,7 +98,7 @@ __host__ __device__ inline Layout make_layout(int bins_pad) {
   L.bias = L.ptile + PBYTES;
   L.colinfo = L.bias + ((NS * bins_pad * 4 + 15) & ~15);
   L.bins_w = L.colinfo + 2 * kRows * 4;
-  L.bars = (L.bins_w + 4 * bins_pad * 4 + 7) & ~7u;
+  L.bars = (L.bins_w + bins_pad * 8 + 7) & ~7u;   // two int32 arrays
   L.misc = L.bars + 8 * 32;
   L.total = L.misc + 16;
   return L;
@@ -256,11 +258,6 @@ __device__ inline uint64_t desc_mnmajor_tile(uint32_t base, int k16) {
 __device__ inline uint64_t desc_p_kmajor(uint32_t base, int k16) {
   return smem_desc(base + (k16 >> 2) * 16384 + (k16 & 3) * 32, 16, 1024, kSwizzle128);
 }
-// As MN-major A of the transpose (M = columns, K = rows): region stride 16 KB
-// between the two 64-column atoms, 8-row groups 1 KB apart.
-__device__ inline uint64_t desc_p_mnmajor(uint32_t base, int k16) {
-  return smem_desc(base + k16 * 2048, 16384, 1024, kSwizzle128);
-}
 
 // Writes this thread's row of a P-style tile: columns [col0, col0 + NCOL) from
 // `vals` (already scaled), rounded to bf16, 128-byte swizzled.
@@ -288,26 +285,121 @@ __device__ inline void store_row_bf16(void* dst, const float* v, float mul) {
                  pack_bf16(v[c * 8 + 6] * mul, v[c * 8 + 7] * mul));
 }
 
+// Warp-collective (.sync.aligned): every lane of the warp must reach it.
 template <int NCOL>
 __device__ inline void tmem_load_cols(uint32_t taddr, float* v) {
+  __syncwarp();
 #pragma unroll
   for (int c = 0; c < NCOL / 32; ++c) tmem_ld32(taddr + c * 32, v + c * 32);
 }
 
 // ================================================================================
+// Per-row softmax pieces of the warpgroup
+// ================================================================================
+// A window is "plain" when it does not straddle the wrap seam and holds no pad
+// token: one TMA box, slots in row-major order, a single shift region, all keys
+// real. For 8 x 8 windows its key offsets into the bias table are compile-time
+// constants, so no per-key word is read and no mask is applied.
+template <int WW>
+__host__ __device__ constexpr int plain_off(int j) {
+  return (j / WW) * (2 * WW - 1) + (j % WW);
+}
+
+__device__ inline bool window_plain(const Geo& g, long long win) {
+  if (win >= g.n_win) return false;
+  int b, wy, wx;
+  window_coords(g, win, b, wy, wx);
+  if (g.sh > 0 && wy == g.nWy - 1) return false;
+  if (g.sw > 0 && wx == g.nWx - 1) return false;
+  return wy * g.wh + g.sh + g.wh <= g.H && wx * g.ww + g.sw + g.ww <= g.W;
+}
+
+template <int WW>
+__device__ inline RowInfo plain_row_info(const Geo& g, long long win, int r) {
+  int b, wy, wx;
+  window_coords(g, win, b, wy, wx);
+  const int iy = r / (WW > 0 ? WW : 1), ix = r % (WW > 0 ? WW : 1);
+  RowInfo ri;
+  ri.valid = true;
+  ri.label = 0;
+  ri.bias_base = (iy + WW - 1) * (2 * WW - 1) + ix + WW - 1;
+  ri.key_off = iy * (2 * WW - 1) + ix;
+  ri.token = ((long long)b * g.H + wy * WW + g.sh + iy) * g.W + wx * WW + g.sw + ix;
+  return ri;
+}
+
+// Logits in log2 units, x <- scale*log2(e)*s + bias (bias pre-scaled), for
+// the N keys of a plain window; returns the row maximum.
+template <int N, int WW>
+__device__ inline float logits_plain(float* x, const float* bias_q, float c) {
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < N; j += 4) {
+    x[j + 0] = fmaf(x[j + 0], c, bias_q[-plain_off<WW>(j + 0)]);
+    x[j + 1] = fmaf(x[j + 1], c, bias_q[-plain_off<WW>(j + 1)]);
+    x[j + 2] = fmaf(x[j + 2], c, bias_q[-plain_off<WW>(j + 2)]);
+    x[j + 3] = fmaf(x[j + 3], c, bias_q[-plain_off<WW>(j + 3)]);
+    m0 = fmaxf(m0, x[j + 0]);
+    m1 = fmaxf(m1, x[j + 1]);
+    m2 = fmaxf(m2, x[j + 2]);
+    m3 = fmaxf(m3, x[j + 3]);
+  }
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+// Same for any window: per-key words give the bias offset and the shift region
+// (15 = pad key); keys of another region or pad keys get -inf.
+template <int N>
+__device__ inline float logits_general(float* x, const float* brow, const uint32_t* cw, int base,
+                                       int label, float c) {
+  float mm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int j0 = 0; j0 < N; j0 += 8) {
+#pragma unroll
+    for (int j = j0; j < j0 + 8; ++j) {
+      const uint32_t w = cw[j];
+      const bool ok = (int)(w >> 16) == label;
+      x[j] = ok ? fmaf(x[j], c, brow[base - (int)(w & 0xFFFF)]) : -INFINITY;
+      mm[j & 3] = fmaxf(mm[j & 3], x[j]);
+    }
+    asm volatile("" ::: "memory");   // bound the loads in flight (registers)
+  }
+  return fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3]));
+}
+
+// x <- 2^(x - m); returns the sum.
+template <int N>
+__device__ inline float exp_sum(float* x, float m) {
+  float l[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    x[j] = ex2(x[j] - m);
+    l[j & 3] += x[j];
+  }
+  return (l[0] + l[1]) + (l[2] + l[3]);
+}
+
+// ================================================================================
 // Forward
 // ================================================================================
+// Per tile: S = Q K^T (MMA) -> softmax row per thread -> P (bf16, smem) ->
+// O = P V (MMA) -> normalise and store. The warpgroup runs one tile behind
+// on the epilogue (softmax of tile k, then the store of tile k-1) so the PV
+// product of a tile overlaps the next tile's softmax; the MMA warp issues S of
+// tile k+1 before PV of tile k. Three TMEM slots of 128 columns, two P tiles.
 constexpr int kFwdStages = 3;
-constexpr int kFwdSlots = 2;   // TMEM slots of 128 columns (S, then O in its first HD)
+constexpr int kFwdSlots = 3;
+constexpr int kFwdPBufs = 2;
 
-template <int HD, int N>
+template <int HD, int WW>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FastParams p) {
+  constexpr int N = 64, G = kRows / N;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  constexpr int NS = kFwdStages, NT = kFwdSlots, G = kRows / N;
+  constexpr int NS = kFwdStages, NT = kFwdSlots;
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   const Geo& g = p.g;
-  const Layout L = make_layout<HD, NS, 3, NT * 32768>(p.bins_pad);
+  const Layout L = make_layout<HD, NS, 3, kFwdPBufs * 32768>(p.bins_pad);
   uint8_t* tiles = smem + L.tiles;
   uint8_t* ptile = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
@@ -339,12 +431,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   if (warp == kProducerWarp && lane == 0)
     for (int tt = 0; tt < 3; ++tt)
       for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
-  // P tiles start at zero: rows never write the columns of other windows.
-  for (uint32_t i = threadIdx.x; i < NT * 32768 / 16; i += kThreads)
+  // P tiles start at zero: rows never write the columns of the other window.
+  for (uint32_t i = threadIdx.x; i < kFwdPBufs * 32768 / 16; i += kThreads)
     reinterpret_cast<uint4*>(ptile)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async();
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, NT * 128);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -372,29 +464,42 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16(kRows, HD, 0, 1);
-      long long k = 0;
-      for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
-        const int s = (int)(k % NS), sl = (int)(k % NT);
-        const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
-        if (!mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs)) break;
-        if (!mbar_wait(&t_empty[sl], pht ^ 1, abort, p.status, kWaitLimitNs)) break;
+      auto issue_s = [&](long long kk) -> bool {
+        const int s = (int)(kk % NS), sl = (int)(kk % NT);
+        if (!mbar_wait(&full[s], (uint32_t)((kk / NS) & 1), abort, p.status, kWaitLimitNs))
+          return false;
+        if (!mbar_wait(&t_empty[sl], (uint32_t)(((kk / NT) & 1) ^ 1), abort, p.status,
+                       kWaitLimitNs))
+          return false;
         tc_fence_after();
         const uint32_t q_s = smem_u32(tiles + (s * 3 + 0) * tile_bytes);
         const uint32_t k_s = smem_u32(tiles + (s * 3 + 1) * tile_bytes);
-        const uint32_t v_s = smem_u32(tiles + (s * 3 + 2) * tile_bytes);
-        const uint32_t d = tmem + sl * 128;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          umma_ss(d, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk), idesc_s, kk);
+        for (int kk16 = 0; kk16 < HD / 16; ++kk16)
+          umma_ss(tmem + sl * 128, desc_kmajor_tile<HD>(q_s, kk16), desc_kmajor_tile<HD>(k_s, kk16),
+                  idesc_s, kk16);
         umma_commit(&s_full[sl]);
-        if (!mbar_wait(&p_full[sl], pht, abort, p.status, kWaitLimitNs)) break;
+        return true;
+      };
+      long long k = 0, t = blockIdx.x;
+      bool ok = t < p.n_tiles ? issue_s(0) : false;
+      while (ok) {
+        const long long tn = t + gridDim.x;
+        if (tn < p.n_tiles && !issue_s(k + 1)) break;
+        const int s = (int)(k % NS), sl = (int)(k % NT);
+        if (!mbar_wait(&p_full[sl], (uint32_t)((k / NT) & 1), abort, p.status, kWaitLimitNs)) break;
         tc_fence_after();
-        const uint32_t p_s = smem_u32(ptile + sl * 32768);
+        const uint32_t v_s = smem_u32(tiles + (s * 3 + 2) * tile_bytes);
+        const uint32_t p_s = smem_u32(ptile + (k % kFwdPBufs) * 32768);
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)
-          umma_ss(d, desc_p_kmajor(p_s, kk), desc_mnmajor_tile<HD>(v_s, kk), idesc_o, kk);
+        for (int kk16 = 0; kk16 < kRows / 16; ++kk16)
+          umma_ss(tmem + sl * 128, desc_p_kmajor(p_s, kk16), desc_mnmajor_tile<HD>(v_s, kk16),
+                  idesc_o, kk16);
         umma_commit(&o_full[sl]);
         umma_commit(&empty[s]);
+        if (tn >= p.n_tiles) break;
+        t = tn;
+        ++k;
       }
       if (*abort) {
         umma_commit(drain);
@@ -404,15 +509,36 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   } else {
     // Softmax / epilogue warpgroup: thread = tile row = TMEM lane.
     const int row = threadIdx.x;
-    const int gw = row / N;
+    const int gw = row / N, lr = row - gw * N;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // the tile whose output is still in TMEM
+    bool pend = false, pvalid = false;
+    long long ptoken = 0, pk = 0;
+    int phead = 0;
+    float pinv = 1.f, plse = 0.f;
+    auto epilogue = [&]() {
+      const int sl = (int)(pk % NT);
+      mbar_wait(&o_full[sl], (uint32_t)((pk / NT) & 1), abort, p.status, kWaitLimitNs);
+      tc_fence_after();
+      float o[HD];
+      tmem_load_cols<HD>(tmem + lane_base + sl * 128, o);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&t_empty[sl]);
+      if (pvalid && !*abort) {
+        store_row_bf16<HD>((__nv_bfloat16*)p.out0 + (ptoken * g.heads + phead) * HD, o, pinv);
+        if (p.lse) p.lse[ptoken * g.heads + phead] = plse;
+      }
+    };
     long long k = 0;
     for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
       const int s = (int)(k % NS), sl = (int)(k % NT);
       const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
       const long long group = t / g.heads;
       const int h = (int)(t - group * g.heads);
-      const RowInfo me = row_info(g, group * G + gw, row - gw * N);
+      const long long win = group * G + gw;
+      const bool plain = WW > 0 && window_plain(g, win);
+      const RowInfo me = plain ? plain_row_info<WW>(g, win, lr) : row_info(g, win, lr);
       uint32_t* ci = colinfo + (k & 1) * kRows;
       ci[row] = key_word(me);
       if (named_sync_or(1, kWg, *abort)) break;
@@ -424,50 +550,38 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       tmem_load_cols<N>(tmem + lane_base + sl * 128 + gw * N, x);
       tmem_wait_ld();
       const float* brow = bias + s * p.bins_pad;
-      const uint32_t* cw = ci + gw * N;
-      float m = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < N; ++j) {
-        const uint32_t w = cw[j];
-        const bool ok = (int)(w >> 16) == me.label;
-        x[j] = ok ? fmaf(x[j], p.scale_log2, brow[me.bias_base - (int)(w & 0xFFFF)]) : -INFINITY;
-        m = fmaxf(m, x[j]);
-      }
-      float l = 0.f;
+      float m;
+      if (plain)
+        m = logits_plain<N, (WW > 0 ? WW : 8)>(x, brow + me.bias_base, p.scale_log2);
+      else
+        m = logits_general<N>(x, brow, ci + gw * N, me.bias_base, me.label, p.scale_log2);
+      float l = 1.f;
       if (me.valid) {
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-          x[j] = ex2(x[j] - m);
-          l += x[j];
-        }
+        l = exp_sum<N>(x, m);
       } else {
 #pragma unroll
         for (int j = 0; j < N; ++j) x[j] = 0.f;
-        l = 1.f;
       }
-      store_p_row<N>(smem_u32(ptile + sl * 32768), row, gw * N, x);
+      store_p_row<N>(smem_u32(ptile + (k % kFwdPBufs) * 32768), row, gw * N, x);
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&p_full[sl]);
-      mbar_wait(&o_full[sl], pht, abort, p.status, kWaitLimitNs);
-      tc_fence_after();
-      float o[HD];
-      tmem_load_cols<HD>(tmem + lane_base + sl * 128, o);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&t_empty[sl]);
-      if (me.valid) {
-        const float inv = 1.f / l;
-        store_row_bf16<HD>((__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD, o, inv);
-        if (p.lse) p.lse[me.token * g.heads + h] = (m + __log2f(l)) * 0.69314718055994531f;
-      }
+      if (pend) epilogue();
+      pend = true;
+      pvalid = me.valid;
+      ptoken = me.token;
+      phead = h;
+      pk = k;
+      pinv = 1.f / l;
+      plse = (m + __log2f(l)) * 0.69314718055994531f;
     }
+    if (pend) epilogue();
   }
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, NT * 128);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -476,21 +590,32 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 // ================================================================================
 // P and scale*dS feed the dV, dQ and dK products. Rounded to bf16 alone they
 // would cost up to 2.5% of the output RMS on the largest gradients, so each is
-// split into bf16 hi + lo parts (x = hi + lo to ~2^-17 relative) and both parts
-// are accumulated in TMEM. The two windows of a tile never mix: each operand is
-// two 64 x 64 blocks (8 KB, 128-byte swizzle, 128-byte rows) plus shared zero
-// blocks Z1, Z2, in this order:
+// split into bf16 hi + lo parts (hi = x with the low 16 bits cleared, lo =
+// bf16(x - hi); x = hi + lo to ~2^-16 relative) and both parts are accumulated
+// in TMEM. The two windows of a tile never mix: each operand is two 64 x 64
+// blocks (8 KB, 128-byte swizzle, 128-byte rows) plus shared zero blocks Z1,
+// Z2, in this order:
 //   [P0h][P0l][dS0h][Z1][dS1h][dS0l][Z2][dS1l][P1h][P1l]
 // As a K-major A (dQ = dS K: rows = queries, K = keys) the key half 0 of dS is
 // the 16 KB run [dS0 | Z] and the key half 1 is [Z | dS1]. As an MN-major A
 // (dV = P^T dO, dK = dS^T Q: M = keys, K = queries) the second 64-key atom is
 // addressed through the leading byte offset, so the query half 0 reads
 // (X0, Z) and the query half 1 reads (Z, X1) for any X0 < Z < X1.
+//
+// Per tile the warpgroup computes P, dS and the bias-gradient bins of tile k,
+// waits until the MMAs of tile k-1 have read the operand blocks, writes tile
+// k's blocks, then stores tile k-1's gradients. The MMA warp issues S and dP
+// of tile k+1 as soon as tile k-1's TMEM slot is free, ahead of tile k's
+// gradient products, so the warpgroup rarely waits on the tensor pipe.
 constexpr int kBwdStages = 2;
 constexpr int kBwdSlots = 2;   // TMEM slots of 256 columns: S | dP, then dV | dQ | dK
 constexpr uint32_t kBlk = 8192;
 enum { kP0h = 0, kP0l, kS0h, kZ1, kS1h, kS0l, kZ2, kS1l, kP1h, kP1l, kNumBlk };
 constexpr int kAccMax = 64;    // thread-local bias-gradient accumulators
+// Fixed point of the bias-gradient sums: resolution 2^-24 per dS (|dS| must
+// stay below 2^22); per-tile bins hold at most 128 terms, so the int32 parts
+// cannot overflow, and the per-CTA int64 sums are exact.
+constexpr double kFixInv = 5.9604644775390625e-08;  // 2^-24
 
 __device__ inline uint64_t desc_blk_kmajor(uint32_t base, int blk0, int blk1, int k16) {
   // keys [0,64) read the run starting at blk0, keys [64,128) the run at blk1
@@ -504,25 +629,39 @@ __device__ inline uint64_t desc_blk_mnmajor(uint32_t base, int x0, int z, int x1
   return smem_desc(start, (uint32_t)(second - first) * kBlk, 1024, kSwizzle128);
 }
 
-// Row `lr` (0..63) of one 64 x 64 block, from 64 fp32 values.
-__device__ inline void store_blk_row(uint32_t blk, int lr, const float* v) {
+// Columns [C0, C0 + NC) of row `lr` (0..63) of the hi and lo blocks of one
+// operand, from NC fp32 values v[0..NC).
+template <int NC>
+__device__ inline void store_split_cols_part(uint32_t blk_hi, uint32_t blk_lo, int lr, int c0,
+                                             const float* v) {
 #pragma unroll
-  for (int c = 0; c < 8; ++c)
-    st_shared_v4(blk + lr * 128 + ((c ^ (lr & 7)) << 4), pack_bf16(v[c * 8 + 0], v[c * 8 + 1]),
-                 pack_bf16(v[c * 8 + 2], v[c * 8 + 3]), pack_bf16(v[c * 8 + 4], v[c * 8 + 5]),
-                 pack_bf16(v[c * 8 + 6], v[c * 8 + 7]));
+  for (int cc = 0; cc < NC / 8; ++cc) {
+    const int c = c0 / 8 + cc;
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t a = __float_as_uint(v[cc * 8 + 2 * e]) & 0xFFFF0000u;
+      const uint32_t b = __float_as_uint(v[cc * 8 + 2 * e + 1]) & 0xFFFF0000u;
+      hw[e] = __byte_perm(a, b, 0x7632);
+      lw[e] = pack_bf16(v[cc * 8 + 2 * e] - __uint_as_float(a),
+                        v[cc * 8 + 2 * e + 1] - __uint_as_float(b));
+    }
+    const uint32_t off = lr * 128 + ((c ^ (lr & 7)) << 4);
+    st_shared_v4(blk_hi + off, hw[0], hw[1], hw[2], hw[3]);
+    st_shared_v4(blk_lo + off, lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+template <int C0, int NC>
+__device__ inline void store_split_cols(uint32_t blk_hi, uint32_t blk_lo, int lr, const float* v) {
+  store_split_cols_part<NC>(blk_hi, blk_lo, lr, C0, v + C0);
 }
 
-__device__ inline float bf16_round(float x) {
-  return __bfloat162float(__float2bfloat16_rn(x));
-}
-
-template <int HD>
+template <int HD, int WW>
 __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ FastParams p) {
-  constexpr int N = 64;
+  constexpr int N = 64, G = kRows / N;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  constexpr int NS = kBwdStages, NT = kBwdSlots, G = kRows / N;
+  constexpr int NS = kBwdStages, NT = kBwdSlots;
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   const Geo& g = p.g;
   const Layout L = make_layout<HD, NS, 4, kNumBlk * kBlk>(p.bins_pad);
@@ -530,7 +669,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* blocks = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
   uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
-  float* bins_w = (float*)(smem + L.bins_w);  // [4 warps][bins_pad]
+  int* bins_hi = (int*)(smem + L.bins_w);   // [bins_pad], units of 2^-8
+  int* bins_lo = bins_hi + p.bins_pad;      // [bins_pad], units of 2^-24
   uint64_t* bars = (uint64_t*)(smem + L.bars);
   uint64_t* full = bars;
   uint64_t* empty = full + NS;
@@ -563,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     reinterpret_cast<uint4*>(blocks + kZ1 * kBlk)[i] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(blocks + kZ2 * kBlk)[i] = make_uint4(0, 0, 0, 0);
   }
-  for (int i = threadIdx.x; i < 4 * bp; i += kThreads) bins_w[i] = 0.f;
+  for (int i = threadIdx.x; i < bp; i += kThreads) bins_hi[i] = bins_lo[i] = 0;
   fence_proxy_async();
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, NT * 256);
@@ -596,12 +736,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       constexpr uint32_t idesc_t = idesc_bf16(kRows, HD, 1, 1);         // dV, dK: A = X^T
       constexpr uint32_t idesc_q = idesc_bf16(kRows, HD, 0, 1);         // dQ
       const uint32_t bb = smem_u32(blocks);
-      long long k = 0;
-      for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
-        const int s = (int)(k % NS), sl = (int)(k % NT);
-        const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
-        if (!mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs)) break;
-        if (!mbar_wait(&t_empty[sl], pht ^ 1, abort, p.status, kWaitLimitNs)) break;
+      auto issue_sdp = [&](long long kk) -> bool {
+        const int s = (int)(kk % NS), sl = (int)(kk % NT);
+        if (!mbar_wait(&full[s], (uint32_t)((kk / NS) & 1), abort, p.status, kWaitLimitNs))
+          return false;
+        if (!mbar_wait(&t_empty[sl], (uint32_t)(((kk / NT) & 1) ^ 1), abort, p.status,
+                       kWaitLimitNs))
+          return false;
         tc_fence_after();
         const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
         const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
@@ -609,15 +750,29 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
         const uint32_t d = tmem + sl * 256;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          umma_ss(d, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk), idesc_s, kk);
+        for (int kk16 = 0; kk16 < HD / 16; ++kk16)
+          umma_ss(d, desc_kmajor_tile<HD>(q_s, kk16), desc_kmajor_tile<HD>(k_s, kk16), idesc_s,
+                  kk16);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          umma_ss(d + 128, desc_kmajor_tile<HD>(do_s, kk), desc_kmajor_tile<HD>(v_s, kk), idesc_s,
-                  kk);
+        for (int kk16 = 0; kk16 < HD / 16; ++kk16)
+          umma_ss(d + 128, desc_kmajor_tile<HD>(do_s, kk16), desc_kmajor_tile<HD>(v_s, kk16),
+                  idesc_s, kk16);
         umma_commit(&sdp_full[sl]);
-        if (!mbar_wait(&pds_full[sl], pht, abort, p.status, kWaitLimitNs)) break;
+        return true;
+      };
+      long long k = 0, t = blockIdx.x;
+      bool ok = t < p.n_tiles ? issue_sdp(0) : false;
+      while (ok) {
+        const long long tn = t + gridDim.x;
+        const int s = (int)(k % NS), sl = (int)(k % NT);
+        if (!mbar_wait(&pds_full[sl], (uint32_t)((k / NT) & 1), abort, p.status, kWaitLimitNs))
+          break;
+        if (tn < p.n_tiles && !issue_sdp(k + 1)) break;
         tc_fence_after();
+        const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
+        const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
+        const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
+        const uint32_t d = tmem + sl * 256;
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk) {  // dV = P^T dO  (hi, then lo)
           umma_ss(d + 0, desc_blk_mnmajor(bb, kP0h, kZ1, kP1h, kk),
@@ -641,6 +796,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         }
         umma_commit(&grad_full[sl]);
         umma_commit(&empty[s]);
+        if (tn >= p.n_tiles) break;
+        t = tn;
+        ++k;
       }
       if (*abort) {
         umma_commit(drain);
@@ -655,18 +813,40 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const uint32_t bb = smem_u32(blocks);
     const uint32_t blk_ph = bb + (gw ? kP1h : kP0h) * kBlk, blk_pl = bb + (gw ? kP1l : kP0l) * kBlk;
     const uint32_t blk_sh = bb + (gw ? kS1h : kS0h) * kBlk, blk_sl = bb + (gw ? kS1l : kS0l) * kBlk;
-    float* my_bins = bins_w + warp * bp;
     const int nb = (g.bins + kWg - 1) / kWg;     // table entries owned by this thread
-    float acc[kAccMax];
+    long long acc[kAccMax];
     if (p.acc_local)
-      for (int i = 0; i < kAccMax; ++i) acc[i] = 0.f;
+      for (int i = 0; i < kAccMax; ++i) acc[i] = 0;
+    bool pend = false, pvalid = false;
+    long long ptoken = 0, pk = 0;
+    int phead = 0;
+    auto epilogue = [&]() {   // gradients of tile pk (its grad_full already waited)
+      const int sl = (int)(pk % NT);
+      tc_fence_after();
+      float o[HD];
+      const bool st = pvalid && !*abort;
+      const long long off = (ptoken * g.heads + phead) * HD;
+      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 0, o);      // dV
+      tmem_wait_ld();
+      if (st) store_row_bf16<HD>((__nv_bfloat16*)p.out2 + off, o, 1.f);
+      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 64, o);     // dQ
+      tmem_wait_ld();
+      if (st) store_row_bf16<HD>((__nv_bfloat16*)p.out0 + off, o, 1.f);
+      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 128, o);    // dK
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&t_empty[sl]);
+      if (st) store_row_bf16<HD>((__nv_bfloat16*)p.out1 + off, o, 1.f);
+    };
     long long k = 0;
     for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
       const int s = (int)(k % NS), sl = (int)(k % NT);
       const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
       const long long group = t / g.heads;
       const int h = (int)(t - group * g.heads);
-      const RowInfo me = row_info(g, group * G + gw, lr);
+      const long long win = group * G + gw;
+      const bool plain = WW > 0 && window_plain(g, win);
+      const RowInfo me = plain ? plain_row_info<WW>(g, win, lr) : row_info(g, win, lr);
       uint32_t* ci = colinfo + (k & 1) * kRows;
       ci[row] = key_word(me);
       if (named_sync_or(1, kWg, *abort)) break;
@@ -674,94 +854,105 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       mbar_wait(&sdp_full[sl], pht, abort, p.status, kWaitLimitNs);
       mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
       tc_fence_after();
-      float x[N], dp[N];
-      tmem_load_cols<N>(tmem + lane_base + sl * 256 + gw * N, x);
-      tmem_load_cols<N>(tmem + lane_base + sl * 256 + 128 + gw * N, dp);
+      // S row -> P (registers); dP is streamed from TMEM in 32-column chunks,
+      // once for D = sum_j P_j dP_j and once for dS, to bound registers.
+      float x[N];
+      const uint32_t s_col = tmem + lane_base + sl * 256 + gw * N;
+      const uint32_t dp_col = s_col + 128;
+      tmem_load_cols<N>(s_col, x);
       tmem_wait_ld();
       const float* brow = bias + s * bp;
       const uint32_t* cw = ci + gw * N;
-      float m = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < N; ++j) {
-        const uint32_t w = cw[j];
-        const bool ok = (int)(w >> 16) == me.label;
-        x[j] = ok ? fmaf(x[j], p.scale_log2, brow[me.bias_base - (int)(w & 0xFFFF)]) : -INFINITY;
-        m = fmaxf(m, x[j]);
-      }
+      float m;
+      if (plain)
+        m = logits_plain<N, (WW > 0 ? WW : 8)>(x, brow + me.bias_base, p.scale_log2);
+      else
+        m = logits_general<N>(x, brow, cw, me.bias_base, me.label, p.scale_log2);
       if (me.valid) {
-        float l = 0.f;
+        const float inv = 1.f / exp_sum<N>(x, m);
 #pragma unroll
-        for (int j = 0; j < N; ++j) {
-          x[j] = ex2(x[j] - m);
-          l += x[j];
-        }
-        const float inv = 1.f / l;
-        float D = 0.f;
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-          x[j] *= inv;
-          D = fmaf(x[j], dp[j], D);
-        }
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-          const float ds = x[j] * (dp[j] - D);
-          const uint32_t w = cw[j];
-          if ((int)(w >> 16) == me.label) {
-            float* bin = my_bins + me.bias_base - (int)(w & 0xFFFF);
-            *bin += ds;
-          }
-          dp[j] = ds * dscale;
-        }
+        for (int j = 0; j < N; ++j) x[j] *= inv;
       } else {
 #pragma unroll
-        for (int j = 0; j < N; ++j) x[j] = dp[j] = 0.f;
+        for (int j = 0; j < N; ++j) x[j] = 0.f;
       }
-      // hi parts, then the residuals as lo parts
-      store_blk_row(blk_ph, lr, x);
-      store_blk_row(blk_sh, lr, dp);
+      // TMEM loads are warp-collective: every lane runs them, valid row or not
+      // (x = 0 on invalid rows, so D = 0 and dS = 0 there).
+      float dd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < N; ++j) {
-        x[j] -= bf16_round(x[j]);
-        dp[j] -= bf16_round(dp[j]);
+      for (int c = 0; c < N / 32; ++c) {
+        float dp[32];
+        __syncwarp();
+        tmem_ld32(dp_col + 32 * c, dp);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dd[j & 3] = fmaf(x[32 * c + j], dp[j], dd[j & 3]);
       }
-      store_blk_row(blk_pl, lr, x);
-      store_blk_row(blk_sl, lr, dp);
+      const float D = (dd[0] + dd[1]) + (dd[2] + dd[3]);
+      if (pend)   // the MMAs of the previous tile are done with the operand blocks
+        mbar_wait(&grad_full[(int)(pk % NT)], (uint32_t)((pk / NT) & 1), abort, p.status,
+                  kWaitLimitNs);
+      store_split_cols<0, N>(blk_ph, blk_pl, lr, x);
+      int* bqh = bins_hi + me.bias_base;
+      int* bql = bins_lo + me.bias_base;
+#pragma unroll
+      for (int c = 0; c < N / 32; ++c) {
+        float ds[32];
+        __syncwarp();
+        tmem_ld32(dp_col + 32 * c, ds);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ds[j] = x[32 * c + j] * (ds[j] - D);   // dS (0 off the row)
+        if (me.valid) {
+          // bias-gradient bins, fixed point: integer adds commute, so the sum
+          // is exact and independent of the order the lanes land in
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(32 * c + j)
+                                  : (int)(lds_u32(cw + 32 * c + j) & 0xFFFF);
+            const float t = ds[j] * 256.0f;                 // units of 2^-8
+            const float hf = rintf(t);
+            red_add_s32(bqh - off, __float2int_rn(hf));
+            red_add_s32(bql - off, __float2int_rn((t - hf) * 65536.0f));
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ds[j] *= dscale;
+        store_split_cols_part<32>(blk_sh, blk_sl, lr, 32 * c, ds);
+      }
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&pds_full[sl]);
-      // Fold the four warps' bias-gradient bins of this tile, in warp order.
+      // Move this tile's bins into the per-CTA accumulators (or the workspace).
       named_sync(2, kWg);
       for (int i = 0; i < nb; ++i) {
         const int b = row + i * kWg;
         if (b >= g.bins) break;
-        const float v4 = bins_w[b] + bins_w[bp + b] + bins_w[2 * bp + b] + bins_w[3 * bp + b];
-        bins_w[b] = bins_w[bp + b] = bins_w[2 * bp + b] = bins_w[3 * bp + b] = 0.f;
+        const long long v = ((long long)bins_hi[b] << 16) + bins_lo[b];   // units of 2^-24
+        bins_hi[b] = bins_lo[b] = 0;
         if (p.acc_local)
-          acc[h * nb + i] += v4;
+          acc[h * nb + i] += v;
         else
-          p.partial[(group * g.heads + h) * bp + b] = v4;
+          p.partial[(group * g.heads + h) * bp + b] = (float)((double)v * kFixInv);
       }
-      mbar_wait(&grad_full[sl], pht, abort, p.status, kWaitLimitNs);
-      tc_fence_after();
-      float o[HD];
-      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 0, o);      // dV
-      tmem_wait_ld();
-      if (me.valid) store_row_bf16<HD>((__nv_bfloat16*)p.out2 + (me.token * g.heads + h) * HD, o, 1.f);
-      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 64, o);     // dQ
-      tmem_wait_ld();
-      if (me.valid) store_row_bf16<HD>((__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD, o, 1.f);
-      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 128, o);    // dK
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&t_empty[sl]);
-      if (me.valid) store_row_bf16<HD>((__nv_bfloat16*)p.out1 + (me.token * g.heads + h) * HD, o, 1.f);
+      if (pend) epilogue();
+      pend = true;
+      pvalid = me.valid;
+      ptoken = me.token;
+      phead = h;
+      pk = k;
+    }
+    if (pend) {
+      mbar_wait(&grad_full[(int)(pk % NT)], (uint32_t)((pk / NT) & 1), abort, p.status,
+                kWaitLimitNs);
+      epilogue();
     }
     if (p.acc_local) {
       float* dst = p.partial + (long long)blockIdx.x * g.heads * bp;
       for (int hh = 0; hh < g.heads; ++hh)
         for (int i = 0; i < nb; ++i) {
           const int b = row + i * kWg;
-          if (b < bp) dst[hh * bp + b] = b < g.bins ? acc[hh * nb + i] : 0.f;
+          if (b < bp) dst[hh * bp + b] = b < g.bins ? (float)((double)acc[hh * nb + i] * kFixInv) : 0.f;
         }
     }
   }
@@ -849,7 +1040,7 @@ constexpr size_t kSmemLimit = 227 * 1024;
 
 template <int HD>
 size_t fwd_smem(const Geo& g) {
-  return make_layout<HD, kFwdStages, 3, kFwdSlots * 32768>(bins_padded(g.bins)).total + 1024;
+  return make_layout<HD, kFwdStages, 3, kFwdPBufs * 32768>(bins_padded(g.bins)).total + 1024;
 }
 template <int HD>
 size_t bwd_smem(const Geo& g) {
@@ -938,8 +1129,12 @@ cudaError_t fast_forward(const Geo& g, const void* q, const void* k, const void*
     return cudaErrorInvalidValue;
   cudaError_t e = prep_bias(g, table, bias_t, st);
   if (e != cudaSuccess) return e;
-  return g.hd == 64 ? launch(fwd_kernel<64, 64>, p, fwd_smem<64>(g), st)
-                    : launch(fwd_kernel<32, 64>, p, fwd_smem<32>(g), st);
+  const bool w8 = g.wh == 8 && g.ww == 8;
+  if (g.hd == 64)
+    return w8 ? launch(fwd_kernel<64, 8>, p, fwd_smem<64>(g), st)
+              : launch(fwd_kernel<64, 0>, p, fwd_smem<64>(g), st);
+  return w8 ? launch(fwd_kernel<32, 8>, p, fwd_smem<32>(g), st)
+            : launch(fwd_kernel<32, 0>, p, fwd_smem<32>(g), st);
 }
 
 cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void* v,
@@ -960,7 +1155,11 @@ cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void
   cudaError_t e = prep_bias(g, table, bias_t, st);
   if (e != cudaSuccess) return e;
   const size_t smem = g.hd == 64 ? bwd_smem<64>(g) : bwd_smem<32>(g);
-  e = g.hd == 64 ? launch(bwd_kernel<64>, p, smem, st) : launch(bwd_kernel<32>, p, smem, st);
+  const bool w8 = g.wh == 8 && g.ww == 8;
+  if (g.hd == 64)
+    e = w8 ? launch(bwd_kernel<64, 8>, p, smem, st) : launch(bwd_kernel<64, 0>, p, smem, st);
+  else
+    e = w8 ? launch(bwd_kernel<32, 8>, p, smem, st) : launch(bwd_kernel<32, 0>, p, smem, st);
   if (e != cudaSuccess) return e;
   const long long grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
   return dbias_reduce(g, partial, p.acc_local ? grid : p.n_groups, dtable, st);
