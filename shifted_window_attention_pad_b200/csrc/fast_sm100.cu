@@ -26,12 +26,12 @@
 //    from per-slot coordinates (no mask tensor), runs the softmax in registers
 //    (a whole window row is in the tile, so no running rescale is needed), writes
 //    P (and dS) to shared memory for the next MMAs, and stores outputs straight
-//    to their grid rows. The bias-table gradient is summed in fixed point: each
-//    dS, in units of 2^-24, is split into a high part (units of 2^-8) and a low
-//    part (units of 2^-24, |lo| <= 2^15) added with two native shared-memory
-//    int32 reductions, so the per-tile bins are exact sums whose value does not
-//    depend on the order in which threads land; per CTA they accumulate in
-//    int64, and a second kernel adds the CTAs in a fixed order.
+//    to their grid rows. The bias-table gradient is summed in fixed point
+//    (units of 2^-16): a tile's bins are int32 shared-memory reductions, folded
+//    per tile into one int64 table in global memory with global reductions.
+//    Integer sums are exact and do not depend on the order in which threads or
+//    CTAs land, so the result is bitwise repeatable; a last small kernel
+//    converts it to fp32.
 //  * Warp roles: warps 0-3 softmax/epilogue, warp 4 TMA producer, warp 5 MMA
 //    issuer and TMEM owner. Persistent grid of one CTA per SM; tiles go
 //    round-robin, head fastest, so the SMs stream neighbouring bytes together.
@@ -54,10 +54,11 @@ namespace {
 using namespace ptx;
 
 constexpr int kRows = 128;        // tile rows = TMEM lanes = UMMA M
-constexpr int kWg = 128;          // softmax / epilogue threads (warps 0-3)
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 192;
+constexpr int kWg = 128;          // threads of one softmax / epilogue warpgroup
+constexpr int kNumWg = 2;         // warpgroups 0 (warps 0-3) and 1 (warps 4-7) alternate tiles
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr int kMaxMaps = 9;       // box shapes: {full, seam part 1, seam part 2}^2
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestLimitNs = 1000000ull;
@@ -69,14 +70,13 @@ struct FastParams {
   long long n_groups;             // tiles per head: ceil(n_win / G)
   long long n_tiles;              // n_groups * heads
   int bins_pad;
-  int acc_local;                  // bias-gradient accumulation per CTA in thread-local memory
   float scale_log2;               // head_dim^-1/2 * log2(e)
   const float* bias_t;            // [heads][bins_pad], times log2(e)
   void* out0;                     // forward: out;  backward: dq
   void* out1;                     // backward: dk
   void* out2;                     // backward: dv
   float* lse;                     // forward, optional
-  float* partial;                 // backward: bias-gradient partials [unit][heads][bins_pad]
+  long long* dt_fixed;            // backward: bias gradient [heads][bins_pad], units of 2^-16
   int* status;                    // device status word (workspace header)
   int test_timeout;
 };
@@ -87,8 +87,9 @@ struct Layout {
 };
 
 // NS stages of NTEN input tiles, then PBYTES of P / dS operand blocks, the
-// bias rows of the stages, the key words, the tile's bias-gradient bins (two
-// fixed-point int32 parts), mbarriers and two words (TMEM base, abort flag).
+// bias rows of the stages, per warpgroup two buffers of key words and the
+// tile's bias-gradient bins (two fixed-point int32 parts), mbarriers and two
+// words (TMEM base, abort flag).
 template <int HD, int NS, int NTEN, uint32_t PBYTES>
 __host__ __device__ inline Layout make_layout(int bins_pad) {
   constexpr uint32_t tile_bytes = kRows * HD * 2;
@@ -97,8 +98,8 @@ __host__ __device__ inline Layout make_layout(int bins_pad) {
   L.ptile = L.tiles + NS * NTEN * tile_bytes;
   L.bias = L.ptile + PBYTES;
   L.colinfo = L.bias + ((NS * bins_pad * 4 + 15) & ~15);
-  L.bins_w = L.colinfo + 2 * kRows * 4;
-  L.bars = (L.bins_w + bins_pad * 8 + 7) & ~7u;   // two int32 arrays
+  L.bins_w = L.colinfo + kNumWg * 2 * kRows * 4;
+  L.bars = (L.bins_w + kNumWg * bins_pad * 8 + 7) & ~7u;
   L.misc = L.bars + 8 * 32;
   L.total = L.misc + 16;
   return L;
@@ -383,13 +384,20 @@ __device__ inline float exp_sum(float* x, float m) {
 // Forward
 // ================================================================================
 // Per tile: S = Q K^T (MMA) -> softmax row per thread -> P (bf16, smem) ->
-// O = P V (MMA) -> normalise and store. The warpgroup runs one tile behind
-// on the epilogue (softmax of tile k, then the store of tile k-1) so the PV
-// product of a tile overlaps the next tile's softmax; the MMA warp issues S of
-// tile k+1 before PV of tile k. Three TMEM slots of 128 columns, two P tiles.
+// O = P V (MMA) -> normalise and store. Two warpgroups take alternate tiles, so
+// while one waits on TMEM loads or an MMA the other computes (two warps per
+// scheduler). The MMA warp polls: it issues S of the next tile as soon as its
+// data and TMEM slot are ready and PV of a tile as soon as its P is written.
+// Four TMEM slots of 128 columns (S, then O in the first HD), one P tile per
+// warpgroup, three input stages.
 constexpr int kFwdStages = 3;
-constexpr int kFwdSlots = 3;
-constexpr int kFwdPBufs = 2;
+constexpr int kFwdSlots = 4;
+constexpr int kFwdPBufs = kNumWg;
+
+// Number of tiles CTA `cta` takes in a grid of `grid` CTAs.
+__device__ inline long long local_tiles(long long n_tiles, long long cta, long long grid) {
+  return cta < n_tiles ? (n_tiles - 1 - cta) / grid + 1 : 0;
+}
 
 template <int HD, int WW>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FastParams p) {
@@ -417,6 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   volatile int* abort = (volatile int*)(smem + L.misc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long n_local = local_tiles(p.n_tiles, blockIdx.x, gridDim.x);
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < NT; ++i) {
@@ -464,42 +473,52 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16(kRows, HD, 0, 1);
-      auto issue_s = [&](long long kk) -> bool {
-        const int s = (int)(kk % NS), sl = (int)(kk % NT);
-        if (!mbar_wait(&full[s], (uint32_t)((kk / NS) & 1), abort, p.status, kWaitLimitNs))
-          return false;
-        if (!mbar_wait(&t_empty[sl], (uint32_t)(((kk / NT) & 1) ^ 1), abort, p.status,
-                       kWaitLimitNs))
-          return false;
-        tc_fence_after();
-        const uint32_t q_s = smem_u32(tiles + (s * 3 + 0) * tile_bytes);
-        const uint32_t k_s = smem_u32(tiles + (s * 3 + 1) * tile_bytes);
+      long long ns = 0, np = 0;               // next S to issue, next PV to issue
+      uint64_t t0 = globaltimer();
+      while (np < n_local) {
+        bool prog = false;
+        if (ns < n_local) {
+          const int s = (int)(ns % NS), sl = (int)(ns % NT);
+          if (mbar_test(&full[s], (uint32_t)((ns / NS) & 1)) &&
+              mbar_test(&t_empty[sl], (uint32_t)(((ns / NT) & 1) ^ 1))) {
+            tc_fence_after();
+            const uint32_t q_s = smem_u32(tiles + (s * 3 + 0) * tile_bytes);
+            const uint32_t k_s = smem_u32(tiles + (s * 3 + 1) * tile_bytes);
 #pragma unroll
-        for (int kk16 = 0; kk16 < HD / 16; ++kk16)
-          umma_ss(tmem + sl * 128, desc_kmajor_tile<HD>(q_s, kk16), desc_kmajor_tile<HD>(k_s, kk16),
-                  idesc_s, kk16);
-        umma_commit(&s_full[sl]);
-        return true;
-      };
-      long long k = 0, t = blockIdx.x;
-      bool ok = t < p.n_tiles ? issue_s(0) : false;
-      while (ok) {
-        const long long tn = t + gridDim.x;
-        if (tn < p.n_tiles && !issue_s(k + 1)) break;
-        const int s = (int)(k % NS), sl = (int)(k % NT);
-        if (!mbar_wait(&p_full[sl], (uint32_t)((k / NT) & 1), abort, p.status, kWaitLimitNs)) break;
-        tc_fence_after();
-        const uint32_t v_s = smem_u32(tiles + (s * 3 + 2) * tile_bytes);
-        const uint32_t p_s = smem_u32(ptile + (k % kFwdPBufs) * 32768);
+            for (int kk = 0; kk < HD / 16; ++kk)
+              umma_ss(tmem + sl * 128, desc_kmajor_tile<HD>(q_s, kk),
+                      desc_kmajor_tile<HD>(k_s, kk), idesc_s, kk);
+            umma_commit(&s_full[sl]);
+            ++ns;
+            prog = true;
+          }
+        }
+        if (np < ns) {
+          const int s = (int)(np % NS), sl = (int)(np % NT);
+          if (mbar_test(&p_full[sl], (uint32_t)((np / NT) & 1))) {
+            tc_fence_after();
+            const uint32_t v_s = smem_u32(tiles + (s * 3 + 2) * tile_bytes);
+            const uint32_t p_s = smem_u32(ptile + (np % kFwdPBufs) * 32768);
 #pragma unroll
-        for (int kk16 = 0; kk16 < kRows / 16; ++kk16)
-          umma_ss(tmem + sl * 128, desc_p_kmajor(p_s, kk16), desc_mnmajor_tile<HD>(v_s, kk16),
-                  idesc_o, kk16);
-        umma_commit(&o_full[sl]);
-        umma_commit(&empty[s]);
-        if (tn >= p.n_tiles) break;
-        t = tn;
-        ++k;
+            for (int kk = 0; kk < kRows / 16; ++kk)
+              umma_ss(tmem + sl * 128, desc_p_kmajor(p_s, kk), desc_mnmajor_tile<HD>(v_s, kk),
+                      idesc_o, kk);
+            umma_commit(&o_full[sl]);
+            umma_commit(&empty[s]);
+            ++np;
+            prog = true;
+          }
+        }
+        if (prog) {
+          t0 = globaltimer();
+        } else {
+          if (*abort) break;
+          if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicExch(p.status, -5);
+            break;
+          }
+        }
       }
       if (*abort) {
         umma_commit(drain);
@@ -507,31 +526,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       }
     }
   } else {
-    // Softmax / epilogue warpgroup: thread = tile row = TMEM lane.
-    const int row = threadIdx.x;
+    // Softmax / epilogue warpgroups: thread = tile row = TMEM lane.
+    const int wg = warp >> 2;
+    const int row = threadIdx.x & (kWg - 1);
     const int gw = row / N, lr = row - gw * N;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    // the tile whose output is still in TMEM
-    bool pend = false, pvalid = false;
-    long long ptoken = 0, pk = 0;
-    int phead = 0;
-    float pinv = 1.f, plse = 0.f;
-    auto epilogue = [&]() {
-      const int sl = (int)(pk % NT);
-      mbar_wait(&o_full[sl], (uint32_t)((pk / NT) & 1), abort, p.status, kWaitLimitNs);
-      tc_fence_after();
-      float o[HD];
-      tmem_load_cols<HD>(tmem + lane_base + sl * 128, o);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&t_empty[sl]);
-      if (pvalid && !*abort) {
-        store_row_bf16<HD>((__nv_bfloat16*)p.out0 + (ptoken * g.heads + phead) * HD, o, pinv);
-        if (p.lse) p.lse[ptoken * g.heads + phead] = plse;
-      }
-    };
-    long long k = 0;
-    for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t p_s = smem_u32(ptile + wg * 32768);
+    long long k = wg;
+    for (long long t = blockIdx.x + wg * (long long)gridDim.x; t < p.n_tiles;
+         t += kNumWg * (long long)gridDim.x, k += kNumWg) {
       const int s = (int)(k % NS), sl = (int)(k % NT);
       const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
       const long long group = t / g.heads;
@@ -539,9 +542,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const long long win = group * G + gw;
       const bool plain = WW > 0 && window_plain(g, win);
       const RowInfo me = plain ? plain_row_info<WW>(g, win, lr) : row_info(g, win, lr);
-      uint32_t* ci = colinfo + (k & 1) * kRows;
+      uint32_t* ci = colinfo + (wg * 2 + ((k / kNumWg) & 1)) * kRows;
       ci[row] = key_word(me);
-      if (named_sync_or(1, kWg, *abort)) break;
+      if (named_sync_or(1 + wg, kWg, *abort)) break;
       if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
       mbar_wait(&s_full[sl], pht, abort, p.status, kWaitLimitNs);
       mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
@@ -562,20 +565,30 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
         for (int j = 0; j < N; ++j) x[j] = 0.f;
       }
-      store_p_row<N>(smem_u32(ptile + (k % kFwdPBufs) * 32768), row, gw * N, x);
+      store_p_row<N>(p_s, row, gw * N, x);
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&p_full[sl]);
-      if (pend) epilogue();
-      pend = true;
-      pvalid = me.valid;
-      ptoken = me.token;
-      phead = h;
-      pk = k;
-      pinv = 1.f / l;
-      plse = (m + __log2f(l)) * 0.69314718055994531f;
+      // epilogue: O row from TMEM, normalised, straight to its grid token
+      mbar_wait(&o_full[sl], pht, abort, p.status, kWaitLimitNs);
+      tc_fence_after();
+      const bool st = me.valid && !*abort;
+      const float inv = 1.f / l;
+      __nv_bfloat16* dst = (__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        float o[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_base + sl * 128 + 32 * c, o);
+        tmem_wait_ld();
+        if (c == HD / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(&t_empty[sl]);
+        }
+        if (st) store_row_bf16<32>(dst + 32 * c, o, inv);
+      }
+      if (st && p.lse) p.lse[me.token * g.heads + h] = (m + __log2f(l)) * 0.69314718055994531f;
     }
-    if (pend) epilogue();
   }
   tc_fence_before();
   __syncthreads();
@@ -602,20 +615,20 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 // addressed through the leading byte offset, so the query half 0 reads
 // (X0, Z) and the query half 1 reads (Z, X1) for any X0 < Z < X1.
 //
-// Per tile the warpgroup computes P, dS and the bias-gradient bins of tile k,
-// waits until the MMAs of tile k-1 have read the operand blocks, writes tile
-// k's blocks, then stores tile k-1's gradients. The MMA warp issues S and dP
-// of tile k+1 as soon as tile k-1's TMEM slot is free, ahead of tile k's
-// gradient products, so the warpgroup rarely waits on the tensor pipe.
+// Two warpgroups take alternate tiles, each with its own TMEM slot of 256
+// columns (S | dP, then dV | dQ | dK). The operand blocks are shared: tile k
+// writes them once the gradient products of tile k-1 have completed. The MMA
+// warp polls: S and dP of a tile go out as soon as its data and slot are ready,
+// the gradient products as soon as its blocks are written.
 constexpr int kBwdStages = 2;
-constexpr int kBwdSlots = 2;   // TMEM slots of 256 columns: S | dP, then dV | dQ | dK
+constexpr int kBwdSlots = 2;
 constexpr uint32_t kBlk = 8192;
 enum { kP0h = 0, kP0l, kS0h, kZ1, kS1h, kS0l, kZ2, kS1l, kP1h, kP1l, kNumBlk };
-constexpr int kAccMax = 64;    // thread-local bias-gradient accumulators
-// Fixed point of the bias-gradient sums: resolution 2^-24 per dS (|dS| must
-// stay below 2^22); per-tile bins hold at most 128 terms, so the int32 parts
-// cannot overflow, and the per-CTA int64 sums are exact.
-constexpr double kFixInv = 5.9604644775390625e-08;  // 2^-24
+// Fixed point of the bias-gradient sums, in units of 2^-16: a dS below 64 in
+// magnitude goes whole into the low int32 part; larger ones (|dS| < 2^22) are
+// split into an integer high part and a low remainder. A tile's bins hold at
+// most 128 terms, so neither part can overflow; the global table is int64.
+constexpr double kFixInv = 1.52587890625e-05;  // 2^-16
 
 __device__ inline uint64_t desc_blk_kmajor(uint32_t base, int blk0, int blk1, int k16) {
   // keys [0,64) read the run starting at blk0, keys [64,128) the run at blk1
@@ -629,7 +642,7 @@ __device__ inline uint64_t desc_blk_mnmajor(uint32_t base, int x0, int z, int x1
   return smem_desc(start, (uint32_t)(second - first) * kBlk, 1024, kSwizzle128);
 }
 
-// Columns [C0, C0 + NC) of row `lr` (0..63) of the hi and lo blocks of one
+// Columns [c0, c0 + NC) of row `lr` (0..63) of the hi and lo blocks of one
 // operand, from NC fp32 values v[0..NC).
 template <int NC>
 __device__ inline void store_split_cols_part(uint32_t blk_hi, uint32_t blk_lo, int lr, int c0,
@@ -651,9 +664,11 @@ __device__ inline void store_split_cols_part(uint32_t blk_hi, uint32_t blk_lo, i
     st_shared_v4(blk_lo + off, lw[0], lw[1], lw[2], lw[3]);
   }
 }
-template <int C0, int NC>
-__device__ inline void store_split_cols(uint32_t blk_hi, uint32_t blk_lo, int lr, const float* v) {
-  store_split_cols_part<NC>(blk_hi, blk_lo, lr, C0, v + C0);
+
+// x (|x| < 2^22) rounded to the nearest integer with the float adder:
+// adding 1.5 * 2^23 leaves round(x) in the low mantissa bits.
+__device__ inline int round_int_fma(float x) {
+  return __float_as_int(x + 12582912.0f) - 0x4B400000;
 }
 
 template <int HD, int WW>
@@ -664,13 +679,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   constexpr int NS = kBwdStages, NT = kBwdSlots;
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   const Geo& g = p.g;
-  const Layout L = make_layout<HD, NS, 4, kNumBlk * kBlk>(p.bins_pad);
+  const int bp = p.bins_pad;
+  const Layout L = make_layout<HD, NS, 4, kNumBlk * kBlk>(bp);
   uint8_t* tiles = smem + L.tiles;
   uint8_t* blocks = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
   uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
-  int* bins_hi = (int*)(smem + L.bins_w);   // [bins_pad], units of 2^-8
-  int* bins_lo = bins_hi + p.bins_pad;      // [bins_pad], units of 2^-24
+  int* bins = (int*)(smem + L.bins_w);   // [wg][hi, lo][bins_pad]
   uint64_t* bars = (uint64_t*)(smem + L.bars);
   uint64_t* full = bars;
   uint64_t* empty = full + NS;
@@ -684,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   volatile int* abort = (volatile int*)(smem + L.misc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bp = p.bins_pad;
+  const long long n_local = local_tiles(p.n_tiles, blockIdx.x, gridDim.x);
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < NT; ++i) {
@@ -703,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     reinterpret_cast<uint4*>(blocks + kZ1 * kBlk)[i] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(blocks + kZ2 * kBlk)[i] = make_uint4(0, 0, 0, 0);
   }
-  for (int i = threadIdx.x; i < bp; i += kThreads) bins_hi[i] = bins_lo[i] = 0;
+  for (int i = threadIdx.x; i < kNumWg * 2 * bp; i += kThreads) bins[i] = 0;
   fence_proxy_async();
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, NT * 256);
@@ -736,69 +751,78 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       constexpr uint32_t idesc_t = idesc_bf16(kRows, HD, 1, 1);         // dV, dK: A = X^T
       constexpr uint32_t idesc_q = idesc_bf16(kRows, HD, 0, 1);         // dQ
       const uint32_t bb = smem_u32(blocks);
-      auto issue_sdp = [&](long long kk) -> bool {
-        const int s = (int)(kk % NS), sl = (int)(kk % NT);
-        if (!mbar_wait(&full[s], (uint32_t)((kk / NS) & 1), abort, p.status, kWaitLimitNs))
-          return false;
-        if (!mbar_wait(&t_empty[sl], (uint32_t)(((kk / NT) & 1) ^ 1), abort, p.status,
-                       kWaitLimitNs))
-          return false;
-        tc_fence_after();
-        const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
-        const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
-        const uint32_t v_s = smem_u32(tiles + (s * 4 + 2) * tile_bytes);
-        const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
-        const uint32_t d = tmem + sl * 256;
+      long long ns = 0, ng = 0;               // next S/dP to issue, next gradient products
+      uint64_t t0 = globaltimer();
+      while (ng < n_local) {
+        bool prog = false;
+        if (ns < n_local) {
+          const int s = (int)(ns % NS), sl = (int)(ns % NT);
+          if (mbar_test(&full[s], (uint32_t)((ns / NS) & 1)) &&
+              mbar_test(&t_empty[sl], (uint32_t)(((ns / NT) & 1) ^ 1))) {
+            tc_fence_after();
+            const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
+            const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
+            const uint32_t v_s = smem_u32(tiles + (s * 4 + 2) * tile_bytes);
+            const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
+            const uint32_t d = tmem + sl * 256;
 #pragma unroll
-        for (int kk16 = 0; kk16 < HD / 16; ++kk16)
-          umma_ss(d, desc_kmajor_tile<HD>(q_s, kk16), desc_kmajor_tile<HD>(k_s, kk16), idesc_s,
-                  kk16);
+            for (int kk = 0; kk < HD / 16; ++kk)
+              umma_ss(d, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk), idesc_s,
+                      kk);
 #pragma unroll
-        for (int kk16 = 0; kk16 < HD / 16; ++kk16)
-          umma_ss(d + 128, desc_kmajor_tile<HD>(do_s, kk16), desc_kmajor_tile<HD>(v_s, kk16),
-                  idesc_s, kk16);
-        umma_commit(&sdp_full[sl]);
-        return true;
-      };
-      long long k = 0, t = blockIdx.x;
-      bool ok = t < p.n_tiles ? issue_sdp(0) : false;
-      while (ok) {
-        const long long tn = t + gridDim.x;
-        const int s = (int)(k % NS), sl = (int)(k % NT);
-        if (!mbar_wait(&pds_full[sl], (uint32_t)((k / NT) & 1), abort, p.status, kWaitLimitNs))
-          break;
-        if (tn < p.n_tiles && !issue_sdp(k + 1)) break;
-        tc_fence_after();
-        const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
-        const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
-        const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
-        const uint32_t d = tmem + sl * 256;
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk) {  // dV = P^T dO  (hi, then lo)
-          umma_ss(d + 0, desc_blk_mnmajor(bb, kP0h, kZ1, kP1h, kk),
-                  desc_mnmajor_tile<HD>(do_s, kk), idesc_t, kk);
-          umma_ss(d + 0, desc_blk_mnmajor(bb, kP0l, kZ1, kP1l, kk),
-                  desc_mnmajor_tile<HD>(do_s, kk), idesc_t, 1);
+            for (int kk = 0; kk < HD / 16; ++kk)
+              umma_ss(d + 128, desc_kmajor_tile<HD>(do_s, kk), desc_kmajor_tile<HD>(v_s, kk),
+                      idesc_s, kk);
+            umma_commit(&sdp_full[sl]);
+            ++ns;
+            prog = true;
+          }
         }
+        if (ng < ns) {
+          const int s = (int)(ng % NS), sl = (int)(ng % NT);
+          if (mbar_test(&pds_full[sl], (uint32_t)((ng / NT) & 1))) {
+            tc_fence_after();
+            const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
+            const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
+            const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
+            const uint32_t d = tmem + sl * 256;
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk) {  // dQ = dS K
-          umma_ss(d + 64, desc_blk_kmajor(bb, kS0h, kZ1, kk), desc_mnmajor_tile<HD>(k_s, kk),
-                  idesc_q, kk);
-          umma_ss(d + 64, desc_blk_kmajor(bb, kS0l, kZ2, kk), desc_mnmajor_tile<HD>(k_s, kk),
-                  idesc_q, 1);
-        }
+            for (int kk = 0; kk < kRows / 16; ++kk) {  // dV = P^T dO  (hi, then lo)
+              umma_ss(d + 0, desc_blk_mnmajor(bb, kP0h, kZ1, kP1h, kk),
+                      desc_mnmajor_tile<HD>(do_s, kk), idesc_t, kk);
+              umma_ss(d + 0, desc_blk_mnmajor(bb, kP0l, kZ1, kP1l, kk),
+                      desc_mnmajor_tile<HD>(do_s, kk), idesc_t, 1);
+            }
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk) {  // dK = dS^T Q
-          umma_ss(d + 128, desc_blk_mnmajor(bb, kS0h, kZ1, kS1h, kk),
-                  desc_mnmajor_tile<HD>(q_s, kk), idesc_t, kk);
-          umma_ss(d + 128, desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, kk),
-                  desc_mnmajor_tile<HD>(q_s, kk), idesc_t, 1);
+            for (int kk = 0; kk < kRows / 16; ++kk) {  // dQ = dS K
+              umma_ss(d + 64, desc_blk_kmajor(bb, kS0h, kZ1, kk), desc_mnmajor_tile<HD>(k_s, kk),
+                      idesc_q, kk);
+              umma_ss(d + 64, desc_blk_kmajor(bb, kS0l, kZ2, kk), desc_mnmajor_tile<HD>(k_s, kk),
+                      idesc_q, 1);
+            }
+#pragma unroll
+            for (int kk = 0; kk < kRows / 16; ++kk) {  // dK = dS^T Q
+              umma_ss(d + 128, desc_blk_mnmajor(bb, kS0h, kZ1, kS1h, kk),
+                      desc_mnmajor_tile<HD>(q_s, kk), idesc_t, kk);
+              umma_ss(d + 128, desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, kk),
+                      desc_mnmajor_tile<HD>(q_s, kk), idesc_t, 1);
+            }
+            umma_commit(&grad_full[sl]);
+            umma_commit(&empty[s]);
+            ++ng;
+            prog = true;
+          }
         }
-        umma_commit(&grad_full[sl]);
-        umma_commit(&empty[s]);
-        if (tn >= p.n_tiles) break;
-        t = tn;
-        ++k;
+        if (prog) {
+          t0 = globaltimer();
+        } else {
+          if (*abort) break;
+          if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicExch(p.status, -5);
+            break;
+          }
+        }
       }
       if (*abort) {
         umma_commit(drain);
@@ -806,40 +830,19 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       }
     }
   } else {
-    const int row = threadIdx.x;
+    const int wg = warp >> 2;
+    const int row = threadIdx.x & (kWg - 1);
     const int gw = row / N, lr = row - gw * N;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float dscale = p.scale_log2 * (1.0f / kLog2e);  // head_dim^-1/2
     const uint32_t bb = smem_u32(blocks);
     const uint32_t blk_ph = bb + (gw ? kP1h : kP0h) * kBlk, blk_pl = bb + (gw ? kP1l : kP0l) * kBlk;
     const uint32_t blk_sh = bb + (gw ? kS1h : kS0h) * kBlk, blk_sl = bb + (gw ? kS1l : kS0l) * kBlk;
-    const int nb = (g.bins + kWg - 1) / kWg;     // table entries owned by this thread
-    long long acc[kAccMax];
-    if (p.acc_local)
-      for (int i = 0; i < kAccMax; ++i) acc[i] = 0;
-    bool pend = false, pvalid = false;
-    long long ptoken = 0, pk = 0;
-    int phead = 0;
-    auto epilogue = [&]() {   // gradients of tile pk (its grad_full already waited)
-      const int sl = (int)(pk % NT);
-      tc_fence_after();
-      float o[HD];
-      const bool st = pvalid && !*abort;
-      const long long off = (ptoken * g.heads + phead) * HD;
-      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 0, o);      // dV
-      tmem_wait_ld();
-      if (st) store_row_bf16<HD>((__nv_bfloat16*)p.out2 + off, o, 1.f);
-      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 64, o);     // dQ
-      tmem_wait_ld();
-      if (st) store_row_bf16<HD>((__nv_bfloat16*)p.out0 + off, o, 1.f);
-      tmem_load_cols<HD>(tmem + lane_base + sl * 256 + 128, o);    // dK
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&t_empty[sl]);
-      if (st) store_row_bf16<HD>((__nv_bfloat16*)p.out1 + off, o, 1.f);
-    };
-    long long k = 0;
-    for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
+    int* bins_hi = bins + wg * 2 * bp;
+    int* bins_lo = bins_hi + bp;
+    long long k = wg;
+    for (long long t = blockIdx.x + wg * (long long)gridDim.x; t < p.n_tiles;
+         t += kNumWg * (long long)gridDim.x, k += kNumWg) {
       const int s = (int)(k % NS), sl = (int)(k % NT);
       const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
       const long long group = t / g.heads;
@@ -847,14 +850,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const long long win = group * G + gw;
       const bool plain = WW > 0 && window_plain(g, win);
       const RowInfo me = plain ? plain_row_info<WW>(g, win, lr) : row_info(g, win, lr);
-      uint32_t* ci = colinfo + (k & 1) * kRows;
+      uint32_t* ci = colinfo + (wg * 2 + ((k / kNumWg) & 1)) * kRows;
       ci[row] = key_word(me);
-      if (named_sync_or(1, kWg, *abort)) break;
+      if (named_sync_or(1 + wg, kWg, *abort)) break;
       if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
       mbar_wait(&sdp_full[sl], pht, abort, p.status, kWaitLimitNs);
       mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
       tc_fence_after();
-      // S row -> P (registers); dP is streamed from TMEM in 32-column chunks,
+      // S row -> P (registers); dP is streamed from TMEM in 16-column chunks,
       // once for D = sum_j P_j dP_j and once for dS, to bound registers.
       float x[N];
       const uint32_t s_col = tmem + lane_base + sl * 256 + gw * N;
@@ -880,80 +883,98 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       // (x = 0 on invalid rows, so D = 0 and dS = 0 there).
       float dd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < N / 32; ++c) {
-        float dp[32];
+      for (int c = 0; c < N / 16; ++c) {
+        float dp[16];
         __syncwarp();
-        tmem_ld32(dp_col + 32 * c, dp);
+        tmem_ld16(dp_col + 16 * c, dp);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dd[j & 3] = fmaf(x[32 * c + j], dp[j], dd[j & 3]);
+        for (int j = 0; j < 16; ++j) dd[j & 3] = fmaf(x[16 * c + j], dp[j], dd[j & 3]);
       }
       const float D = (dd[0] + dd[1]) + (dd[2] + dd[3]);
-      if (pend)   // the MMAs of the previous tile are done with the operand blocks
-        mbar_wait(&grad_full[(int)(pk % NT)], (uint32_t)((pk / NT) & 1), abort, p.status,
-                  kWaitLimitNs);
-      store_split_cols<0, N>(blk_ph, blk_pl, lr, x);
+      if (k > 0)   // the gradient products of tile k-1 are done with the operand blocks
+        mbar_wait(&grad_full[(int)((k - 1) % NT)], (uint32_t)(((k - 1) / NT) & 1), abort,
+                  p.status, kWaitLimitNs);
+      store_split_cols_part<N>(blk_ph, blk_pl, lr, 0, x);
+      // P goes back into this lane's S columns (free until the gradient products
+      // of this tile, which are issued only after the dS loop below) so that the
+      // dS loop streams P and dP in 16-column chunks instead of holding P.
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < N / 32; ++c) tmem_st32(s_col + 32 * c, x + 32 * c);
+      tmem_wait_st();
+      // Large |dS| rows take the two-part fixed-point form (rare).
+      float amax = 0.f;
       int* bqh = bins_hi + me.bias_base;
       int* bql = bins_lo + me.bias_base;
-#pragma unroll
-      for (int c = 0; c < N / 32; ++c) {
-        float ds[32];
+#pragma unroll 1
+      for (int c = 0; c < N / 16; ++c) {
+        float ds[16], pc[16];
         __syncwarp();
-        tmem_ld32(dp_col + 32 * c, ds);
+        tmem_ld16(dp_col + 16 * c, ds);
+        tmem_ld16(s_col + 16 * c, pc);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ds[j] = x[32 * c + j] * (ds[j] - D);   // dS (0 off the row)
+        for (int j = 0; j < 16; ++j) {
+          ds[j] = pc[j] * (ds[j] - D);   // dS (0 off the row)
+          amax = fmaxf(amax, fabsf(ds[j]));
+        }
         if (me.valid) {
           // bias-gradient bins, fixed point: integer adds commute, so the sum
           // is exact and independent of the order the lanes land in
+          if (amax < 64.f) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(32 * c + j)
-                                  : (int)(lds_u32(cw + 32 * c + j) & 0xFFFF);
-            const float t = ds[j] * 256.0f;                 // units of 2^-8
-            const float hf = rintf(t);
-            red_add_s32(bqh - off, __float2int_rn(hf));
-            red_add_s32(bql - off, __float2int_rn((t - hf) * 65536.0f));
+            for (int j = 0; j < 16; ++j) {
+              const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(16 * c + j)
+                                    : (int)(lds_u32(cw + 16 * c + j) & 0xFFFF);
+              red_add_s32(bql - off, round_int_fma(ds[j] * 65536.0f));
+            }
+          } else {
+#pragma unroll 1
+            for (int j = 0; j < 16; ++j) {
+              const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(16 * c + j)
+                                    : (int)(lds_u32(cw + 16 * c + j) & 0xFFFF);
+              const float hf = rintf(ds[j]);
+              red_add_s32(bqh - off, __float2int_rn(hf));
+              red_add_s32(bql - off, round_int_fma((ds[j] - hf) * 65536.0f));
+            }
           }
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ds[j] *= dscale;
-        store_split_cols_part<32>(blk_sh, blk_sl, lr, 32 * c, ds);
+        for (int j = 0; j < 16; ++j) ds[j] *= dscale;
+        store_split_cols_part<16>(blk_sh, blk_sl, lr, 16 * c, ds);
       }
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&pds_full[sl]);
-      // Move this tile's bins into the per-CTA accumulators (or the workspace).
-      named_sync(2, kWg);
-      for (int i = 0; i < nb; ++i) {
-        const int b = row + i * kWg;
-        if (b >= g.bins) break;
-        const long long v = ((long long)bins_hi[b] << 16) + bins_lo[b];   // units of 2^-24
+      // Move this tile's bins into the global int64 table.
+      named_sync(3 + wg, kWg);
+      for (int b = row; b < g.bins; b += kWg) {
+        const long long v = ((long long)bins_hi[b] << 16) + bins_lo[b];   // units of 2^-16
         bins_hi[b] = bins_lo[b] = 0;
-        if (p.acc_local)
-          acc[h * nb + i] += v;
-        else
-          p.partial[(group * g.heads + h) * bp + b] = (float)((double)v * kFixInv);
+        if (v != 0) red_add_global_s64(p.dt_fixed + h * bp + b, v);
       }
-      if (pend) epilogue();
-      pend = true;
-      pvalid = me.valid;
-      ptoken = me.token;
-      phead = h;
-      pk = k;
-    }
-    if (pend) {
-      mbar_wait(&grad_full[(int)(pk % NT)], (uint32_t)((pk / NT) & 1), abort, p.status,
-                kWaitLimitNs);
-      epilogue();
-    }
-    if (p.acc_local) {
-      float* dst = p.partial + (long long)blockIdx.x * g.heads * bp;
-      for (int hh = 0; hh < g.heads; ++hh)
-        for (int i = 0; i < nb; ++i) {
-          const int b = row + i * kWg;
-          if (b < bp) dst[hh * bp + b] = b < g.bins ? (float)((double)acc[hh * nb + i] * kFixInv) : 0.f;
+      // epilogue: dV, dQ, dK rows from TMEM straight to their grid token
+      mbar_wait(&grad_full[sl], pht, abort, p.status, kWaitLimitNs);
+      tc_fence_after();
+      const bool st = me.valid && !*abort;
+      const long long off = (me.token * g.heads + h) * HD;
+#pragma unroll
+      for (int part = 0; part < 3; ++part) {
+        __nv_bfloat16* dst = (__nv_bfloat16*)(part == 0 ? p.out2 : (part == 1 ? p.out0 : p.out1)) + off;
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          float o[32];
+          __syncwarp();
+          tmem_ld32(tmem + lane_base + sl * 256 + part * 64 + 32 * c, o);
+          tmem_wait_ld();
+          if (part == 2 && c == HD / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(&t_empty[sl]);
+          }
+          if (st) store_row_bf16<32>(dst + 32 * c, o, 1.f);
         }
+      }
     }
   }
   tc_fence_before();
@@ -964,13 +985,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   }
 }
 
-// Bias table transposed to [heads][bins_pad] and scaled by log2(e).
+// Bias table transposed to [heads][bins_pad] and scaled by log2(e); clears
+// the fixed-point bias-gradient table when one is given.
 __global__ void bias_prep_kernel(const float* __restrict__ table, int bins, int heads,
-                                 int bins_pad, float* __restrict__ out) {
+                                 int bins_pad, float* __restrict__ out,
+                                 long long* __restrict__ dt_fixed) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= heads * bins_pad) return;
   const int h = i / bins_pad, b = i - h * bins_pad;
   out[i] = b < bins ? table[b * heads + h] * kLog2e : 0.f;
+  if (dt_fixed) dt_fixed[i] = 0;
+}
+
+// dtable[bin][h] = fixed-point sum [h][bin] * 2^-16.
+__global__ void dbias_finish_kernel(const long long* __restrict__ dt_fixed, int bins, int heads,
+                                    int bins_pad, float* __restrict__ dtable) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= bins * heads) return;
+  const int b = i / heads, h = i - b * heads;
+  dtable[i] = (float)((double)dt_fixed[h * bins_pad + b] * kFixInv);
 }
 
 // ================================================================================
@@ -1053,11 +1086,6 @@ bool smem_ok(const Geo& g) {
   return f <= kSmemLimit && b <= kSmemLimit;
 }
 
-// Bias-gradient sums per CTA in thread-local memory when every thread's share
-// (its table entries for all heads) fits; per tile in the workspace otherwise.
-int acc_mode(const Geo& g) {
-  return (long long)g.heads * ((g.bins + kWg - 1) / kWg) <= kAccMax ? 1 : 0;
-}
 
 void fill_common(FastParams& p, const Geo& g, const float* bias_t, int* status, int flags) {
   memset(&p, 0, sizeof(p));
@@ -1082,10 +1110,11 @@ cudaError_t launch(K kernel, const FastParams& p, size_t smem, cudaStream_t st) 
   return cudaGetLastError();
 }
 
-cudaError_t prep_bias(const Geo& g, const float* table, float* bias_t, cudaStream_t st) {
+cudaError_t prep_bias(const Geo& g, const float* table, float* bias_t, long long* dt_fixed,
+                      cudaStream_t st) {
   const int n = g.heads * bins_padded(g.bins);
   bias_prep_kernel<<<(n + 255) / 256, 256, 0, st>>>(table, g.bins, g.heads, bins_padded(g.bins),
-                                                    bias_t);
+                                                    bias_t, dt_fixed);
   note_launch();
   return cudaGetLastError();
 }
@@ -1108,13 +1137,11 @@ bool fast_supported(const Geo& g, int dtype) {
   return smem_ok(g);
 }
 
+// Workspace: header (status word), bias table [heads][bins_pad] fp32, and the
+// fixed-point bias gradient [heads][bins_pad] int64.
 size_t fast_workspace(const Geo& g) {
   const int bp = bins_padded(g.bins);
-  const int G = kRows / g.N;
-  const long long groups = (g.n_win + G - 1) / G;
-  const size_t per_tile = (size_t)groups * g.heads * bp * 4;
-  const size_t per_cta = (size_t)1024 * g.heads * bp * 4;  // any grid up to 1024 CTAs
-  return kWsHeader + align256((size_t)g.heads * bp * 4) + align256(per_tile > per_cta ? per_tile : per_cta);
+  return kWsHeader + align256((size_t)g.heads * bp * 4) + align256((size_t)g.heads * bp * 8);
 }
 
 cudaError_t fast_forward(const Geo& g, const void* q, const void* k, const void* v,
@@ -1127,7 +1154,7 @@ cudaError_t fast_forward(const Geo& g, const void* q, const void* k, const void*
   p.lse = lse;
   if (!encode_maps(p, 0, q) || !encode_maps(p, 1, k) || !encode_maps(p, 2, v))
     return cudaErrorInvalidValue;
-  cudaError_t e = prep_bias(g, table, bias_t, st);
+  cudaError_t e = prep_bias(g, table, bias_t, nullptr, st);
   if (e != cudaSuccess) return e;
   const bool w8 = g.wh == 8 && g.ww == 8;
   if (g.hd == 64)
@@ -1141,18 +1168,18 @@ cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void
                           const float* table, const void* dout, void* dq, void* dk, void* dv,
                           float* dtable, void* ws, int flags, cudaStream_t st) {
   float* bias_t = (float*)((char*)ws + kWsHeader);
-  float* partial = (float*)((char*)ws + kWsHeader + align256((size_t)g.heads * bins_padded(g.bins) * 4));
+  long long* dt_fixed =
+      (long long*)((char*)ws + kWsHeader + align256((size_t)g.heads * bins_padded(g.bins) * 4));
   static thread_local FastParams p;
   fill_common(p, g, bias_t, (int*)ws, flags);
   p.out0 = dq;
   p.out1 = dk;
   p.out2 = dv;
-  p.partial = partial;
-  p.acc_local = acc_mode(g);
+  p.dt_fixed = dt_fixed;
   if (!encode_maps(p, 0, q) || !encode_maps(p, 1, k) || !encode_maps(p, 2, v) ||
       !encode_maps(p, 3, dout))
     return cudaErrorInvalidValue;
-  cudaError_t e = prep_bias(g, table, bias_t, st);
+  cudaError_t e = prep_bias(g, table, bias_t, dt_fixed, st);
   if (e != cudaSuccess) return e;
   const size_t smem = g.hd == 64 ? bwd_smem<64>(g) : bwd_smem<32>(g);
   const bool w8 = g.wh == 8 && g.ww == 8;
@@ -1161,8 +1188,11 @@ cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void
   else
     e = w8 ? launch(bwd_kernel<32, 8>, p, smem, st) : launch(bwd_kernel<32, 0>, p, smem, st);
   if (e != cudaSuccess) return e;
-  const long long grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
-  return dbias_reduce(g, partial, p.acc_local ? grid : p.n_groups, dtable, st);
+  const int n = g.bins * g.heads;
+  dbias_finish_kernel<<<(n + 255) / 256, 256, 0, st>>>(dt_fixed, g.bins, g.heads,
+                                                       bins_padded(g.bins), dtable);
+  note_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace swin
