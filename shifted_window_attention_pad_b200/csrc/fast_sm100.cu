@@ -32,9 +32,11 @@
 //    Integer sums are exact and do not depend on the order in which threads or
 //    CTAs land, so the result is bitwise repeatable; a last small kernel
 //    converts it to fp32.
-//  * Warp roles: warps 0-3 softmax/epilogue, warp 4 TMA producer, warp 5 MMA
-//    issuer and TMEM owner. Persistent grid of one CTA per SM; tiles go
-//    round-robin, head fastest, so the SMs stream neighbouring bytes together.
+//  * Warp roles: warps 0-3 and 4-7 two softmax/epilogue warpgroups taking
+//    alternate tiles, warp 8 TMA producer, warp 9 issues S (and dP) and owns
+//    TMEM, warp 10 issues PV (or the gradient products). Persistent grid of one
+//    CTA per SM; tiles go round-robin, head fastest, so the SMs stream
+//    neighbouring bytes together.
 //  * Every mbarrier wait is bounded (%globaltimer); a wait that runs out records
 //    a timeout in the workspace status word and the kernel drains and returns.
 #include <cuda.h>
@@ -57,8 +59,9 @@ constexpr int kRows = 128;        // tile rows = TMEM lanes = UMMA M
 constexpr int kWg = 128;          // threads of one softmax / epilogue warpgroup
 constexpr int kNumWg = 2;         // warpgroups 0 (warps 0-3) and 1 (warps 4-7) alternate tiles
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kMmaWarp = 9;       // issues S (and dP); allocates and frees TMEM
+constexpr int kMma2Warp = 10;     // issues PV (forward) or the gradient products (backward)
+constexpr int kThreads = 352;
 constexpr int kMaxMaps = 9;       // box shapes: {full, seam part 1, seam part 2}^2
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestLimitNs = 1000000ull;
@@ -66,6 +69,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct FastParams {
   CUtensorMap maps[4][kMaxMaps];  // [q, k, v, dout][ky * 3 + kx]
+  CUtensorMap omaps[3][kMaxMaps]; // outputs: forward [out]; backward [dq, dk, dv]
   Geo g;
   long long n_groups;             // tiles per head: ceil(n_win / G)
   long long n_tiles;              // n_groups * heads
@@ -239,6 +243,81 @@ __device__ inline void issue_tile_loads(const FastParams& p, long long t, uint8_
   bulk_load(bias_dst, p.bias_t + (size_t)h * p.bins_pad, p.bins_pad * 4, full);
 }
 
+// One elected thread: TMA-stores the staged output rows of tile `t` with the
+// same sub-box decomposition as the loads, for NOUT tensors. Window gw of
+// tensor tt is staged at staged + tt * tile_stride + gw * win_stride, rows of
+// HD bf16 back to back in sub-box order. Sub-boxes wholly in the padding are
+// skipped; the others are clipped to the grid by the TMA unit.
+template <int HD, int NOUT>
+__device__ inline void issue_tile_stores(const FastParams& p, long long t, const uint8_t* staged,
+                                         uint32_t tile_stride, uint32_t win_stride) {
+  const Geo& g = p.g;
+  const int G = kRows / g.N;
+  const long long group = t / g.heads;
+  const int h = (int)(t - group * g.heads);
+  constexpr uint32_t row_bytes = HD * 2;
+  for (int gw = 0; gw < G; ++gw) {
+    const long long win = group * G + gw;
+    if (win >= g.n_win) continue;
+    int b, wy, wx;
+    window_coords(g, win, b, wy, wx);
+    SubBox sb[4];
+    const int n = plan_window(g, wy, wx, sb);
+    for (int i = 0; i < n; ++i) {
+      if (sb[i].y >= g.H || sb[i].x >= g.W) continue;
+      for (int tt = 0; tt < NOUT; ++tt)
+        tma_store_5d(&p.omaps[tt][sb[i].map_id],
+                     staged + tt * tile_stride + gw * win_stride + sb[i].row_off * row_bytes, 0,
+                     h, sb[i].x, sb[i].y, b);
+    }
+  }
+  bulk_commit_group();
+}
+
+// The same for the three backward outputs staged in the operand-block area
+// (dV at bwd_stage(0), dQ at bwd_stage(1), dK at bwd_stage(2)).
+__host__ __device__ constexpr uint32_t bwd_stage(int part);
+template <int HD>
+__device__ inline void issue_tile_stores3(const FastParams& p, long long t, const uint8_t* staged) {
+  const Geo& g = p.g;
+  const int G = kRows / g.N;
+  const long long group = t / g.heads;
+  const int h = (int)(t - group * g.heads);
+  constexpr uint32_t row_bytes = HD * 2;
+  for (int gw = 0; gw < G; ++gw) {
+    const long long win = group * G + gw;
+    if (win >= g.n_win) continue;
+    int b, wy, wx;
+    window_coords(g, win, b, wy, wx);
+    SubBox sb[4];
+    const int n = plan_window(g, wy, wx, sb);
+    for (int i = 0; i < n; ++i) {
+      if (sb[i].y >= g.H || sb[i].x >= g.W) continue;
+      const uint32_t r = (gw * g.N + sb[i].row_off) * row_bytes;
+      tma_store_5d(&p.omaps[0][sb[i].map_id], staged + bwd_stage(1) + r, 0, h, sb[i].x, sb[i].y, b);
+      tma_store_5d(&p.omaps[1][sb[i].map_id], staged + bwd_stage(2) + r, 0, h, sb[i].x, sb[i].y, b);
+      tma_store_5d(&p.omaps[2][sb[i].map_id], staged + bwd_stage(0) + r, 0, h, sb[i].x, sb[i].y, b);
+    }
+  }
+  bulk_commit_group();
+}
+
+// Stages one output row of HD values (times `mul`, rounded to bf16) at
+// row_addr, with the tensor maps' swizzle (128-byte for HD = 64, 64-byte for
+// HD = 32: 16-byte chunk index XOR address bits 7.., on a 1024-aligned buffer).
+template <int HD>
+__device__ inline void stage_row(uint32_t row_addr, const float* v, float mul) {
+#pragma unroll
+  for (int c = 0; c < HD / 8; ++c) {
+    const uint32_t off = row_addr + c * 16;
+    const uint32_t swz = HD == 64 ? ((off >> 7) & 7) : ((off >> 7) & 3);
+    st_shared_v4(off ^ (swz << 4), pack_bf16(v[c * 8 + 0] * mul, v[c * 8 + 1] * mul),
+                 pack_bf16(v[c * 8 + 2] * mul, v[c * 8 + 3] * mul),
+                 pack_bf16(v[c * 8 + 4] * mul, v[c * 8 + 5] * mul),
+                 pack_bf16(v[c * 8 + 6] * mul, v[c * 8 + 7] * mul));
+  }
+}
+
 // K-major operand, rows of HD bf16 (128-byte swizzle for HD = 64, 64-byte for 32),
 // advanced by k16 steps of 16 elements along K.
 template <int HD>
@@ -386,13 +465,14 @@ __device__ inline float exp_sum(float* x, float m) {
 // Per tile: S = Q K^T (MMA) -> softmax row per thread -> P (bf16, smem) ->
 // O = P V (MMA) -> normalise and store. Two warpgroups take alternate tiles, so
 // while one waits on TMEM loads or an MMA the other computes (two warps per
-// scheduler). The MMA warp polls: it issues S of the next tile as soon as its
-// data and TMEM slot are ready and PV of a tile as soon as its P is written.
+// scheduler). One thread issues S of each tile as soon as its data and TMEM
+// slot are ready, another PV as soon as its P is written.
 // Four TMEM slots of 128 columns (S, then O in the first HD), one P tile per
 // warpgroup, three input stages.
 constexpr int kFwdStages = 3;
 constexpr int kFwdSlots = 4;
 constexpr int kFwdPBufs = kNumWg;
+
 
 // Number of tiles CTA `cta` takes in a grid of `grid` CTAs.
 __device__ inline long long local_tiles(long long n_tiles, long long cta, long long grid) {
@@ -419,8 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   uint64_t* p_full = s_full + NT;
   uint64_t* o_full = p_full + NT;
   uint64_t* t_empty = o_full + NT;
-  uint64_t* drain = t_empty + NT;
-  uint64_t* never = drain + 1;
+  uint64_t* drain = t_empty + NT;   // [2]: one per MMA-issuing thread
+  uint64_t* never = drain + 2;
   uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
   volatile int* abort = (volatile int*)(smem + L.misc + 4);
 
@@ -432,7 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       mbar_init(&s_full[i], 1); mbar_init(&p_full[i], kWg);
       mbar_init(&o_full[i], 1); mbar_init(&t_empty[i], kWg);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     mbar_init(never, 1);
     *abort = 0;
     fence_mbar_init();
@@ -470,59 +551,48 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       }
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
+    if (lane == 0) {   // S = Q K^T of every tile, as soon as its data and TMEM slot are ready
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);
-      constexpr uint32_t idesc_o = idesc_bf16(kRows, HD, 0, 1);
-      long long ns = 0, np = 0;               // next S to issue, next PV to issue
-      uint64_t t0 = globaltimer();
-      while (np < n_local) {
-        bool prog = false;
-        if (ns < n_local) {
-          const int s = (int)(ns % NS), sl = (int)(ns % NT);
-          if (mbar_test(&full[s], (uint32_t)((ns / NS) & 1)) &&
-              mbar_test(&t_empty[sl], (uint32_t)(((ns / NT) & 1) ^ 1))) {
-            tc_fence_after();
-            const uint32_t q_s = smem_u32(tiles + (s * 3 + 0) * tile_bytes);
-            const uint32_t k_s = smem_u32(tiles + (s * 3 + 1) * tile_bytes);
+      for (long long k = 0; k < n_local; ++k) {
+        const int s = (int)(k % NS), sl = (int)(k % NT);
+        if (!mbar_wait(&full[s], (uint32_t)((k / NS) & 1), abort, p.status, kWaitLimitNs)) break;
+        if (!mbar_wait(&t_empty[sl], (uint32_t)(((k / NT) & 1) ^ 1), abort, p.status,
+                       kWaitLimitNs))
+          break;
+        tc_fence_after();
+        const uint32_t q_s = smem_u32(tiles + (s * 3 + 0) * tile_bytes);
+        const uint32_t k_s = smem_u32(tiles + (s * 3 + 1) * tile_bytes);
 #pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk)
-              umma_ss(tmem + sl * 128, desc_kmajor_tile<HD>(q_s, kk),
-                      desc_kmajor_tile<HD>(k_s, kk), idesc_s, kk);
-            umma_commit(&s_full[sl]);
-            ++ns;
-            prog = true;
-          }
-        }
-        if (np < ns) {
-          const int s = (int)(np % NS), sl = (int)(np % NT);
-          if (mbar_test(&p_full[sl], (uint32_t)((np / NT) & 1))) {
-            tc_fence_after();
-            const uint32_t v_s = smem_u32(tiles + (s * 3 + 2) * tile_bytes);
-            const uint32_t p_s = smem_u32(ptile + (np % kFwdPBufs) * 32768);
-#pragma unroll
-            for (int kk = 0; kk < kRows / 16; ++kk)
-              umma_ss(tmem + sl * 128, desc_p_kmajor(p_s, kk), desc_mnmajor_tile<HD>(v_s, kk),
-                      idesc_o, kk);
-            umma_commit(&o_full[sl]);
-            umma_commit(&empty[s]);
-            ++np;
-            prog = true;
-          }
-        }
-        if (prog) {
-          t0 = globaltimer();
-        } else {
-          if (*abort) break;
-          if (globaltimer() - t0 > kWaitLimitNs) {
-            *abort = 1;
-            atomicExch(p.status, -5);
-            break;
-          }
-        }
+        for (int kk = 0; kk < HD / 16; ++kk)
+          umma_ss(tmem + sl * 128, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk),
+                  idesc_s, kk);
+        umma_commit(&s_full[sl]);
       }
       if (*abort) {
-        umma_commit(drain);
-        mbar_drain(drain, 0, kTestLimitNs * 100);
+        umma_commit(&drain[0]);
+        mbar_drain(&drain[0], 0, kTestLimitNs * 100);
+      }
+    }
+  } else if (warp == kMma2Warp) {
+    if (lane == 0) {   // O = P V of every tile, as soon as its P is written
+      constexpr uint32_t idesc_o = idesc_bf16(kRows, HD, 0, 1);
+      for (long long k = 0; k < n_local; ++k) {
+        const int s = (int)(k % NS), sl = (int)(k % NT);
+        if (!mbar_wait(&p_full[sl], (uint32_t)((k / NT) & 1), abort, p.status, kWaitLimitNs))
+          break;
+        tc_fence_after();
+        const uint32_t v_s = smem_u32(tiles + (s * 3 + 2) * tile_bytes);
+        const uint32_t p_s = smem_u32(ptile + (k % kFwdPBufs) * 32768);
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          umma_ss(tmem + sl * 128, desc_p_kmajor(p_s, kk), desc_mnmajor_tile<HD>(v_s, kk),
+                  idesc_o, kk);
+        umma_commit(&o_full[sl]);
+        umma_commit(&empty[s]);
+      }
+      if (*abort) {
+        umma_commit(&drain[1]);
+        mbar_drain(&drain[1], 0, kTestLimitNs * 100);
       }
     }
   } else {
@@ -570,24 +640,20 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       tc_fence_before();
       mbar_arrive(&p_full[sl]);
       // epilogue: O row from TMEM, normalised, straight to its grid token
+      // (direct stores measured faster here than staging for a TMA store)
       mbar_wait(&o_full[sl], pht, abort, p.status, kWaitLimitNs);
       tc_fence_after();
-      const bool st = me.valid && !*abort;
-      const float inv = 1.f / l;
-      __nv_bfloat16* dst = (__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD;
-#pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        float o[32];
-        __syncwarp();
-        tmem_ld32(tmem + lane_base + sl * 128 + 32 * c, o);
+      {
+        float o[HD];
+        tmem_load_cols<HD>(tmem + lane_base + sl * 128, o);
         tmem_wait_ld();
-        if (c == HD / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(&t_empty[sl]);
-        }
-        if (st) store_row_bf16<32>(dst + 32 * c, o, inv);
+        tc_fence_before();
+        mbar_arrive(&t_empty[sl]);
+        if (me.valid && !*abort)
+          store_row_bf16<HD>((__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD, o, 1.f / l);
       }
-      if (st && p.lse) p.lse[me.token * g.heads + h] = (m + __log2f(l)) * 0.69314718055994531f;
+      if (me.valid && !*abort && p.lse)
+        p.lse[me.token * g.heads + h] = (m + __log2f(l)) * 0.69314718055994531f;
     }
   }
   tc_fence_before();
@@ -617,8 +683,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 //
 // Two warpgroups take alternate tiles, each with its own TMEM slot of 256
 // columns (S | dP, then dV | dQ | dK). The operand blocks are shared: tile k
-// writes them once the gradient products of tile k-1 have completed. The MMA
-// warp polls: S and dP of a tile go out as soon as its data and slot are ready,
+// writes them once the gradient products of tile k-1 have completed. One thread
+// issues S and dP of each tile as soon as its data and slot are ready, another
 // the gradient products as soon as its blocks are written.
 constexpr int kBwdStages = 2;
 constexpr int kBwdSlots = 2;
@@ -629,6 +695,12 @@ enum { kP0h = 0, kP0l, kS0h, kZ1, kS1h, kS0l, kZ2, kS1l, kP1h, kP1l, kNumBlk };
 // split into an integer high part and a low remainder. A tile's bins hold at
 // most 128 terms, so neither part can overflow; the global table is int64.
 constexpr double kFixInv = 1.52587890625e-05;  // 2^-16
+// Output staging in the operand-block area, clear of the zero blocks Z1
+// (24-32 KB) and Z2 (48-56 KB): dV at 0, dQ at 32 KB, dK at 56 KB, each
+// 128 rows of HD bf16.
+__host__ __device__ constexpr uint32_t bwd_stage(int part) {
+  return part == 0 ? 0u : (part == 1 ? 32768u : 57344u);
+}
 
 __device__ inline uint64_t desc_blk_kmajor(uint32_t base, int blk0, int blk1, int k16) {
   // keys [0,64) read the run starting at blk0, keys [64,128) the run at blk1
@@ -693,8 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint64_t* pds_full = sdp_full + NT;
   uint64_t* grad_full = pds_full + NT;
   uint64_t* t_empty = grad_full + NT;
-  uint64_t* drain = t_empty + NT;
-  uint64_t* never = drain + 1;
+  uint64_t* drain = t_empty + NT;   // [2]: one per MMA-issuing thread
+  uint64_t* never = drain + 2;
+  uint64_t* blk_free = never + 1;   // operand-block area free of staged outputs
   uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
   volatile int* abort = (volatile int*)(smem + L.misc + 4);
 
@@ -706,8 +779,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       mbar_init(&sdp_full[i], 1); mbar_init(&pds_full[i], kWg);
       mbar_init(&grad_full[i], 1); mbar_init(&t_empty[i], kWg);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     mbar_init(never, 1);
+    mbar_init(blk_free, 1);
     *abort = 0;
     fence_mbar_init();
   }
@@ -746,87 +821,75 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       }
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);      // S, dP
+    if (lane == 0) {   // S = Q K^T and dP = dO V^T of every tile
+      constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);
+      for (long long k = 0; k < n_local; ++k) {
+        const int s = (int)(k % NS), sl = (int)(k % NT);
+        if (!mbar_wait(&full[s], (uint32_t)((k / NS) & 1), abort, p.status, kWaitLimitNs)) break;
+        if (!mbar_wait(&t_empty[sl], (uint32_t)(((k / NT) & 1) ^ 1), abort, p.status,
+                       kWaitLimitNs))
+          break;
+        tc_fence_after();
+        const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
+        const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
+        const uint32_t v_s = smem_u32(tiles + (s * 4 + 2) * tile_bytes);
+        const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
+        const uint32_t d = tmem + sl * 256;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          umma_ss(d, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk), idesc_s, kk);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          umma_ss(d + 128, desc_kmajor_tile<HD>(do_s, kk), desc_kmajor_tile<HD>(v_s, kk), idesc_s,
+                  kk);
+        umma_commit(&sdp_full[sl]);
+      }
+      if (*abort) {
+        umma_commit(&drain[0]);
+        mbar_drain(&drain[0], 0, kTestLimitNs * 100);
+      }
+    }
+  } else if (warp == kMma2Warp) {
+    if (lane == 0) {   // dV, dQ, dK of every tile, once its operand blocks are written
       constexpr uint32_t idesc_t = idesc_bf16(kRows, HD, 1, 1);         // dV, dK: A = X^T
       constexpr uint32_t idesc_q = idesc_bf16(kRows, HD, 0, 1);         // dQ
       const uint32_t bb = smem_u32(blocks);
-      long long ns = 0, ng = 0;               // next S/dP to issue, next gradient products
-      uint64_t t0 = globaltimer();
-      while (ng < n_local) {
-        bool prog = false;
-        if (ns < n_local) {
-          const int s = (int)(ns % NS), sl = (int)(ns % NT);
-          if (mbar_test(&full[s], (uint32_t)((ns / NS) & 1)) &&
-              mbar_test(&t_empty[sl], (uint32_t)(((ns / NT) & 1) ^ 1))) {
-            tc_fence_after();
-            const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
-            const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
-            const uint32_t v_s = smem_u32(tiles + (s * 4 + 2) * tile_bytes);
-            const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
-            const uint32_t d = tmem + sl * 256;
+      for (long long k = 0; k < n_local; ++k) {
+        const int s = (int)(k % NS), sl = (int)(k % NT);
+        if (!mbar_wait(&pds_full[sl], (uint32_t)((k / NT) & 1), abort, p.status, kWaitLimitNs))
+          break;
+        tc_fence_after();
+        const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
+        const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
+        const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
+        const uint32_t d = tmem + sl * 256;
 #pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk)
-              umma_ss(d, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk), idesc_s,
-                      kk);
-#pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk)
-              umma_ss(d + 128, desc_kmajor_tile<HD>(do_s, kk), desc_kmajor_tile<HD>(v_s, kk),
-                      idesc_s, kk);
-            umma_commit(&sdp_full[sl]);
-            ++ns;
-            prog = true;
-          }
+        for (int kk = 0; kk < kRows / 16; ++kk) {  // dV = P^T dO  (hi, then lo)
+          umma_ss(d + 0, desc_blk_mnmajor(bb, kP0h, kZ1, kP1h, kk),
+                  desc_mnmajor_tile<HD>(do_s, kk), idesc_t, kk);
+          umma_ss(d + 0, desc_blk_mnmajor(bb, kP0l, kZ1, kP1l, kk),
+                  desc_mnmajor_tile<HD>(do_s, kk), idesc_t, 1);
         }
-        if (ng < ns) {
-          const int s = (int)(ng % NS), sl = (int)(ng % NT);
-          if (mbar_test(&pds_full[sl], (uint32_t)((ng / NT) & 1))) {
-            tc_fence_after();
-            const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
-            const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
-            const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
-            const uint32_t d = tmem + sl * 256;
 #pragma unroll
-            for (int kk = 0; kk < kRows / 16; ++kk) {  // dV = P^T dO  (hi, then lo)
-              umma_ss(d + 0, desc_blk_mnmajor(bb, kP0h, kZ1, kP1h, kk),
-                      desc_mnmajor_tile<HD>(do_s, kk), idesc_t, kk);
-              umma_ss(d + 0, desc_blk_mnmajor(bb, kP0l, kZ1, kP1l, kk),
-                      desc_mnmajor_tile<HD>(do_s, kk), idesc_t, 1);
-            }
-#pragma unroll
-            for (int kk = 0; kk < kRows / 16; ++kk) {  // dQ = dS K
-              umma_ss(d + 64, desc_blk_kmajor(bb, kS0h, kZ1, kk), desc_mnmajor_tile<HD>(k_s, kk),
-                      idesc_q, kk);
-              umma_ss(d + 64, desc_blk_kmajor(bb, kS0l, kZ2, kk), desc_mnmajor_tile<HD>(k_s, kk),
-                      idesc_q, 1);
-            }
-#pragma unroll
-            for (int kk = 0; kk < kRows / 16; ++kk) {  // dK = dS^T Q
-              umma_ss(d + 128, desc_blk_mnmajor(bb, kS0h, kZ1, kS1h, kk),
-                      desc_mnmajor_tile<HD>(q_s, kk), idesc_t, kk);
-              umma_ss(d + 128, desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, kk),
-                      desc_mnmajor_tile<HD>(q_s, kk), idesc_t, 1);
-            }
-            umma_commit(&grad_full[sl]);
-            umma_commit(&empty[s]);
-            ++ng;
-            prog = true;
-          }
+        for (int kk = 0; kk < kRows / 16; ++kk) {  // dQ = dS K
+          umma_ss(d + 64, desc_blk_kmajor(bb, kS0h, kZ1, kk), desc_mnmajor_tile<HD>(k_s, kk),
+                  idesc_q, kk);
+          umma_ss(d + 64, desc_blk_kmajor(bb, kS0l, kZ2, kk), desc_mnmajor_tile<HD>(k_s, kk),
+                  idesc_q, 1);
         }
-        if (prog) {
-          t0 = globaltimer();
-        } else {
-          if (*abort) break;
-          if (globaltimer() - t0 > kWaitLimitNs) {
-            *abort = 1;
-            atomicExch(p.status, -5);
-            break;
-          }
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk) {  // dK = dS^T Q
+          umma_ss(d + 128, desc_blk_mnmajor(bb, kS0h, kZ1, kS1h, kk),
+                  desc_mnmajor_tile<HD>(q_s, kk), idesc_t, kk);
+          umma_ss(d + 128, desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, kk),
+                  desc_mnmajor_tile<HD>(q_s, kk), idesc_t, 1);
         }
+        umma_commit(&grad_full[sl]);
+        umma_commit(&empty[s]);
       }
       if (*abort) {
-        umma_commit(drain);
-        mbar_drain(drain, 0, kTestLimitNs * 100);
+        umma_commit(&drain[1]);
+        mbar_drain(&drain[1], 0, kTestLimitNs * 100);
       }
     }
   } else {
@@ -857,8 +920,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       mbar_wait(&sdp_full[sl], pht, abort, p.status, kWaitLimitNs);
       mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
       tc_fence_after();
-      // S row -> P (registers); dP is streamed from TMEM in 16-column chunks,
-      // once for D = sum_j P_j dP_j and once for dS, to bound registers.
+      // S row -> P (registers) -> D from dP; P back into its S columns; dS and
+      // the bias-gradient bins from P and dP chunks; scale * dS into the dP
+      // columns. All of this runs before the shared operand blocks are free.
       float x[N];
       const uint32_t s_col = tmem + lane_base + sl * 256 + gw * N;
       const uint32_t dp_col = s_col + 128;
@@ -882,23 +946,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       // TMEM loads are warp-collective: every lane runs them, valid row or not
       // (x = 0 on invalid rows, so D = 0 and dS = 0 there).
       float dd[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < N / 16; ++c) {
-        float dp[16];
-        __syncwarp();
-        tmem_ld16(dp_col + 16 * c, dp);
+      {
+        float dp[N];
+        tmem_load_cols<N>(dp_col, dp);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) dd[j & 3] = fmaf(x[16 * c + j], dp[j], dd[j & 3]);
+        for (int j = 0; j < N; ++j) dd[j & 3] = fmaf(x[j], dp[j], dd[j & 3]);
       }
       const float D = (dd[0] + dd[1]) + (dd[2] + dd[3]);
-      if (k > 0)   // the gradient products of tile k-1 are done with the operand blocks
-        mbar_wait(&grad_full[(int)((k - 1) % NT)], (uint32_t)(((k - 1) / NT) & 1), abort,
-                  p.status, kWaitLimitNs);
-      store_split_cols_part<N>(blk_ph, blk_pl, lr, 0, x);
-      // P goes back into this lane's S columns (free until the gradient products
-      // of this tile, which are issued only after the dS loop below) so that the
-      // dS loop streams P and dP in 16-column chunks instead of holding P.
       __syncwarp();
 #pragma unroll
       for (int c = 0; c < N / 32; ++c) tmem_st32(s_col + 32 * c, x + 32 * c);
@@ -908,14 +963,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       int* bqh = bins_hi + me.bias_base;
       int* bql = bins_lo + me.bias_base;
 #pragma unroll 1
-      for (int c = 0; c < N / 16; ++c) {
-        float ds[16], pc[16];
+      for (int c = 0; c < N / 32; ++c) {
+        float ds[32], pc[32];
         __syncwarp();
-        tmem_ld16(dp_col + 16 * c, ds);
-        tmem_ld16(s_col + 16 * c, pc);
+        tmem_ld32(dp_col + 32 * c, ds);
+        tmem_ld32(s_col + 32 * c, pc);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 32; ++j) {
           ds[j] = pc[j] * (ds[j] - D);   // dS (0 off the row)
           amax = fmaxf(amax, fabsf(ds[j]));
         }
@@ -924,16 +979,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           // is exact and independent of the order the lanes land in
           if (amax < 64.f) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(16 * c + j)
-                                    : (int)(lds_u32(cw + 16 * c + j) & 0xFFFF);
+            for (int j = 0; j < 32; ++j) {
+              const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(32 * c + j)
+                                    : (int)(lds_u32(cw + 32 * c + j) & 0xFFFF);
               red_add_s32(bql - off, round_int_fma(ds[j] * 65536.0f));
             }
-          } else {
-#pragma unroll 1
-            for (int j = 0; j < 16; ++j) {
-              const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(16 * c + j)
-                                    : (int)(lds_u32(cw + 16 * c + j) & 0xFFFF);
+          } else {   // (unrolled: a runtime index would put ds in local memory)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(32 * c + j)
+                                    : (int)(lds_u32(cw + 32 * c + j) & 0xFFFF);
               const float hf = rintf(ds[j]);
               red_add_s32(bqh - off, __float2int_rn(hf));
               red_add_s32(bql - off, round_int_fma((ds[j] - hf) * 65536.0f));
@@ -941,8 +996,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           }
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) ds[j] *= dscale;
-        store_split_cols_part<16>(blk_sh, blk_sl, lr, 16 * c, ds);
+        for (int j = 0; j < 32; ++j) ds[j] *= dscale;
+        __syncwarp();
+        tmem_st32(dp_col + 32 * c, ds);
+      }
+      tmem_wait_st();
+      // The operand blocks are free once the previous tile's outputs, staged
+      // there, have been read out by its TMA stores.
+      if (k > 0)
+        mbar_wait(blk_free, (uint32_t)((k - 1) & 1), abort, p.status, kWaitLimitNs);
+#pragma unroll 1
+      for (int c = 0; c < N / 32; ++c) {
+        float pc[32], ds[32];
+        __syncwarp();
+        tmem_ld32(s_col + 32 * c, pc);
+        tmem_ld32(dp_col + 32 * c, ds);
+        tmem_wait_ld();
+        store_split_cols_part<32>(blk_ph, blk_pl, lr, 32 * c, pc);
+        store_split_cols_part<32>(blk_sh, blk_sl, lr, 32 * c, ds);
       }
       fence_proxy_async();
       tc_fence_before();
@@ -954,28 +1025,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         bins_hi[b] = bins_lo[b] = 0;
         if (v != 0) red_add_global_s64(p.dt_fixed + h * bp + b, v);
       }
-      // epilogue: dV, dQ, dK rows from TMEM straight to their grid token
+      // epilogue: dV, dQ, dK rows from TMEM, staged in the operand-block area
+      // (free of readers once the gradient products are done), TMA-stored to
+      // grid order by one thread, which then frees the area for the next tile.
       mbar_wait(&grad_full[sl], pht, abort, p.status, kWaitLimitNs);
       tc_fence_after();
-      const bool st = me.valid && !*abort;
-      const long long off = (me.token * g.heads + h) * HD;
 #pragma unroll
       for (int part = 0; part < 3; ++part) {
-        __nv_bfloat16* dst = (__nv_bfloat16*)(part == 0 ? p.out2 : (part == 1 ? p.out0 : p.out1)) + off;
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          float o[32];
-          __syncwarp();
-          tmem_ld32(tmem + lane_base + sl * 256 + part * 64 + 32 * c, o);
-          tmem_wait_ld();
-          if (part == 2 && c == HD / 32 - 1) {
-            tc_fence_before();
-            mbar_arrive(&t_empty[sl]);
-          }
-          if (st) store_row_bf16<32>(dst + 32 * c, o, 1.f);
+        float o[HD];
+        tmem_load_cols<HD>(tmem + lane_base + sl * 256 + part * 64, o);
+        tmem_wait_ld();
+        if (part == 2) {
+          tc_fence_before();
+          mbar_arrive(&t_empty[sl]);
         }
+        stage_row<HD>(bb + bwd_stage(part) + (gw * N + lr) * (HD * 2), o, 1.f);
+      }
+      fence_proxy_async();
+      named_sync(3 + wg, kWg);
+      if (row == 0) {
+        if (!*abort) issue_tile_stores3<HD>(p, t, blocks);
+        bulk_wait_read0();
+        mbar_arrive(blk_free);
       }
     }
+    if (row == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
@@ -1049,16 +1123,22 @@ bool encode_map(CUtensorMap* m, const void* base, const Geo& g, int by, int bx) 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool encode_maps(FastParams& p, int which, const void* base) {
-  const Geo& g = p.g;
+// The nine box shapes of one tensor into dst[0..8].
+bool encode_map_set(CUtensorMap* dst, const void* base, const Geo& g) {
   for (int ky = 0; ky < 3; ++ky)
     for (int kx = 0; kx < 3; ++kx) {
       int by = box_len(ky, g.wh, g.sh), bx = box_len(kx, g.ww, g.sw);
       if (by <= 0) by = g.wh;  // shape unused when the axis has no shift
       if (bx <= 0) bx = g.ww;
-      if (!encode_map(&p.maps[which][ky * 3 + kx], base, g, by, bx)) return false;
+      if (!encode_map(&dst[ky * 3 + kx], base, g, by, bx)) return false;
     }
   return true;
+}
+bool encode_maps(FastParams& p, int which, const void* base) {
+  return encode_map_set(p.maps[which], base, p.g);
+}
+bool encode_omaps(FastParams& p, int which, const void* base) {
+  return encode_map_set(p.omaps[which], base, p.g);
 }
 
 int num_sms() {
@@ -1177,7 +1257,8 @@ cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void
   p.out2 = dv;
   p.dt_fixed = dt_fixed;
   if (!encode_maps(p, 0, q) || !encode_maps(p, 1, k) || !encode_maps(p, 2, v) ||
-      !encode_maps(p, 3, dout))
+      !encode_maps(p, 3, dout) || !encode_omaps(p, 0, dq) || !encode_omaps(p, 1, dk) ||
+      !encode_omaps(p, 2, dv))
     return cudaErrorInvalidValue;
   cudaError_t e = prep_bias(g, table, bias_t, dt_fixed, st);
   if (e != cudaSuccess) return e;
