@@ -34,9 +34,10 @@
 //    converts it to fp32.
 //  * Warp roles: warps 0-3 and 4-7 two softmax/epilogue warpgroups taking
 //    alternate tiles, warp 8 TMA producer, warp 9 issues S (and dP) and owns
-//    TMEM, warp 10 issues PV (or the gradient products). Persistent grid of one
-//    CTA per SM; tiles go round-robin, head fastest, so the SMs stream
-//    neighbouring bytes together.
+//    TMEM, warp 10 issues PV (or the gradient products), warp 11 (backward)
+//    TMA-stores the staged gradients. Persistent grid of one CTA per SM; tiles
+//    go round-robin, head fastest, so the SMs stream neighbouring bytes
+//    together.
 //  * Every mbarrier wait is bounded (%globaltimer); a wait that runs out records
 //    a timeout in the workspace status word and the kernel drains and returns.
 #include <cuda.h>
@@ -61,7 +62,8 @@ constexpr int kNumWg = 2;         // warpgroups 0 (warps 0-3) and 1 (warps 4-7) 
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;       // issues S (and dP); allocates and frees TMEM
 constexpr int kMma2Warp = 10;     // issues PV (forward) or the gradient products (backward)
-constexpr int kThreads = 352;
+constexpr int kStoreWarp = 11;    // backward: TMA-stores the staged gradients
+constexpr int kThreads = 384;
 constexpr int kMaxMaps = 9;       // box shapes: {full, seam part 1, seam part 2}^2
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestLimitNs = 1000000ull;
@@ -595,8 +597,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         mbar_drain(&drain[1], 0, kTestLimitNs * 100);
       }
     }
-  } else {
-    // Softmax / epilogue warpgroups: thread = tile row = TMEM lane.
+  } else if (warp < kNumWg * 4) {
+    // Softmax / epilogue warpgroups: thread = tile row = TMEM lane. (Warp 11
+    // has no role in the forward and goes straight to the final barrier.)
     const int wg = warp >> 2;
     const int row = threadIdx.x & (kWg - 1);
     const int gw = row / N, lr = row - gw * N;
@@ -768,6 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint64_t* drain = t_empty + NT;   // [2]: one per MMA-issuing thread
   uint64_t* never = drain + 2;
   uint64_t* blk_free = never + 1;   // operand-block area free of staged outputs
+  uint64_t* staged = blk_free + 1;  // a tile's gradients are staged in the block area
   uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
   volatile int* abort = (volatile int*)(smem + L.misc + 4);
 
@@ -783,6 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     mbar_init(&drain[1], 1);
     mbar_init(never, 1);
     mbar_init(blk_free, 1);
+    mbar_init(staged, kWg);
     *abort = 0;
     fence_mbar_init();
   }
@@ -854,35 +859,46 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       constexpr uint32_t idesc_t = idesc_bf16(kRows, HD, 1, 1);         // dV, dK: A = X^T
       constexpr uint32_t idesc_q = idesc_bf16(kRows, HD, 0, 1);         // dQ
       const uint32_t bb = smem_u32(blocks);
+      // Operand descriptors for K-steps 0 and 4 (the two query / key halves);
+      // steps 1-3 and 5-7 only move the start address, which sits in the
+      // low 14 bits, so they are a small integer add.
+      const uint64_t aPh[2] = {desc_blk_mnmajor(bb, kP0h, kZ1, kP1h, 0),
+                               desc_blk_mnmajor(bb, kP0h, kZ1, kP1h, 4)};
+      const uint64_t aPl[2] = {desc_blk_mnmajor(bb, kP0l, kZ1, kP1l, 0),
+                               desc_blk_mnmajor(bb, kP0l, kZ1, kP1l, 4)};
+      const uint64_t aQh[2] = {desc_blk_kmajor(bb, kS0h, kZ1, 0), desc_blk_kmajor(bb, kS0h, kZ1, 4)};
+      const uint64_t aQl[2] = {desc_blk_kmajor(bb, kS0l, kZ2, 0), desc_blk_kmajor(bb, kS0l, kZ2, 4)};
+      const uint64_t aKh[2] = {desc_blk_mnmajor(bb, kS0h, kZ1, kS1h, 0),
+                               desc_blk_mnmajor(bb, kS0h, kZ1, kS1h, 4)};
+      const uint64_t aKl[2] = {desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, 0),
+                               desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, 4)};
+      constexpr uint32_t kStepMN = 2048 >> 4, kStepK = 32 >> 4, kStepB = (16 * HD * 2) >> 4;
       for (long long k = 0; k < n_local; ++k) {
         const int s = (int)(k % NS), sl = (int)(k % NT);
         if (!mbar_wait(&pds_full[sl], (uint32_t)((k / NT) & 1), abort, p.status, kWaitLimitNs))
           break;
         tc_fence_after();
-        const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
-        const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
-        const uint32_t do_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
+        const uint64_t bQ = desc_mnmajor_tile<HD>(smem_u32(tiles + (s * 4 + 0) * tile_bytes), 0);
+        const uint64_t bK = desc_mnmajor_tile<HD>(smem_u32(tiles + (s * 4 + 1) * tile_bytes), 0);
+        const uint64_t bO = desc_mnmajor_tile<HD>(smem_u32(tiles + (s * 4 + 3) * tile_bytes), 0);
         const uint32_t d = tmem + sl * 256;
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk) {  // dV = P^T dO  (hi, then lo)
-          umma_ss(d + 0, desc_blk_mnmajor(bb, kP0h, kZ1, kP1h, kk),
-                  desc_mnmajor_tile<HD>(do_s, kk), idesc_t, kk);
-          umma_ss(d + 0, desc_blk_mnmajor(bb, kP0l, kZ1, kP1l, kk),
-                  desc_mnmajor_tile<HD>(do_s, kk), idesc_t, 1);
+          const uint32_t a = (kk & 3) * kStepMN, b = kk * kStepB;
+          umma_ss(d + 0, aPh[kk >> 2] + a, bO + b, idesc_t, kk);
+          umma_ss(d + 0, aPl[kk >> 2] + a, bO + b, idesc_t, 1);
         }
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk) {  // dQ = dS K
-          umma_ss(d + 64, desc_blk_kmajor(bb, kS0h, kZ1, kk), desc_mnmajor_tile<HD>(k_s, kk),
-                  idesc_q, kk);
-          umma_ss(d + 64, desc_blk_kmajor(bb, kS0l, kZ2, kk), desc_mnmajor_tile<HD>(k_s, kk),
-                  idesc_q, 1);
+          const uint32_t a = (kk & 3) * kStepK, b = kk * kStepB;
+          umma_ss(d + 64, aQh[kk >> 2] + a, bK + b, idesc_q, kk);
+          umma_ss(d + 64, aQl[kk >> 2] + a, bK + b, idesc_q, 1);
         }
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk) {  // dK = dS^T Q
-          umma_ss(d + 128, desc_blk_mnmajor(bb, kS0h, kZ1, kS1h, kk),
-                  desc_mnmajor_tile<HD>(q_s, kk), idesc_t, kk);
-          umma_ss(d + 128, desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, kk),
-                  desc_mnmajor_tile<HD>(q_s, kk), idesc_t, 1);
+          const uint32_t a = (kk & 3) * kStepMN, b = kk * kStepB;
+          umma_ss(d + 128, aKh[kk >> 2] + a, bQ + b, idesc_t, kk);
+          umma_ss(d + 128, aKl[kk >> 2] + a, bQ + b, idesc_t, 1);
         }
         umma_commit(&grad_full[sl]);
         umma_commit(&empty[s]);
@@ -892,7 +908,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         mbar_drain(&drain[1], 0, kTestLimitNs * 100);
       }
     }
-  } else {
+  } else if (warp == kStoreWarp) {
+    if (lane == 0) {   // staged gradients of every tile -> global, then free the block area
+      for (long long k = 0, t = blockIdx.x; k < n_local; ++k, t += gridDim.x) {
+        if (!mbar_wait(staged, (uint32_t)(k & 1), abort, p.status, kWaitLimitNs)) break;
+        if (!*abort) issue_tile_stores3<HD>(p, t, blocks);
+        bulk_wait_read0();
+        mbar_arrive(blk_free);
+      }
+      bulk_wait0();
+    }
+  } else if (warp < kNumWg * 4) {
     const int wg = warp >> 2;
     const int row = threadIdx.x & (kWg - 1);
     const int gw = row / N, lr = row - gw * N;
@@ -1026,8 +1052,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         if (v != 0) red_add_global_s64(p.dt_fixed + h * bp + b, v);
       }
       // epilogue: dV, dQ, dK rows from TMEM, staged in the operand-block area
-      // (free of readers once the gradient products are done), TMA-stored to
-      // grid order by one thread, which then frees the area for the next tile.
+      // (free of readers once the gradient products are done); warp 11
+      // TMA-stores them to grid order and then frees the area for the next tile.
       mbar_wait(&grad_full[sl], pht, abort, p.status, kWaitLimitNs);
       tc_fence_after();
 #pragma unroll
@@ -1042,14 +1068,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         stage_row<HD>(bb + bwd_stage(part) + (gw * N + lr) * (HD * 2), o, 1.f);
       }
       fence_proxy_async();
-      named_sync(3 + wg, kWg);
-      if (row == 0) {
-        if (!*abort) issue_tile_stores3<HD>(p, t, blocks);
-        bulk_wait_read0();
-        mbar_arrive(blk_free);
-      }
+      mbar_arrive(staged);   // warp 11 stores them and frees the block area
     }
-    if (row == 0) bulk_wait0();
   }
   tc_fence_before();
   __syncthreads();
