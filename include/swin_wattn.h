@@ -109,6 +109,32 @@ int swin_wattn_bwd(const swin_wattn_desc* desc, const void* q, const void* k, co
                    const float* bias_table, const void* dout, void* dq, void* dk, void* dv,
                    float* dbias_table, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward without a workspace argument, for callers that cannot allocate
+ * device memory or hand over a workspace when they run it: hosts whose memory
+ * manager owns every device byte and forbids raw cudaMalloc, or loops that must
+ * not allocate because an allocation can synchronise the device. (The pages
+ * have no counterpart; this is a calling convention, not a different
+ * computation.)
+ *
+ * Same arguments, results and kernels as swin_wattn_bwd. The scratch is a
+ * static device array of SWIN_NOALLOC_SCRATCH_BYTES inside the library, which
+ * every GPU that loads the library holds until the process exits; nothing is
+ * allocated or freed. The first call on a device looks the array's address up
+ * with that device current (cudaGetSymbolAddress), so make that first call
+ * before any stream capture. All calls on a device share the array: calls
+ * that overlap on the GPU (other streams, other host threads) race and give
+ * undefined results. Each call clears the device status word before it runs;
+ * a bounded device wait that runs out leaves the outputs undefined and is not
+ * reported by this entry point.
+ * Returns SWIN_ERR_UNSUPPORTED when the description does not run on the
+ * tcgen05 kernels (swin_wattn_path != 1) and SWIN_ERR_WORKSPACE when the
+ * workspace it needs exceeds SWIN_NOALLOC_SCRATCH_BYTES (heads * padded
+ * bias-table entries * 12 bytes + 768 bytes must fit). */
+#define SWIN_NOALLOC_SCRATCH_BYTES (1u << 20)
+int swin_wattn_bwd_noalloc(const swin_wattn_desc* desc, const void* q, const void* k,
+                           const void* v, const float* bias_table, const void* dout, void* dq,
+                           void* dk, void* dv, float* dbias_table, void* stream);
+
 /* Layout stage alone (steps 1-3): map[b, wy, wx, slot] = (b*H + y)*W + x, the
  * grid token that window slot holds, or -1 for a pad slot. */
 int swin_wattn_index_map(const swin_wattn_desc* desc, int32_t* map, void* stream);

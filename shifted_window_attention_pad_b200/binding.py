@@ -24,8 +24,9 @@ SWIN_FLAG_FORCE_GENERIC = 1
 SWIN_FLAG_TEST_TIMEOUT = 2
 
 EXPORTED = ("swin_wattn_path", "swin_wattn_workspace_size", "swin_wattn_fwd", "swin_wattn_bwd",
-            "swin_wattn_index_map", "swin_wattn_poll_status", "swin_wattn_strerror",
-            "swin_wattn_launch_count")
+            "swin_wattn_bwd_noalloc", "swin_wattn_index_map", "swin_wattn_poll_status",
+            "swin_wattn_strerror", "swin_wattn_launch_count")
+SWIN_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 
 class SwinWattnDesc(ctypes.Structure):
@@ -57,6 +58,7 @@ def lib():
         L.swin_wattn_workspace_size.argtypes = [D, ctypes.POINTER(ctypes.c_size_t)]
         L.swin_wattn_fwd.argtypes = [D, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.swin_wattn_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.swin_wattn_bwd_noalloc.argtypes = [D, P, P, P, P, P, P, P, P, P, P]
         L.swin_wattn_index_map.argtypes = [D, P, P]
         L.swin_wattn_poll_status.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
         L.swin_wattn_strerror.argtypes = [ctypes.c_int]
@@ -64,7 +66,8 @@ def lib():
         L.swin_wattn_launch_count.argtypes = []
         L.swin_wattn_launch_count.restype = ctypes.c_uint64
         for f in ("swin_wattn_path", "swin_wattn_workspace_size", "swin_wattn_fwd",
-                  "swin_wattn_bwd", "swin_wattn_index_map", "swin_wattn_poll_status"):
+                  "swin_wattn_bwd", "swin_wattn_bwd_noalloc", "swin_wattn_index_map",
+                  "swin_wattn_poll_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -156,6 +159,22 @@ def swin_wattn_bwd(desc, q, k, v, bias_table, dout, dq, dk, dv, dbias_table, wor
                               _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
                               _stream(stream))
     _check(rc, "swin_wattn_bwd")
+    return dq, dk, dv, dbias_table
+
+
+def swin_wattn_bwd_noalloc(desc, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
+                           stream=None):
+    """swin_wattn_bwd with the library's static scratch instead of a workspace
+    (for callers that cannot allocate; see include/swin_wattn.h)."""
+    el = _elem(desc)
+    rc = lib().swin_wattn_bwd_noalloc(ctypes.byref(desc), _ptr(q, el, "q"), _ptr(k, el, "k"),
+                                      _ptr(v, el, "v"),
+                                      _ptr(bias_table, torch.float32, "bias_table"),
+                                      _ptr(dout, el, "dout"), _ptr(dq, el, "dq"),
+                                      _ptr(dk, el, "dk"), _ptr(dv, el, "dv"),
+                                      _ptr(dbias_table, torch.float32, "dbias_table"),
+                                      _stream(stream))
+    _check(rc, "swin_wattn_bwd_noalloc")
     return dq, dk, dv, dbias_table
 
 
