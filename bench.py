@@ -38,7 +38,21 @@ from shifted_window_attention_pad_b200.synth import make_inputs  # noqa: E402
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 METRIC = "shifted-window attn fwd+bwd tokens/s"
-DOMINANT = "bwd_kernel<64,64> (fused backward: S, dP, dV, dQ, dK, dT)"
+# The backward kernel of each kernel family (75-80 % of a step on every workload).
+DOMINANT = {
+    1: "bwd_kernel<64,8> (tcgen05/TMA fused backward: S, dP, dV, dQ, dK, dT)",
+    2: "tiled_bwd_kernel<64,256,32> (warp-MMA backward, one CTA per window and head)",
+    0: "generic backward kernels (portable, per token)",
+}
+# Sources each family's kernels are built from (recorded ncu traffic is used
+# only while they are unchanged).
+KERNEL_SOURCES = {
+    1: ("shifted_window_attention_pad_b200/csrc/fast_sm100.cu",
+        "shifted_window_attention_pad_b200/csrc/sm100_ptx.cuh"),
+    2: ("shifted_window_attention_pad_b200/csrc/tiled_mma.cu",
+        "shifted_window_attention_pad_b200/csrc/sm100_ptx.cuh"),
+    0: ("shifted_window_attention_pad_b200/csrc/generic_kernels.cu",),
+}
 
 
 def parse_args(argv=None):
@@ -92,16 +106,15 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(path=1):
     h = hashlib.sha256()
-    for rel in ("shifted_window_attention_pad_b200/csrc/fast_sm100.cu",
-                "shifted_window_attention_pad_b200/csrc/sm100_ptx.cuh"):
+    for rel in KERNEL_SOURCES[path]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload):
+def recorded_traffic(workload, kpath):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, or None when absent or taken on a different kernel source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -109,7 +122,7 @@ def recorded_traffic(workload):
         with open(path) as f:
             d = json.load(f)
         e = d[workload]
-        if e.get("source_hash") != kernel_source_hash():
+        if e.get("path", 1) != kpath or e.get("source_hash") != kernel_source_hash(kpath):
             return None
         return float(e["bytes_per_launch"])
     except Exception:
@@ -362,7 +375,8 @@ def run_ours(args):
         cpu = cpu_baseline(wl, args.cpu_budget_s)
 
     if rank == 0:
-        traffic = recorded_traffic(wl.name)
+        kpath = sb.swin_wattn_path(desc)
+        traffic = recorded_traffic(wl.name, kpath)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms / K,
@@ -376,7 +390,7 @@ def run_ours(args):
             "tflops": tflops,
             "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
             "hbm_gbs_step": step_gbs, "hbm_gbs_fwd": fwd_achieved,
-            "roofline": {"bound": "hbm", "kernel": DOMINANT, "achieved": achieved,
+            "roofline": {"bound": "hbm", "kernel": DOMINANT[kpath], "achieved": achieved,
                          "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                          "peak_source": peak_src, "traffic": traffic,
                          "alg_bytes_per_launch": bwd_bytes},

@@ -69,9 +69,12 @@ enum swin_wattn_dtype { SWIN_DTYPE_F32 = 0, SWIN_DTYPE_BF16 = 1 };
 enum swin_wattn_flags {
   SWIN_FLAG_FORCE_GENERIC = 1 << 0, /* use the portable per-token kernels even where the
                                        tcgen05 kernels apply (testing, odd shapes) */
-  SWIN_FLAG_TEST_TIMEOUT = 1 << 1   /* testing only: the fast kernels wait on a barrier
+  SWIN_FLAG_TEST_TIMEOUT = 1 << 1,  /* testing only: the fast kernels wait on a barrier
                                        nothing arrives on, with a ~1 ms limit, and report
-                                       SWIN_ERR_TIMEOUT */
+                                       SWIN_ERR_TIMEOUT (no effect on the other kernel
+                                       families, which have no device-side waits) */
+  SWIN_FLAG_FORCE_TILED = 1 << 2    /* use the warp-level tensor-core kernels where they
+                                       apply, even where the tcgen05 kernels would (testing) */
 };
 
 /* Problem description. Sizes: B, H, W >= 1; 1 <= win_h, win_w <= 64;
@@ -86,9 +89,14 @@ typedef struct swin_wattn_desc {
   int32_t flags; /* enum swin_wattn_flags */
 } swin_wattn_desc;
 
-/* Kernel family a description runs on: 1 = tcgen05/TMA sm_100a kernels,
- * 0 = portable per-token CUDA kernels. Returns a negative status for an invalid
- * description. Host only, no CUDA call. */
+/* Kernel family a description runs on:
+ *   1 = tcgen05/TMA sm_100a kernels (bf16, 64-token windows, head_dim 32 or 64);
+ *   2 = warp-level tensor-core kernels, one CTA per (window, head) with the
+ *       whole window in shared memory (bf16, windows of up to 256 tokens, e.g.
+ *       16 x 16, head_dim 32 or 64);
+ *   0 = portable per-token CUDA kernels (everything else, fp32 included).
+ * Returns a negative status for an invalid description. Host only, no CUDA
+ * call. */
 int swin_wattn_path(const swin_wattn_desc* desc);
 
 /* Bytes of workspace swin_wattn_fwd and swin_wattn_bwd need for `desc`

@@ -22,6 +22,7 @@ SWIN_DTYPE_F32 = 0
 SWIN_DTYPE_BF16 = 1
 SWIN_FLAG_FORCE_GENERIC = 1
 SWIN_FLAG_TEST_TIMEOUT = 2
+SWIN_FLAG_FORCE_TILED = 4
 
 EXPORTED = ("swin_wattn_path", "swin_wattn_workspace_size", "swin_wattn_fwd", "swin_wattn_bwd",
             "swin_wattn_bwd_noalloc", "swin_wattn_index_map", "swin_wattn_poll_status",

@@ -1,7 +1,9 @@
 // api.cu -- the C ABI of libswinwattn.so (declared in include/swin_wattn.h).
 //
-// Host-side checks, workspace sizing and the choice between the tcgen05/TMA
-// kernels (bf16 shapes they cover) and the portable per-token kernels. No
+// Host-side checks, workspace sizing and the choice of kernel family: the
+// tcgen05/TMA kernels (bf16, 64-token windows), the warp-level tensor-core
+// kernels (bf16, windows of up to 256 tokens) or the portable per-token
+// kernels (everything else, fp32 included). No
 // device memory is allocated here and no stream is synchronised except by
 // swin_wattn_poll_status.
 #include <cuda_runtime.h>
@@ -36,14 +38,22 @@ static int check_desc(const swin_wattn_desc* d) {
   return SWIN_OK;
 }
 
-static bool use_fast(const swin_wattn_desc* d, const Geo& g) {
-  return !(d->flags & SWIN_FLAG_FORCE_GENERIC) && fast_supported(g, d->dtype);
+// 1 = tcgen05/TMA kernels, 2 = warp-level tensor-core kernels, 0 = portable.
+static int choose_path(const swin_wattn_desc* d, const Geo& g) {
+  if (d->flags & SWIN_FLAG_FORCE_GENERIC) return 0;
+  if (!(d->flags & SWIN_FLAG_FORCE_TILED) && fast_supported(g, d->dtype)) return 1;
+  if (tiled_supported(g, d->dtype)) return 2;
+  return 0;
 }
 
 static int cuda_status(cudaError_t e) { return e == cudaSuccess ? SWIN_OK : SWIN_ERR_CUDA; }
 
 static size_t need_workspace(const swin_wattn_desc* d, const Geo& g) {
-  return use_fast(d, g) ? fast_workspace(g) : generic_workspace(g);
+  switch (choose_path(d, g)) {
+    case 1: return fast_workspace(g);
+    case 2: return tiled_workspace(g);
+    default: return generic_workspace(g);
+  }
 }
 
 static int check_ws(const swin_wattn_desc* d, const Geo& g, void* ws, size_t bytes) {
@@ -61,7 +71,7 @@ extern "C" {
 int swin_wattn_path(const swin_wattn_desc* desc) {
   const int rc = check_desc(desc);
   if (rc) return rc;
-  return use_fast(desc, make_geo(*desc)) ? 1 : 0;
+  return choose_path(desc, make_geo(*desc));
 }
 
 int swin_wattn_workspace_size(const swin_wattn_desc* desc, size_t* bytes) {
@@ -85,8 +95,11 @@ int swin_wattn_fwd(const swin_wattn_desc* desc, const void* q, const void* k, co
   rc = check_ws(desc, g, workspace, workspace_bytes);
   if (rc) return rc;
   cudaStream_t st = (cudaStream_t)stream;
-  if (use_fast(desc, g))
+  const int path = choose_path(desc, g);
+  if (path == 1)
     return cuda_status(fast_forward(g, q, k, v, bias_table, out, lse, workspace, desc->flags, st));
+  if (path == 2)
+    return cuda_status(tiled_forward(g, q, k, v, bias_table, out, lse, workspace, st));
   return cuda_status(
       generic_forward(g, desc->dtype, q, k, v, bias_table, out, lse, workspace, st));
 }
@@ -105,9 +118,13 @@ int swin_wattn_bwd(const swin_wattn_desc* desc, const void* q, const void* k, co
   rc = check_ws(desc, g, workspace, workspace_bytes);
   if (rc) return rc;
   cudaStream_t st = (cudaStream_t)stream;
-  if (use_fast(desc, g))
+  const int path = choose_path(desc, g);
+  if (path == 1)
     return cuda_status(fast_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
                                      workspace, desc->flags, st));
+  if (path == 2)
+    return cuda_status(tiled_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
+                                      workspace, st));
   return cuda_status(generic_backward(g, desc->dtype, q, k, v, bias_table, dout, dq, dk, dv,
                                       dbias_table, workspace, st));
 }

@@ -42,4 +42,14 @@ cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void
                           const float* table, const void* dout, void* dq, void* dk, void* dv,
                           float* dtable, void* ws, int flags, cudaStream_t st);
 
+// ---- warp-level tensor-core kernels: one CTA per (window, head), windows of
+// up to 256 tokens (bf16, head_dim 32 or 64) ----------------------------------
+bool tiled_supported(const Geo& g, int dtype);
+size_t tiled_workspace(const Geo& g);
+cudaError_t tiled_forward(const Geo& g, const void* q, const void* k, const void* v,
+                          const float* table, void* out, float* lse, void* ws, cudaStream_t st);
+cudaError_t tiled_backward(const Geo& g, const void* q, const void* k, const void* v,
+                           const float* table, const void* dout, void* dq, void* dk, void* dv,
+                           float* dtable, void* ws, cudaStream_t st);
+
 }  // namespace swin

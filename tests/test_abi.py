@@ -42,13 +42,27 @@ def test_library_exports_every_declared_symbol(L):
         assert ctypes.cast(getattr(L, n), ctypes.c_void_p).value
 
 
-def test_fast_path_covers_the_bf16_window64_workloads(L):
+def test_path_selection_on_the_workloads(L):
+    """tcgen05 kernels (1) for bf16 64-token windows, warp-MMA kernels (2) for
+    the 256-token windows, portable kernels (0) for fp32."""
     expect = {"tiny-16x16-w4": 0, "ragged-90x180-w8": 1, "twelfth-degree-256x544-w8": 1,
-              "downsampled-128x272-w16": 0, "small-patch-2x512x1088-w8": 1}
+              "downsampled-128x272-w16": 2, "small-patch-2x512x1088-w8": 1}
     for name, want in expect.items():
         assert sb.swin_wattn_path(sb.desc_for(WORKLOADS[name])) == want, name
     d = sb.desc_for(WORKLOADS["twelfth-degree-256x544-w8"], flags=sb.SWIN_FLAG_FORCE_GENERIC)
     assert sb.swin_wattn_path(d) == 0
+    d = sb.desc_for(WORKLOADS["twelfth-degree-256x544-w8"], flags=sb.SWIN_FLAG_FORCE_TILED)
+    assert sb.swin_wattn_path(d) == 2
+    d = sb.desc_for(WORKLOADS["tiny-16x16-w4"], flags=sb.SWIN_FLAG_FORCE_TILED)
+    assert sb.swin_wattn_path(d) == 0      # fp32 has no tensor-core path
+
+
+@pytest.mark.parametrize("win,hd,want", [((7, 7), 64, 2), ((8, 12), 32, 2), ((16, 16), 64, 2),
+                                         ((12, 12), 32, 2), ((16, 17), 64, 0), ((32, 32), 64, 0),
+                                         ((16, 16), 128, 0), ((8, 8), 64, 1)])
+def test_tiled_path_covers_windows_up_to_256_tokens(L, win, hd, want):
+    d = sb.make_desc(1, 40, 52, win, (win[0] // 2, win[1] // 2), 2, hd, "bf16")
+    assert sb.swin_wattn_path(d) == want
 
 
 @pytest.mark.parametrize("field,value", [("shift_h", 8), ("shift_w", -1), ("win_h", 0),

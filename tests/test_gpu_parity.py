@@ -136,6 +136,73 @@ def test_fast_path_non_square_windows(win, shift):
 
 
 # ---------------------------------------------------------------------------
+# Warp-level tensor-core kernels (path 2): windows of up to 256 tokens
+# ---------------------------------------------------------------------------
+# (B, H, W, window, shift, heads, head_dim, seed): 16 x 16 windows on a padded
+# grid, window sizes that fill 64, 128 and 256 slots only partly, head_dim 32,
+# batch > 1, no shift.
+TILED = [
+    (1, 40, 52, (16, 16), (8, 8), 2, 64, 31),
+    (2, 23, 30, (7, 7), (3, 3), 2, 64, 32),
+    (1, 30, 41, (8, 12), (4, 6), 3, 32, 33),
+    (1, 37, 26, (12, 12), (6, 6), 2, 32, 34),
+    (1, 32, 48, (16, 8), (0, 0), 2, 64, 35),
+    (1, 20, 36, (4, 16), (2, 5), 2, 64, 36),
+]
+
+
+@pytest.mark.parametrize("case", TILED, ids=lambda c: "%dx%d-w%dx%d-hd%d" % (c[1], c[2], *c[3], c[6]))
+def test_tiled_path_parity(case):
+    B, H, W, win, shift, heads, hd, seed = case
+    d = sb.make_desc(B, H, W, win, shift, heads, hd, "bf16")
+    assert sb.swin_wattn_path(d) == 2
+    wl = Workload("tiled", B, H, W, win[0], shift[0], heads, hd, "bf16", seed)
+    inp = make_inputs(wl, shape_override=(B, H, W, heads, hd))
+    nb = (2 * win[0] - 1) * (2 * win[1] - 1)
+    inp["table"] = torch.from_numpy(np.random.Generator(np.random.PCG64(seed)).standard_normal(
+        (nb, heads)).astype(np.float32) * 0.02)
+    errs = compare(run_gpu(d, inp), run_oracle(d, inp), "bf16")
+    print(case, errs)
+    for n, e in errs.items():
+        assert e <= BF16_TOL, (case, n, e)
+
+
+@pytest.mark.parametrize("name", ["ragged-90x180-w8", "small-patch-2x512x1088-w8"])
+def test_tiled_path_forced_on_window64_workloads(name):
+    """The warp-MMA kernels on the 8 x 8-window workloads the tcgen05 kernels
+    normally take (ragged grid in full; the large batch-2 grid on two heads)."""
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl, flags=sb.SWIN_FLAG_FORCE_TILED)
+    assert sb.swin_wattn_path(d) == 2
+    gpu = run_gpu(d, inp, want_lse=(wl.B == 1))
+    if wl.B == 1:
+        errs = compare(gpu, run_oracle(d, inp), "bf16")
+        for n, e in errs.items():
+            assert e <= BF16_TOL, (n, e)
+        return
+    for h in (0, 11):
+        sub = {n: inp[n][:, :, :, h:h + 1].contiguous() for n in ("q", "k", "v", "dout")}
+        sub["table"] = inp["table"][:, h:h + 1].contiguous()
+        ds = sb.make_desc(wl.B, wl.H, wl.W, wl.win, wl.shift, 1, wl.head_dim, wl.dtype)
+        g = {n: gpu[n][:, :, :, h:h + 1] for n in ("o", "dq", "dk", "dv")}
+        g["dT"] = gpu["dT"][:, h:h + 1]
+        for n, e in compare(g, run_oracle(ds, sub), "bf16").items():
+            assert e <= BF16_TOL, (h, n, e)
+
+
+def test_tiled_backward_is_deterministic():
+    wl = WORKLOADS["downsampled-128x272-w16"]
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    assert sb.swin_wattn_path(d) == 2
+    a = run_gpu(d, inp, want_lse=False)
+    b = run_gpu(d, inp, want_lse=False)
+    for n in ("o", "dq", "dk", "dv", "dT"):
+        assert torch.equal(a[n], b[n]), n
+
+
+# ---------------------------------------------------------------------------
 # Exact cases and invariants
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
