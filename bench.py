@@ -333,36 +333,62 @@ def run_ours(args):
     fwd_achieved = wl.alg_bytes_fwd() / (fwd_ms / 1e3) / 1e9
     step_gbs = (wl.alg_bytes_fwd() + wl.alg_bytes_bwd()) * K / secs / 1e9
 
-    # end to end through the public API with pinned host buffers
-    hq, hk, hv, hdo = (inp[n].pin_memory() for n in ("q", "k", "v", "dout"))
-    hT = inp["table"].pin_memory()
-    ho, hdq, hdk, hdv = (torch.empty_like(hq).pin_memory() for _ in range(4))
-    hdT = torch.empty_like(hT).pin_memory()
+    # End to end through the public API with pinned host buffers: every step
+    # uploads its own inputs and downloads its own results inside the timed
+    # region. Two device buffer sets and three streams (upload, compute,
+    # download) let step i+1's upload run while step i computes and downloads,
+    # as a caller streaming batches would; PCIe is full duplex.
+    IN, OUTS = ("q", "k", "v", "dout", "table"), ("o", "dq", "dk", "dv", "dT")
+    h_in = {n: inp[n].pin_memory() for n in IN}
+    d_in = [{"q": q, "k": k, "v": v, "dout": do, "table": T},
+            {n: torch.empty_like(h_in[n], device=dev) for n in IN}]
+    d_out = [{"o": out, "dq": dq, "dk": dk, "dv": dv, "dT": dT},
+             {"o": torch.empty_like(out), "dq": torch.empty_like(dq), "dk": torch.empty_like(dk),
+              "dv": torch.empty_like(dv), "dT": torch.empty_like(dT)}]
+    h_out = {n: torch.empty_like(d_out[0][n], device="cpu").pin_memory() for n in OUTS}
+    s_up, s_comp, s_down = (torch.cuda.Stream(dev) for _ in range(3))
+    up_done, comp_done, down_done = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
 
-    def e2e_step():
-        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True); do.copy_(hdo, non_blocking=True)
-        T.copy_(hT, non_blocking=True)
-        sb.swin_wattn_fwd(desc, q, k, v, T, out, None, ws, stream)
-        sb.swin_wattn_bwd(desc, q, k, v, T, do, dq, dk, dv, dT, ws, stream)
-        ho.copy_(out, non_blocking=True); hdq.copy_(dq, non_blocking=True)
-        hdk.copy_(dk, non_blocking=True); hdv.copy_(dv, non_blocking=True)
-        hdT.copy_(dT, non_blocking=True)
+    def e2e_steps(n, start=None, end=None):
+        torch.cuda.synchronize(dev)
+        if start is not None:
+            start.record(s_up)
+        for i in range(n):
+            b = i & 1
+            I, O = d_in[b], d_out[b]
+            if i >= 2:
+                s_up.wait_event(comp_done[b])      # step i-2 has consumed these inputs
+            with torch.cuda.stream(s_up):
+                for nm in IN:
+                    I[nm].copy_(h_in[nm], non_blocking=True)
+            up_done[b].record(s_up)
+            s_comp.wait_event(up_done[b])
+            if i >= 2:
+                s_comp.wait_event(down_done[b])    # step i-2's results are read out
+            sb.swin_wattn_fwd(desc, I["q"], I["k"], I["v"], I["table"], O["o"], None, ws, s_comp)
+            sb.swin_wattn_bwd(desc, I["q"], I["k"], I["v"], I["table"], I["dout"], O["dq"],
+                              O["dk"], O["dv"], O["dT"], ws, s_comp)
+            comp_done[b].record(s_comp)
+            s_down.wait_event(comp_done[b])
+            with torch.cuda.stream(s_down):
+                for nm in OUTS:
+                    h_out[nm].copy_(O[nm], non_blocking=True)
+            down_done[b].record(s_down)
+        if end is not None:
+            end.record(s_down)                     # the last download ends the chain
+        torch.cuda.synchronize(dev)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
+    e2e_steps(2)
     E = max(1, args.e2e_steps)
     if world > 1:
         dist.barrier()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record(stream)
-    for _ in range(E):
-        e2e_step()
-    s1.record(stream)
-    torch.cuda.synchronize(dev)
+    e2e_steps(E, s0, s1)
     e2e_ms = max_over_ranks(s0.elapsed_time(s1), dev)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo, hT))
-    d2h = sum(t.numel() * t.element_size() for t in (ho, hdq, hdk, hdv, hdT))
+    if sb.swin_wattn_poll_status(ws) != 0:
+        raise RuntimeError("device-side timeout in the end-to-end steps")
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
 
     clk = clocks.summary()
     if world > 1:

@@ -171,26 +171,38 @@ __device__ __forceinline__ int round_int_add(float x) {
 // 16-19 its label as a key (15: pad or past the window, matches nothing), bits
 // 20-23 its label as a query (14: no output). Allowed pair <=> key label ==
 // query label. The bias index of (query i, key j) is pos_i - pos_j + C0.
+// PLAIN: a window with no pad slot and a single shift region, where every
+// pair is allowed. (The bias index is in range for every pair, allowed or not.)
+template <bool PLAIN>
 __device__ __forceinline__ float logit(float s, uint32_t kw, int qp, uint32_t ql,
                                        const float* bias, float sc) {
-  return ((kw >> 16) & 15u) == ql ? fmaf(s, sc, bias[qp - (int)(kw & 0xFFFFu)]) : -INFINITY;
+  const float x = fmaf(s, sc, bias[qp - (int)(kw & 0xFFFFu)]);
+  if constexpr (PLAIN)
+    return x;
+  else
+    return ((kw >> 16) & 15u) == ql ? x : -INFINITY;
 }
 
 // Common tile prologue: slot table, bias row, cleared bins, and the q, k, v
 // (and dO) rows of window `win`, head `h`, copied into swizzled shared tiles.
+// Returns true for a plain window (N = NP slots, all real tokens, one shift
+// region).
 template <int HD, int NP, bool BWD>
-__device__ __forceinline__ void tile_setup(const TiledParams& p, uint8_t* smem, const TLay& L,
+__device__ __forceinline__ bool tile_setup(const TiledParams& p, uint8_t* smem, const TLay& L,
                                            long long win, int h) {
   const Geo& g = p.g;
   const int tid = threadIdx.x;
   uint32_t* info = (uint32_t*)(smem + L.info);
   long long* off = (long long*)(smem + L.off);
+  int plain = 1;
   if (tid < NP) {
     uint32_t w = (14u << 20) | (15u << 16);
     long long o = -1;
+    plain = 0;
     if (tid < g.N) {
       const SlotInfo s = slot_info(g, win, tid);
       const uint32_t pos = (uint32_t)(s.iy * (2 * g.ww - 1) + s.ix);
+      plain = s.valid && s.label == slot_info(g, win, 0).label;
       if (s.valid) {
         w = pos | ((uint32_t)s.label << 16) | ((uint32_t)s.label << 20);
         o = (token_of(g, s) * g.heads + h) * HD;
@@ -207,7 +219,7 @@ __device__ __forceinline__ void tile_setup(const TiledParams& p, uint8_t* smem, 
     int* bins = (int*)(smem + L.bins);
     for (int b = tid; b < 2 * p.bins_pad; b += blockDim.x) bins[b] = 0;
   }
-  __syncthreads();
+  plain = __syncthreads_and(plain);
   constexpr int CH = HD / 8;
   const uint32_t base = smem_u32(smem);
   for (int idx = tid; idx < NP * CH; idx += blockDim.x) {
@@ -223,18 +235,13 @@ __device__ __forceinline__ void tile_setup(const TiledParams& p, uint8_t* smem, 
   }
   cp_async_wait_all();
   __syncthreads();
+  return plain != 0;
 }
 
 // ---- forward ------------------------------------------------------------------
-template <int HD, int NP>
-__global__ void __launch_bounds__(NP * 2, 256 / NP)
-    tiled_fwd_kernel(const __grid_constant__ TiledParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const TLay L = tlayout<HD, NP>(false, p.bins_pad);
+template <int HD, int NP, bool PLAIN>
+__device__ __forceinline__ void fwd_tile(const TiledParams& p, uint8_t* smem, const TLay& L) {
   const Geo& g = p.g;
-  const int h = (int)(blockIdx.x % g.heads);
-  const long long win = blockIdx.x / g.heads;
-  tile_setup<HD, NP, false>(p, smem, L, win, h);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t4 = lane & 3, mi = lane >> 3, rr = lane & 7;
@@ -278,10 +285,10 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
       const uint2 kw = *(const uint2*)(info + kc * 64 + n * 8 + 2 * t4);
-      s[n][0] = logit(s[n][0], kw.x, qp0, ql0, bias, sc);
-      s[n][1] = logit(s[n][1], kw.y, qp0, ql0, bias, sc);
-      s[n][2] = logit(s[n][2], kw.x, qp1, ql1, bias, sc);
-      s[n][3] = logit(s[n][3], kw.y, qp1, ql1, bias, sc);
+      s[n][0] = logit<PLAIN>(s[n][0], kw.x, qp0, ql0, bias, sc);
+      s[n][1] = logit<PLAIN>(s[n][1], kw.y, qp0, ql0, bias, sc);
+      s[n][2] = logit<PLAIN>(s[n][2], kw.x, qp1, ql1, bias, sc);
+      s[n][3] = logit<PLAIN>(s[n][3], kw.y, qp1, ql1, bias, sc);
       c0 = fmaxf(c0, fmaxf(s[n][0], s[n][1]));
       c1 = fmaxf(c1, fmaxf(s[n][2], s[n][3]));
     }
@@ -347,13 +354,27 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
   }
 }
 
+template <int HD, int NP>
+__global__ void __launch_bounds__(NP * 2, 256 / NP)
+    tiled_fwd_kernel(const __grid_constant__ TiledParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const TLay L = tlayout<HD, NP>(false, p.bins_pad);
+  const int h = (int)(blockIdx.x % p.g.heads);
+  const long long win = blockIdx.x / p.g.heads;
+  if (tile_setup<HD, NP, false>(p, smem, L, win, h))
+    fwd_tile<HD, NP, true>(p, smem, L);
+  else
+    fwd_tile<HD, NP, false>(p, smem, L);
+}
+
 // ---- backward -----------------------------------------------------------------
 // Adds dS (one value of the tile) to the fixed-point bins of bias index b:
 // |dS| < 64 goes whole into the low int32 part; larger values (|dS| < 2^22)
 // are split into an integer high part and a low remainder. A tile adds at
 // most NP <= 256 terms to one bin, so neither part can overflow.
+template <bool PLAIN>
 __device__ __forceinline__ void bin_add(int* bins_hi, int* bins_lo, int b, float ds) {
-  if (ds == 0.f) return;
+  if (!PLAIN && ds == 0.f) return;   // masked pairs of seam and pad windows
   if (fabsf(ds) < 64.f) {
     red_add_s32(bins_lo + b, round_int_add(ds * 65536.0f));
   } else {
@@ -363,16 +384,11 @@ __device__ __forceinline__ void bin_add(int* bins_hi, int* bins_lo, int b, float
   }
 }
 
-template <int HD, int NP, int QS>
-__global__ void __launch_bounds__(NP * 2, 256 / NP)
-    tiled_bwd_kernel(const __grid_constant__ TiledParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
+template <int HD, int NP, int QS, bool PLAIN>
+__device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, const TLay& L,
+                                         int h) {
   constexpr int NW = NP / 16;
-  const TLay L = tlayout<HD, NP>(true, p.bins_pad);
   const Geo& g = p.g;
-  const int h = (int)(blockIdx.x % g.heads);
-  const long long win = blockIdx.x / g.heads;
-  tile_setup<HD, NP, true>(p, smem, L, win, h);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t4 = lane & 3, mi = lane >> 3, rr = lane & 7;
@@ -382,9 +398,8 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
   const uint32_t* info = (const uint32_t*)(smem + L.info);
   const long long* off = (const long long*)(smem + L.off);
   const float* bias = (const float*)(smem + L.bias);
-  float* st_m = (float*)(smem + L.stat);
-  float* st_il = st_m + NP;
-  float* st_d = st_m + 2 * NP;
+  float* st_lse = (float*)(smem + L.stat);   // log2 of the row sum of 2^logit
+  float* st_d = st_lse + 2 * NP;
   int* bins_hi = (int*)(smem + L.bins);
   int* bins_lo = bins_hi + p.bins_pad;
   const int C0 = (g.wh - 1) * (2 * g.ww - 1) + g.ww - 1;
@@ -427,10 +442,10 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
 #pragma unroll
       for (int n = 0; n < 8; ++n) {
         const uint2 kw = *(const uint2*)(info + kc * 64 + n * 8 + 2 * t4);
-        s[n][0] = logit(s[n][0], kw.x, qp0, ql0, bias, sc);
-        s[n][1] = logit(s[n][1], kw.y, qp0, ql0, bias, sc);
-        s[n][2] = logit(s[n][2], kw.x, qp1, ql1, bias, sc);
-        s[n][3] = logit(s[n][3], kw.y, qp1, ql1, bias, sc);
+        s[n][0] = logit<PLAIN>(s[n][0], kw.x, qp0, ql0, bias, sc);
+        s[n][1] = logit<PLAIN>(s[n][1], kw.y, qp0, ql0, bias, sc);
+        s[n][2] = logit<PLAIN>(s[n][2], kw.x, qp1, ql1, bias, sc);
+        s[n][3] = logit<PLAIN>(s[n][3], kw.y, qp1, ql1, bias, sc);
         c0 = fmaxf(c0, fmaxf(s[n][0], s[n][1]));
         c1 = fmaxf(c1, fmaxf(s[n][2], s[n][3]));
       }
@@ -466,12 +481,11 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
       d1 += __shfl_xor_sync(0xffffffffu, d1, x);
     }
     if (t4 == 0) {
-      // rows without an allowed key (pad queries) get P = 0 in pass 2
-      st_m[r0 + g8] = m0 == -INFINITY ? 0.f : m0;
-      st_il[r0 + g8] = l0 > 0.f ? 1.f / l0 : 0.f;
+      // P = 2^(logit - lse); rows without an allowed key (pad queries) get
+      // lse = +inf, hence P = 0, in pass 2
+      st_lse[r0 + g8] = l0 > 0.f ? m0 + log2f(l0) : INFINITY;
       st_d[r0 + g8] = l0 > 0.f ? d0 / l0 : 0.f;
-      st_m[r0 + g8 + 8] = m1 == -INFINITY ? 0.f : m1;
-      st_il[r0 + g8 + 8] = l1 > 0.f ? 1.f / l1 : 0.f;
+      st_lse[r0 + g8 + 8] = l1 > 0.f ? m1 + log2f(l1) : INFINITY;
       st_d[r0 + g8 + 8] = l1 > 0.f ? d1 / l1 : 0.f;
     }
   }
@@ -522,23 +536,21 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
       for (int n = 0; n < NT; ++n) {
         const int i = qb + n * 8 + 2 * t4;
         const uint2 qw = *(const uint2*)(info + i);
-        const float2 mq = *(const float2*)(st_m + i);
-        const float2 iq = *(const float2*)(st_il + i);
+        const float2 lq = *(const float2*)(st_lse + i);
         const float2 dq2 = *(const float2*)(st_d + i);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t qwe = (e & 1) ? qw.y : qw.x;
-          const float m = (e & 1) ? mq.y : mq.x;
-          const float il = (e & 1) ? iq.y : iq.x;
+          const float lse = (e & 1) ? lq.y : lq.x;
           const float D = (e & 1) ? dq2.y : dq2.x;
           const int kp = (e >> 1) ? kp1 : kp0;
           const uint32_t kl = (e >> 1) ? kl1 : kl0;
           const int bidx = (int)(qwe & 0xFFFFu) - kp + C0;
-          const bool ok = kl == ((qwe >> 20) & 15u);
+          const bool ok = PLAIN || kl == ((qwe >> 20) & 15u);
           const float x = ok ? fmaf(st[n][e], sc, bias[bidx]) : -INFINITY;
-          const float pe = ex2(x - m) * il;
+          const float pe = ex2(x - lse);
           const float ds = pe * (dpt[n][e] - D);
-          if (ok) bin_add(bins_hi, bins_lo, bidx, ds);
+          if (ok) bin_add<PLAIN>(bins_hi, bins_lo, bidx, ds);
           st[n][e] = pe;
           dpt[n][e] = ds * p.dscale;
         }
@@ -558,17 +570,19 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
 #pragma unroll
         for (int np = 0; np < HD / 16; ++np) {
           const uint32_t ba = swz<HD * 2>(qb + k2 * 16 + (mi & 1) * 8 + rr, 2 * np + (mi >> 1));
-          uint32_t b[4];
-          ldsm4t(sdo + ba, b);
-          mma16816(dv[2 * np], ph, b[0], b[1]);
-          mma16816(dv[2 * np], pl, b[0], b[1]);
-          mma16816(dv[2 * np + 1], ph, b[2], b[3]);
-          mma16816(dv[2 * np + 1], pl, b[2], b[3]);
-          ldsm4t(sq + ba, b);
-          mma16816(dk[2 * np], sh, b[0], b[1]);
-          mma16816(dk[2 * np], sl, b[0], b[1]);
-          mma16816(dk[2 * np + 1], sh, b[2], b[3]);
-          mma16816(dk[2 * np + 1], sl, b[2], b[3]);
+          uint32_t bo[4], bq[4];
+          ldsm4t(sdo + ba, bo);
+          ldsm4t(sq + ba, bq);
+          // high parts into four accumulators, then the low parts: no MMA
+          // waits on the one issued just before it
+          mma16816(dv[2 * np], ph, bo[0], bo[1]);
+          mma16816(dv[2 * np + 1], ph, bo[2], bo[3]);
+          mma16816(dk[2 * np], sh, bq[0], bq[1]);
+          mma16816(dk[2 * np + 1], sh, bq[2], bq[3]);
+          mma16816(dv[2 * np], pl, bo[0], bo[1]);
+          mma16816(dv[2 * np + 1], pl, bo[2], bo[3]);
+          mma16816(dk[2 * np], sl, bq[0], bq[1]);
+          mma16816(dk[2 * np + 1], sl, bq[2], bq[3]);
         }
         // fragment word j holds (key row g8 + 8 (j & 1), queries col + 8 (j >> 1))
         const int col = sub * QS + k2 * 16 + 2 * t4;
@@ -590,10 +604,20 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
       constexpr int ACTIVE = UNITS / U;
       if (warp < ACTIVE) {
         const int unit0 = warp * U, rb = unit0 / NTQ, n0 = unit0 % NTQ;
-        float acc[U][4];
+        // separate accumulators for the high and low parts of dS (summed at
+        // the end) give 2U independent MMA chains; with U >= 4 chains already
+        // (few warps), one set keeps the registers in budget
+        constexpr int UL = U >= 4 ? 1 : U;
+        float acc[U][4], acl[UL][4];
 #pragma unroll
-        for (int u = 0; u < U; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
-#pragma unroll 4
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[u][e] = 0.f;
+#pragma unroll
+        for (int u = 0; u < UL; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acl[u][e] = 0.f;
+#pragma unroll 8
         for (int ks = 0; ks < NP / 16; ++ks) {
           uint32_t ah[4], al[4];
           const uint32_t aa = swz<128>(ks * 16 + (mi >> 1) * 8 + rr, rb * 2 + (mi & 1));
@@ -604,10 +628,21 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
             uint32_t b[4];
             ldsm4t(sk + swz<HD * 2>(ks * 16 + (mi & 1) * 8 + rr, n0 + 2 * up + (mi >> 1)), b);
             mma16816(acc[2 * up], ah, b[0], b[1]);
-            mma16816(acc[2 * up], al, b[0], b[1]);
             mma16816(acc[2 * up + 1], ah, b[2], b[3]);
-            mma16816(acc[2 * up + 1], al, b[2], b[3]);
+            if constexpr (UL == U) {
+              mma16816(acl[2 * up], al, b[0], b[1]);
+              mma16816(acl[2 * up + 1], al, b[2], b[3]);
+            } else {
+              mma16816(acc[2 * up], al, b[0], b[1]);
+              mma16816(acc[2 * up + 1], al, b[2], b[3]);
+            }
           }
+        }
+        if constexpr (UL == U) {
+#pragma unroll
+          for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[u][e] += acl[u][e];
         }
         const int row = qc * 64 + rb * 16 + g8;
         const long long o0 = off[row], o1 = off[row + 8];
@@ -642,6 +677,19 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
     const long long v = ((long long)bins_hi[b] << 16) + bins_lo[b];
     if (v != 0) red_add_global_s64(p.dt_fixed + (size_t)h * p.bins_pad + b, v);
   }
+}
+
+template <int HD, int NP, int QS>
+__global__ void __launch_bounds__(NP * 2, 256 / NP)
+    tiled_bwd_kernel(const __grid_constant__ TiledParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const TLay L = tlayout<HD, NP>(true, p.bins_pad);
+  const int h = (int)(blockIdx.x % p.g.heads);
+  const long long win = blockIdx.x / p.g.heads;
+  if (tile_setup<HD, NP, true>(p, smem, L, win, h))
+    bwd_tile<HD, NP, QS, true>(p, smem, L, h);
+  else
+    bwd_tile<HD, NP, QS, false>(p, smem, L, h);
 }
 
 // Bias table transposed to [heads][bins_pad] and scaled by log2(e); clears the
