@@ -283,7 +283,8 @@ def test_batch_images_are_independent():
     assert np.array_equal(o1[0], o2[0])
 
 
-@pytest.mark.parametrize("H,W,win,shift", [(6, 7, 4, 2), (5, 13, (2, 4), (1, 3)), (8, 8, 4, 2)])
+@pytest.mark.parametrize("H,W,win,shift", [(6, 7, 4, 2), (5, 13, (2, 4), (1, 3)), (8, 8, 4, 2),
+                                           (20, 18, 16, 8), (9, 14, (7, 7), (3, 3))])
 def test_forward_matches_per_token_brute_force(H, W, win, shift):
     """Brute force straight from the per-token description: for a real token,
     the keys are the real tokens whose rolled position falls in the same window
@@ -323,7 +324,8 @@ def _loss(s, q, k, v, T, G):
     return float((o * G).sum())
 
 
-@pytest.mark.parametrize("H,W,win,shift", [(6, 7, 4, 2), (4, 4, 2, 1), (5, 6, (2, 3), (1, 1))])
+@pytest.mark.parametrize("H,W,win,shift", [(6, 7, 4, 2), (4, 4, 2, 1), (5, 6, (2, 3), (1, 1)),
+                                           (20, 18, 16, 8)])
 def test_backward_matches_finite_differences(H, W, win, shift):
     B, heads, hd = 1, 2, 3
     s, q, k, v, T, G = problem(B, H, W, win, shift, heads, hd, seed=51)
