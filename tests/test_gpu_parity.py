@@ -140,7 +140,8 @@ def test_fast_path_non_square_windows(win, shift):
 # ---------------------------------------------------------------------------
 # (B, H, W, window, shift, heads, head_dim, seed): 16 x 16 windows on a padded
 # grid, window sizes that fill 64, 128 and 256 slots only partly, head_dim 32,
-# batch > 1, no shift.
+# batch > 1, no shift; every (slots, head_dim) kernel instance meets both plain
+# windows (no pad, one shift region) and masked ones.
 TILED = [
     (1, 40, 52, (16, 16), (8, 8), 2, 64, 31),
     (2, 23, 30, (7, 7), (3, 3), 2, 64, 32),
@@ -148,6 +149,7 @@ TILED = [
     (1, 37, 26, (12, 12), (6, 6), 2, 32, 34),
     (1, 32, 48, (16, 8), (0, 0), 2, 64, 35),
     (1, 20, 36, (4, 16), (2, 5), 2, 64, 36),
+    (1, 32, 48, (16, 16), (8, 8), 3, 32, 37),
 ]
 
 
