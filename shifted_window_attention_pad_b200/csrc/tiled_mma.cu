@@ -17,7 +17,10 @@
 // (N rounded up); slots past N are masked like pad.
 //
 // Forward, warp w, query rows [16w, 16w + 16): S = Q K^T in 64-key chunks with
-// an online softmax (running row max and sum, O rescaled), O += P V.
+// an online softmax (running row max and sum, O rescaled), O += P V. A
+// 256-slot window runs as two CTAs of 8 warps, one per half of its query rows
+// (both load the whole window; the second read of k and v mostly hits L2), so
+// two CTAs share an SM and one's loads overlap the other's math.
 // Backward, recomputing everything from q, k, v, dO and the table:
 //   pass 1, warp w, query rows [16w, 16w + 16): S and dP = dO V^T per 64-key
 //     chunk with the same online rescaling give the row max m_i, the row sum
@@ -72,7 +75,8 @@ struct TiledParams {
 // q, k, v (, dO) as [NP][hd] bf16 with 16-byte chunks XOR-swizzled per row;
 // backward: the dS^T buffer of one 64-query chunk, high and low parts, as
 // [NP keys][64 queries] bf16; per-slot source offsets and info words; row
-// statistics (backward); the head's bias row; fixed-point bins (backward).
+// statistics (backward: log-sum-exp and D per query); the head's bias row;
+// fixed-point bins (backward).
 struct TLay {
   uint32_t q, k, v, dout, dsh, dsl, off, info, stat, bias, bins, total;
 };
@@ -99,7 +103,7 @@ __host__ __device__ inline TLay tlayout(bool bwd, int bins_pad) {
   L.info = o;
   o += NP * 4;
   L.stat = o;
-  o += bwd ? NP * 12 : 0;
+  o += bwd ? NP * 8 : 0;
   L.bias = o;
   o += (uint32_t)bins_pad * 4;
   L.bins = o;
@@ -240,7 +244,8 @@ __device__ __forceinline__ bool tile_setup(const TiledParams& p, uint8_t* smem, 
 
 // ---- forward ------------------------------------------------------------------
 template <int HD, int NP, bool PLAIN>
-__device__ __forceinline__ void fwd_tile(const TiledParams& p, uint8_t* smem, const TLay& L) {
+__device__ __forceinline__ void fwd_tile(const TiledParams& p, uint8_t* smem, const TLay& L,
+                                         int qbase) {
   const Geo& g = p.g;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -252,7 +257,7 @@ __device__ __forceinline__ void fwd_tile(const TiledParams& p, uint8_t* smem, co
   const float* bias = (const float*)(smem + L.bias);
   const int C0 = (g.wh - 1) * (2 * g.ww - 1) + g.ww - 1;
   const float sc = p.scale_log2;
-  const int r0 = warp * 16;
+  const int r0 = qbase + warp * 16;
 
   uint32_t qa[HD / 16][4];
 #pragma unroll
@@ -354,17 +359,20 @@ __device__ __forceinline__ void fwd_tile(const TiledParams& p, uint8_t* smem, co
   }
 }
 
-template <int HD, int NP>
-__global__ void __launch_bounds__(NP * 2, 256 / NP)
+// PARTS CTAs per (window, head), each on NP / PARTS query rows.
+template <int HD, int NP, int PARTS>
+__global__ void __launch_bounds__(NP * 2 / PARTS, 256 * PARTS / NP)
     tiled_fwd_kernel(const __grid_constant__ TiledParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const TLay L = tlayout<HD, NP>(false, p.bins_pad);
-  const int h = (int)(blockIdx.x % p.g.heads);
-  const long long win = blockIdx.x / p.g.heads;
+  const long long tile = blockIdx.x / PARTS;
+  const int qbase = (int)(blockIdx.x % PARTS) * (NP / PARTS);
+  const int h = (int)(tile % p.g.heads);
+  const long long win = tile / p.g.heads;
   if (tile_setup<HD, NP, false>(p, smem, L, win, h))
-    fwd_tile<HD, NP, true>(p, smem, L);
+    fwd_tile<HD, NP, true>(p, smem, L, qbase);
   else
-    fwd_tile<HD, NP, false>(p, smem, L);
+    fwd_tile<HD, NP, false>(p, smem, L, qbase);
 }
 
 // ---- backward -----------------------------------------------------------------
@@ -399,13 +407,13 @@ __device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, co
   const long long* off = (const long long*)(smem + L.off);
   const float* bias = (const float*)(smem + L.bias);
   float* st_lse = (float*)(smem + L.stat);   // log2 of the row sum of 2^logit
-  float* st_d = st_lse + 2 * NP;
+  float* st_d = st_lse + NP;                 // D = sum_j P_ij dP_ij
   int* bins_hi = (int*)(smem + L.bins);
   int* bins_lo = bins_hi + p.bins_pad;
   const int C0 = (g.wh - 1) * (2 * g.ww - 1) + g.ww - 1;
   const float sc = p.scale_log2;
 
-  // ---- pass 1: row max, row sum and D per query row ----
+  // ---- pass 1: log-sum-exp and D per query row ----
   {
     const int r0 = warp * 16;
     uint32_t qa[HD / 16][4], da[HD / 16][4];
@@ -743,11 +751,11 @@ void fill_params(TiledParams& p, const Geo& g, const float* bias_t) {
 
 template <typename K>
 cudaError_t launch_tiled(K kernel, const TiledParams& p, int threads, size_t smem,
-                         cudaStream_t st) {
+                         cudaStream_t st, int parts = 1) {
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long long tiles = p.g.n_win * p.g.heads;
+  const long long tiles = p.g.n_win * p.g.heads * parts;
   kernel<<<(unsigned)tiles, threads, smem, st>>>(p);
   note_launch();
   return cudaGetLastError();
@@ -768,7 +776,7 @@ bool tiled_supported(const Geo& g, int dtype) {
   if (dtype != SWIN_DTYPE_BF16) return false;
   if (g.hd != 64 && g.hd != 32) return false;
   if (g.N > 256) return false;
-  if (g.n_win * (long long)g.heads > 0x7fffffffLL) return false;
+  if (g.n_win * (long long)g.heads * 2 > 0x7fffffffLL) return false;   // grid size
   return tiled_smem_any(g, true) <= kSmemLimitT && tiled_smem_any(g, false) <= kSmemLimitT;
 }
 
@@ -794,13 +802,13 @@ cudaError_t tiled_forward(const Geo& g, const void* q, const void* k, const void
   const int NP = slots_for(g.N);
   const size_t smem = tiled_smem_any(g, false);
   if (g.hd == 64) {
-    if (NP == 64) return launch_tiled(tiled_fwd_kernel<64, 64>, p, 128, smem, st);
-    if (NP == 128) return launch_tiled(tiled_fwd_kernel<64, 128>, p, 256, smem, st);
-    return launch_tiled(tiled_fwd_kernel<64, 256>, p, 512, smem, st);
+    if (NP == 64) return launch_tiled(tiled_fwd_kernel<64, 64, 1>, p, 128, smem, st);
+    if (NP == 128) return launch_tiled(tiled_fwd_kernel<64, 128, 1>, p, 256, smem, st);
+    return launch_tiled(tiled_fwd_kernel<64, 256, 2>, p, 256, smem, st, 2);
   }
-  if (NP == 64) return launch_tiled(tiled_fwd_kernel<32, 64>, p, 128, smem, st);
-  if (NP == 128) return launch_tiled(tiled_fwd_kernel<32, 128>, p, 256, smem, st);
-  return launch_tiled(tiled_fwd_kernel<32, 256>, p, 512, smem, st);
+  if (NP == 64) return launch_tiled(tiled_fwd_kernel<32, 64, 1>, p, 128, smem, st);
+  if (NP == 128) return launch_tiled(tiled_fwd_kernel<32, 128, 1>, p, 256, smem, st);
+  return launch_tiled(tiled_fwd_kernel<32, 256, 2>, p, 256, smem, st, 2);
 }
 
 cudaError_t tiled_backward(const Geo& g, const void* q, const void* k, const void* v,
