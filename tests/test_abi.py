@@ -106,6 +106,33 @@ def test_workspace_sizes_are_modest(L):
         assert 256 <= n < 512 * 2**20, (wl.name, n)
 
 
+def _a256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("name", ["ragged-90x180-w8", "twelfth-degree-256x544-w8",
+                                  "downsampled-128x272-w16", "small-patch-2x512x1088-w8",
+                                  "tiny-16x16-w4"])
+def test_workspace_size_follows_the_documented_layout(L, name):
+    """Tensor-core families: 256-byte header, the transposed bias table
+    [heads][bins padded to 4] fp32 and the fixed-point bias gradient
+    [heads][bins padded] int64, each region 256-byte aligned. Portable
+    kernels: header, per-row partials (3 floats per window slot and head) and
+    per-window bias-gradient partials."""
+    wl = WORKLOADS[name]
+    d = sb.desc_for(wl)
+    bins = (2 * wl.win - 1) ** 2
+    bp = (bins + 3) // 4 * 4
+    if sb.swin_wattn_path(d) in (1, 2):
+        want = 256 + _a256(wl.heads * bp * 4) + _a256(wl.heads * bp * 8)
+    else:
+        hp = -(-wl.H // wl.win) * wl.win
+        wp = -(-wl.W // wl.win) * wl.win
+        n_win = wl.B * (hp // wl.win) * (wp // wl.win)
+        want = 256 + _a256(n_win * wl.heads * wl.win ** 2 * 3 * 4) + _a256(n_win * wl.heads * bp * 4)
+    assert sb.swin_wattn_workspace_size(d) == want
+
+
 def test_strerror_covers_every_status(L):
     for s in range(-5, 1):
         assert sb.swin_wattn_strerror(s) != "unknown status"
