@@ -107,6 +107,16 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def input_bytes(wl):
+    """Bytes of q, k, v and dO one step reads (bf16)."""
+    return 4 * wl.tokens * wl.heads * wl.head_dim * 2
+
+
+def needs_l2_flush(wl):
+    """Inputs smaller than twice L2 would be served from L2 on the next step."""
+    return input_bytes(wl) < 2 * L2_BYTES
+
+
 def kernel_source_hash(path=1):
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[path]:
@@ -302,8 +312,8 @@ def run_ours(args):
     # Inputs smaller than twice the 126 MB L2 would be served from L2 on the
     # next step: flush it between steps by writing a 256 MB buffer, and time
     # the steps by their own fwd+bwd events (the flush is left out).
-    in_bytes = 4 * wl.tokens * wl.heads * wl.head_dim * 2
-    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev) if in_bytes < 2 * L2_BYTES else None
+    in_bytes = input_bytes(wl)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev) if needs_l2_flush(wl) else None
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = sb.swin_wattn_launch_count()

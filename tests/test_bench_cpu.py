@@ -52,3 +52,13 @@ def test_max_over_ranks_and_rank_seeds_gloo_world2():
         assert p.exitcode == 0
     assert [r[1] for r in res] == [2.5, 2.5]
     assert res[0][2] != res[1][2]
+
+
+def test_l2_flush_only_for_workloads_smaller_than_twice_l2():
+    import bench
+    from shifted_window_attention_pad_b200 import WORKLOADS
+    want = {"ragged-90x180-w8": True, "twelfth-degree-256x544-w8": False,
+            "downsampled-128x272-w16": False, "small-patch-2x512x1088-w8": False}
+    for name, flush in want.items():
+        assert bench.needs_l2_flush(WORKLOADS[name]) == flush, name
+    assert bench.input_bytes(WORKLOADS["twelfth-degree-256x544-w8"]) == 4 * 256 * 544 * 16 * 64 * 2
