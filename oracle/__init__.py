@@ -17,8 +17,11 @@ from . import build as _build
 
 
 class Shape(ctypes.Structure):
+    """Problem shape; valid_h / valid_w (0 = H / W) bound the tokens that carry
+    field data (the others are padding, see swin_oracle.c)."""
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("B", "H", "W", "win_h", "win_w", "shift_h", "shift_w", "heads", "head_dim")]
+                ("B", "H", "W", "win_h", "win_w", "shift_h", "shift_w", "heads", "head_dim",
+                 "valid_h", "valid_w")]
 
 
 _lib = None
@@ -47,10 +50,11 @@ def num_threads() -> int:
     return lib().swin_oracle_num_threads()
 
 
-def make_shape(B, H, W, win, shift, heads, head_dim):
+def make_shape(B, H, W, win, shift, heads, head_dim, valid=None):
     wh, ww = (win, win) if np.isscalar(win) else win
     sh, sw = (shift, shift) if np.isscalar(shift) else shift
-    return Shape(B, H, W, wh, ww, sh, sw, heads, head_dim)
+    vh, vw = valid if valid is not None else (0, 0)
+    return Shape(B, H, W, wh, ww, sh, sw, heads, head_dim, vh, vw)
 
 
 def padded_hw(s: Shape):

@@ -44,6 +44,7 @@ typedef struct {
   int32_t win_h, win_w;
   int32_t shift_h, shift_w;
   int32_t heads, head_dim;
+  int32_t valid_h, valid_w; /* valid extent of the stored grid; 0 = H (or W) */
 } swin_oracle_shape;
 
 enum { ORACLE_OK = 0, ORACLE_BAD_SHAPE = -1, ORACLE_NO_MEMORY = -2, ORACLE_EMPTY_ROW = -3 };
@@ -52,23 +53,36 @@ static int64_t round_up(int64_t n, int64_t w) { return (n + w - 1) / w * w; }
 
 static int shape_ok(const swin_oracle_shape* s) {
   if (s->B < 0 || s->H < 0 || s->W < 0) return 0;
+  if (s->valid_h < 0 || s->valid_h > s->H || s->valid_w < 0 || s->valid_w > s->W) return 0;
   if (s->win_h < 1 || s->win_w < 1 || s->heads < 1 || s->head_dim < 1) return 0;
   if (s->shift_h < 0 || s->shift_h >= s->win_h) return 0;
   if (s->shift_w < 0 || s->shift_w >= s->win_w) return 0;
   return 1;
 }
 
+/* Valid extent of the token grid: the tokens that carry field data. Table I
+ * pads the physical field itself (H x W to H^ x W^ pixels) before patching,
+ * so a stored token can cover only padded pixels. Reading: a token is real
+ * when its patch holds at least one real pixel, i.e. the caller passes
+ * valid_h = ceil(field rows / patch) (and likewise for columns); tokens at or
+ * beyond the valid extent are treated exactly like the pad tokens of step 1.
+ * 0 means the whole stored grid is valid. */
+static int64_t valid_rows(const swin_oracle_shape* s) { return s->valid_h ? s->valid_h : s->H; }
+static int64_t valid_cols(const swin_oracle_shape* s) { return s->valid_w ? s->valid_w : s->W; }
+
 /* ---- Step 1: padding (Table I, H^ x W^) -------------------------------------
  * Reading: pad at the bottom and right, to the smallest multiple of the window;
- * pad values are zero and pad tokens are flagged invalid. One (batch, head)
- * channel slice [H, W, hd] of the [B, H, W, heads, hd] tensor is copied. */
+ * pad values are zero and pad tokens are flagged invalid, as are stored tokens
+ * outside the valid extent. One (batch, head) channel slice [H, W, hd] of the
+ * [B, H, W, heads, hd] tensor is copied. */
 static void step1_pad(const swin_oracle_shape* s, const double* x, int64_t b, int64_t h,
                       int64_t Hp, int64_t Wp, double* xp, unsigned char* valid) {
   const int64_t hd = s->head_dim, C = (int64_t)s->heads * hd;
+  const int64_t Hv = valid_rows(s), Wv = valid_cols(s);
   for (int64_t y = 0; y < Hp; ++y)
     for (int64_t xx = 0; xx < Wp; ++xx) {
       const int inside = (y < s->H) && (xx < s->W);
-      if (valid) valid[y * Wp + xx] = (unsigned char)inside;
+      if (valid) valid[y * Wp + xx] = (unsigned char)((y < Hv) && (xx < Wv));
       for (int64_t e = 0; e < hd; ++e)
         xp[(y * Wp + xx) * hd + e] =
             inside ? x[((b * s->H + y) * s->W + xx) * C + h * hd + e] : 0.0;
@@ -246,7 +260,8 @@ static void step4_window_attention_backward(const swin_oracle_shape* s, const do
 
 /* ---- Step 7: crop (inverse of step 1) -----------------------------------------
  * Writes the [H^, W^, width] padded slice back into channel h of a
- * [B, H, W, heads, width] tensor, dropping pad positions. */
+ * [B, H, W, heads, width] tensor, dropping pad positions. Stored tokens
+ * outside the valid extent receive the zeros step 4 leaves for them. */
 static void step7_crop(const swin_oracle_shape* s, const double* xp, int64_t b, int64_t h,
                        int64_t Hp, int64_t Wp, int64_t width, double* out) {
   (void)Hp;
@@ -416,8 +431,9 @@ int swin_oracle_backward(const swin_oracle_shape* s, const double* q, const doub
 }
 
 /* Index map of steps 1-3: for every (b, window, slot) the source token
- * (b*H + y)*W + x, or -1 where the slot holds a pad position. Built by pushing
- * token ids through the same pad / roll / partition steps as the data. */
+ * (b*H + y)*W + x, or -1 where the slot holds a pad position (or a stored
+ * token outside the valid extent). Built by pushing token ids through the same
+ * pad / roll / partition steps as the data. */
 int swin_oracle_index_map(const swin_oracle_shape* s, int64_t* map) {
   if (!shape_ok(s)) return ORACLE_BAD_SHAPE;
   const int64_t Hp = round_up(s->H, s->win_h), Wp = round_up(s->W, s->win_w);
@@ -428,7 +444,8 @@ int swin_oracle_index_map(const swin_oracle_shape* s, int64_t* map) {
   for (int64_t b = 0; b < s->B; ++b) {
     for (int64_t y = 0; y < Hp; ++y)
       for (int64_t x = 0; x < Wp; ++x)
-        padded[y * Wp + x] = (y < s->H && x < s->W) ? (b * s->H + y) * s->W + x : -1;
+        padded[y * Wp + x] =
+            (y < valid_rows(s) && x < valid_cols(s)) ? (b * s->H + y) * s->W + x : -1;
     step2_roll(padded, rolled, Hp, Wp, sizeof(int64_t), s->shift_h, s->shift_w);
     step3_partition(rolled, map + b * cells, Hp, Wp, s->win_h, s->win_w, sizeof(int64_t));
   }

@@ -370,3 +370,59 @@ def test_bf16_measure_charges_computation_not_storage_rounding():
     rms = np.sqrt(np.mean(o * o))
     bad.reshape(-1)[12345] += 0.03 * rms + gh.half_ulp_bf16(o.reshape(-1)[12345])
     assert gh.err_bf16(bad, o) > gh.BF16_TOL
+
+
+# ---------------------------------------------------------------------------
+# Valid extent (tokens that cover only padded field pixels, Table I): pins
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("H,W,valid,win,shift", [(16, 24, (13, 21), 8, 4), (10, 12, (9, 12), 4, 2),
+                                                 (12, 8, (12, 7), (4, 4), (0, 2))])
+def test_valid_extent_equals_the_smaller_grid_when_padding_agrees(H, W, valid, win, shift):
+    """When the stored grid and its valid extent pad to the same window
+    multiple, the tokens beyond the extent are exactly the pad tokens of the
+    smaller grid: the valid region's outputs equal a plain run on the smaller
+    grid, and every stored token beyond the extent gets exact zeros."""
+    Hv, Wv = valid
+    heads, hd = 2, 3
+    s, q, k, v, T, do = problem(1, H, W, win, shift, heads, hd, seed=61)
+    sv = oracle.make_shape(1, H, W, win, shift, heads, hd, valid=valid)
+    assert oracle.padded_hw(sv) == oracle.padded_hw(oracle.make_shape(1, Hv, Wv, win, shift,
+                                                                      heads, hd))
+    o, lse = oracle.forward(sv, q, k, v, T)
+    dq, dk, dv, dT = oracle.backward(sv, q, k, v, T, do)
+    ss = oracle.make_shape(1, Hv, Wv, win, shift, heads, hd)
+    cut = lambda a: np.ascontiguousarray(a[:, :Hv, :Wv])
+    o2, lse2 = oracle.forward(ss, cut(q), cut(k), cut(v), T)
+    dq2, dk2, dv2, dT2 = oracle.backward(ss, cut(q), cut(k), cut(v), T, cut(do))
+    for a, b in ((o, o2), (lse, lse2), (dq, dq2), (dk, dk2), (dv, dv2)):
+        np.testing.assert_allclose(a[:, :Hv, :Wv], b, rtol=0, atol=1e-13)
+        outside = np.ones(a.shape[:3], bool)
+        outside[:, :Hv, :Wv] = False
+        assert np.all(a[outside] == 0.0)
+    np.testing.assert_allclose(dT, dT2, rtol=0, atol=1e-12)
+
+
+def test_data_beyond_the_valid_extent_changes_nothing():
+    """Tokens beyond the valid extent are masked: new q, k, v, dO values there
+    leave every output bit-identical."""
+    heads, hd = 2, 4
+    s, q, k, v, T, do = problem(1, 14, 19, 4, 2, heads, hd, seed=62)
+    sv = oracle.make_shape(1, 14, 19, 4, 2, heads, hd, valid=(11, 15))
+    ref_f = oracle.forward(sv, q, k, v, T)
+    ref_b = oracle.backward(sv, q, k, v, T, do)
+    q2, k2, v2, do2 = (a.copy() for a in (q, k, v, do))
+    for a in (q2, k2, v2, do2):
+        a[:, 11:] = 7.0
+        a[:, :, 15:] = -3.0
+    for a, b in zip(ref_f + ref_b, oracle.forward(sv, q2, k2, v2, T) +
+                    oracle.backward(sv, q2, k2, v2, T, do2)):
+        assert np.array_equal(a, b)
+
+
+def test_index_map_marks_tokens_beyond_the_valid_extent_as_padding():
+    s = oracle.make_shape(1, 9, 10, 4, 2, 1, 1)
+    sv = oracle.make_shape(1, 9, 10, 4, 2, 1, 1, valid=(7, 8))
+    m, mv = oracle.index_map(s), oracle.index_map(sv)
+    y, x = np.divmod(np.where(m >= 0, m, 0), 10)
+    keep = (m >= 0) & (y < 7) & (x < 8)
+    assert np.array_equal(mv, np.where(keep, m, -1))
