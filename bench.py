@@ -40,11 +40,14 @@ FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "shifted-window attn fwd+bwd tokens/s"
 # The backward kernel of each kernel family (75-80 % of a step on every workload).
-DOMINANT = {
-    1: "bwd_kernel<64,8> (tcgen05/TMA fused backward: S, dP, dV, dQ, dK, dT)",
-    2: "tiled_bwd_kernel<64,256,32> (warp-MMA backward, one CTA per window and head)",
-    0: "generic backward kernels (portable, per token)",
-}
+def dominant_kernel(kpath, wl):
+    if kpath == 1:
+        return ("bwd_kernel<%d,%d> (tcgen05/TMA fused backward: S, dP, dV, dQ, dK, dT)" %
+                (wl.head_dim, 8 if wl.win == 8 else 0))
+    if kpath == 2:
+        return ("tiled_bwd_kernel<%d,%d,32> (warp-MMA backward, one CTA per window and head)" %
+                (wl.head_dim, 64 if wl.win ** 2 <= 64 else (128 if wl.win ** 2 <= 128 else 256)))
+    return "generic backward kernels (portable, per token)"
 # Sources each family's kernels are built from (recorded ncu traffic is used
 # only while they are unchanged).
 KERNEL_SOURCES = {
@@ -310,11 +313,13 @@ def run_ours(args):
 
     K = args.steps
     # Inputs smaller than twice the 126 MB L2 would be served from L2 on the
-    # next step: flush it between steps by writing a 256 MB buffer, and time
-    # the steps by their own fwd+bwd events (the flush is left out).
+    # next step: flush it before the forward and again before the backward
+    # (which would otherwise find q, k, v in L2 from the forward) by writing a
+    # 256 MB buffer, and time the steps by their own fwd and bwd events (the
+    # flushes are left out).
     in_bytes = input_bytes(wl)
     flush = torch.empty(64 << 20, dtype=torch.float32, device=dev) if needs_l2_flush(wl) else None
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = sb.swin_wattn_launch_count()
     with ClockSampler(dev) as clocks:
@@ -328,8 +333,11 @@ def run_ours(args):
             ev[i][0].record(stream)
             sb.swin_wattn_fwd(desc, q, k, v, T, out, None, ws, stream)
             ev[i][1].record(stream)
-            sb.swin_wattn_bwd(desc, q, k, v, T, do, dq, dk, dv, dT, ws, stream)
+            if flush is not None:
+                flush.zero_()
             ev[i][2].record(stream)
+            sb.swin_wattn_bwd(desc, q, k, v, T, do, dq, dk, dv, dT, ws, stream)
+            ev[i][3].record(stream)
         end.record(stream)
         torch.cuda.synchronize(dev)
         if world > 1:
@@ -338,11 +346,11 @@ def run_ours(args):
     if flush is None:
         ms = max_over_ranks(start.elapsed_time(end), dev)
     else:
-        ms = max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in ev), dev)
+        ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) + e[2].elapsed_time(e[3]) for e in ev), dev)
     if sb.swin_wattn_poll_status(ws) != 0:
         raise RuntimeError("device-side timeout in the timed region")
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
-    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / K
 
     secs = ms / 1e3
     tokens = wl.tokens * K * world
@@ -434,12 +442,13 @@ def run_ours(args):
                        "tokens_per_rank_step": wl.tokens, "parallelism": "dp%d" % world,
                        "l2": ("inputs larger than L2 (q,k,v,dO = %.2f GB per step)" % (in_bytes / 1e9)
                               if flush is None else
-                              "L2 flushed between steps (256 MB write, outside the timed fwd+bwd "
-                              "events; q,k,v,dO = %.1f MB per step)" % (in_bytes / 1e6))},
+                              "L2 flushed before the forward and before the backward of every "
+                              "step (256 MB write, outside the timed fwd and bwd events; "
+                              "q,k,v,dO = %.1f MB per step)" % (in_bytes / 1e6))},
             "tflops": tflops,
             "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
             "hbm_gbs_step": step_gbs, "hbm_gbs_fwd": fwd_achieved,
-            "roofline": {"bound": "hbm", "kernel": DOMINANT[kpath], "achieved": achieved,
+            "roofline": {"bound": "hbm", "kernel": dominant_kernel(kpath, wl), "achieved": achieved,
                          "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                          "peak_source": peak_src, "traffic": traffic,
                          "alg_bytes_per_launch": bwd_bytes},

@@ -23,6 +23,8 @@
  * dS_ij = P_ij (dP_ij - D_i), dP_ij = dO_i.v_j, D_i = sum_j P_ij dP_ij. Pad
  * tokens produce and receive nothing.
  *
+ * Tokens beyond the descriptor's valid extent are pad tokens too.
+ *
  * Layouts (all row-major, contiguous):
  *   q, k, v, out, dout, dq, dk, dv : [B, H, W, heads, head_dim] of `dtype`
  *   bias_table, dbias_table        : [(2*win_h-1)*(2*win_w-1), heads] fp32
@@ -73,13 +75,28 @@ enum swin_wattn_flags {
                                        nothing arrives on, with a ~1 ms limit, and report
                                        SWIN_ERR_TIMEOUT (no effect on the other kernel
                                        families, which have no device-side waits) */
-  SWIN_FLAG_FORCE_TILED = 1 << 2    /* use the warp-level tensor-core kernels where they
+  SWIN_FLAG_FORCE_TILED = 1 << 2,   /* use the warp-level tensor-core kernels where they
                                        apply, even where the tcgen05 kernels would (testing) */
+  SWIN_FLAG_DBIAS_SUMS = 1 << 3     /* swin_wattn_bwd on the tensor-core kernels: leave the
+                                       exact bias-gradient sums in the workspace instead of
+                                       writing dbias_table (which may then be NULL), so that
+                                       partial sums of several calls or ranks can be added as
+                                       integers (swin_wattn_dbias_sums) and converted once
+                                       (swin_wattn_dbias_finish) */
 };
 
 /* Problem description. Sizes: B, H, W >= 1; 1 <= win_h, win_w <= 64;
  * 0 <= shift < win per axis; heads >= 1; 8 <= head_dim <= 256 with head_dim a
- * multiple of 8. */
+ * multiple of 8; 0 <= valid_h <= H, 0 <= valid_w <= W.
+ *
+ * Valid extent (valid_h, valid_w; 0 = H, W): Table I of the page pads the
+ * physical field before it is cut into patches, so stored tokens can cover
+ * only padded pixels (a 2041 x 4320 field padded to 2048 x 4352 in patches of
+ * 8 gives 256 x 544 tokens of which columns 540..543 hold no data; pass
+ * valid_h = ceil(field rows / patch), valid_w = ceil(field columns / patch)).
+ * Tokens at row >= valid_h or column >= valid_w are padding: they are no key
+ * of any query and their outputs (out, lse, dq, dk, dv) are written as zeros.
+ * The window grid still follows the stored H x W. */
 typedef struct swin_wattn_desc {
   int32_t B, H, W;
   int32_t win_h, win_w;
@@ -87,6 +104,7 @@ typedef struct swin_wattn_desc {
   int32_t heads, head_dim;
   int32_t dtype; /* enum swin_wattn_dtype: element type of q, k, v, out, dout, dq, dk, dv */
   int32_t flags; /* enum swin_wattn_flags */
+  int32_t valid_h, valid_w; /* valid extent of the token grid; 0 = the whole grid */
 } swin_wattn_desc;
 
 /* Kernel family a description runs on:
@@ -111,11 +129,58 @@ int swin_wattn_fwd(const swin_wattn_desc* desc, const void* q, const void* k, co
 
 /* Backward: dq, dk, dv (same layout and dtype as q) and dbias_table, all
  * overwritten, not accumulated. The softmax rows are recomputed from q, k, v
- * and the table; no forward state is needed. dbias_table is summed in a fixed
- * order, so repeated calls give identical bits. */
+ * and the table; no forward state is needed. On the tensor-core kernels
+ * (paths 1 and 2) dbias_table is summed exactly in integers whose unit follows
+ * the magnitude of each tile's gradients, then rounded once to fp32: repeated
+ * calls give identical bits, and the relative error does not depend on the
+ * scale of dout. A NaN or infinity reaching a head's gradient makes that
+ * head's dbias_table NaN. The portable kernels sum fp32 partials per window in
+ * a fixed order (also repeatable). */
 int swin_wattn_bwd(const swin_wattn_desc* desc, const void* q, const void* k, const void* v,
                    const float* bias_table, const void* dout, void* dq, void* dk, void* dv,
                    float* dbias_table, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Row bands of a grid split across devices (TERRA page, Fig. 6 and Table III:
+ * window layouts placed on devices with boundary-only peer-to-peer
+ * exchange). Band r holds rows [r*R, r*R + H) of a grid of Hg rows, R a
+ * multiple of win_h; the description of a band call is the band's own: H =
+ * its rows (a multiple of win_h except in the last band), everything else as
+ * for the whole grid. The shift moves content up by shift_h, so the band's
+ * last window row reads the shift_h rows below the band -- the next band's
+ * first rows, or for the last band the grid's first rows (the wrap) -- from
+ * `q`, `k`, `v`, `dout` here, each [B, shift_h, W, heads, head_dim], and
+ * writes the outputs of those rows to `out`, `lse`, `dq`, `dk`, `dv` of the
+ * same shape, which belong to the band that owns them. The band's own first
+ * shift_h rows are computed, and their outputs written, by the band above.
+ * `interior` = 1 for every band but the last one: its last window row lies
+ * inside the grid, so no shift-region split applies there. All pointers are
+ * device memory, 16-byte aligned; a band call with interior = 0 and halo
+ * pointers equal to the band's own first rows is the whole-grid call. */
+typedef struct swin_wattn_halo {
+  int32_t interior;
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dout; /* backward only */
+  void* out;        /* forward only */
+  float* lse;       /* forward only; used when the call's lse is not NULL */
+  void* dq;         /* backward only */
+  void* dk;
+  void* dv;
+} swin_wattn_halo;
+
+/* Forward and backward of one row band (tcgen05 kernels only:
+ * SWIN_ERR_UNSUPPORTED where swin_wattn_path != 1). Arguments as for
+ * swin_wattn_fwd / swin_wattn_bwd plus `halo`; dbias_table (or the exact sums
+ * under SWIN_FLAG_DBIAS_SUMS) covers the band's windows, so a grid's table is
+ * the sum over its bands. */
+int swin_wattn_fwd_band(const swin_wattn_desc* desc, const swin_wattn_halo* halo, const void* q,
+                        const void* k, const void* v, const float* bias_table, void* out,
+                        float* lse, void* workspace, size_t workspace_bytes, void* stream);
+int swin_wattn_bwd_band(const swin_wattn_desc* desc, const swin_wattn_halo* halo, const void* q,
+                        const void* k, const void* v, const float* bias_table, const void* dout,
+                        void* dq, void* dk, void* dv, float* dbias_table, void* workspace,
+                        size_t workspace_bytes, void* stream);
 
 /* Backward without a workspace argument, for callers that cannot allocate
  * device memory or hand over a workspace when they run it: hosts whose memory
@@ -134,10 +199,13 @@ int swin_wattn_bwd(const swin_wattn_desc* desc, const void* q, const void* k, co
  * undefined results. Each call clears the device status word before it runs;
  * a bounded device wait that runs out leaves the outputs undefined and is not
  * reported by this entry point.
+ * Arguments are checked on the host before anything is queued.
  * Returns SWIN_ERR_UNSUPPORTED when the description does not run on the
  * tcgen05 kernels (swin_wattn_path != 1) and SWIN_ERR_WORKSPACE when the
- * workspace it needs exceeds SWIN_NOALLOC_SCRATCH_BYTES (heads * padded
- * bias-table entries * 12 bytes + 768 bytes must fit). */
+ * workspace it needs exceeds SWIN_NOALLOC_SCRATCH_BYTES. That workspace is
+ * exactly 256 + r(heads * bp * 4) + r(heads * bp * 80) bytes, bp = bias-table
+ * entries rounded up to a multiple of 4, r() = round up to 256 (with 8 x 8
+ * windows, bp = 228: up to 54 heads fit). */
 #define SWIN_NOALLOC_SCRATCH_BYTES (1u << 20)
 int swin_wattn_bwd_noalloc(const swin_wattn_desc* desc, const void* q, const void* k,
                            const void* v, const float* bias_table, const void* dout, void* dq,
@@ -146,6 +214,32 @@ int swin_wattn_bwd_noalloc(const swin_wattn_desc* desc, const void* q, const voi
 /* Layout stage alone (steps 1-3): map[b, wy, wx, slot] = (b*H + y)*W + x, the
  * grid token that window slot holds, or -1 for a pad slot. */
 int swin_wattn_index_map(const swin_wattn_desc* desc, int32_t* map, void* stream);
+
+/* Where the exact bias-gradient sums of a SWIN_FLAG_DBIAS_SUMS backward sit
+ * in its workspace: `*offset` bytes from the start, `*bytes` long, int64 words
+ * [heads][bins rounded up to 4][10]. Sums of several calls (other images of
+ * a batch, other ranks of a data-parallel group) add word by word as int64
+ * (no carries needed), and swin_wattn_dbias_finish of the added words equals
+ * what one call over all of them would give, bit for bit. Host only;
+ * SWIN_ERR_UNSUPPORTED for the portable kernels (path 0). */
+int swin_wattn_dbias_sums(const swin_wattn_desc* desc, size_t* offset, size_t* bytes);
+
+/* Converts the exact sums at swin_wattn_dbias_sums' offset of `workspace` to
+ * dbias_table ([(2*win_h-1)*(2*win_w-1), heads] fp32, overwritten). */
+int swin_wattn_dbias_finish(const swin_wattn_desc* desc, const void* workspace,
+                            float* dbias_table, void* stream);
+
+/* Layout stage (steps 1-3) exactly as the tcgen05 kernels run it, for
+ * bit-exact checks of their addressing: fills `ids` (caller-owned device
+ * memory of B*H*W*heads*head_dim bf16 words, 16-byte aligned, overwritten)
+ * with token ids, loads every window's tile with the kernels' own TMA boxes
+ * and row order, and writes map[b, wy, wx, slot] = the grid token found in
+ * that slot's row (-1 for a pad slot; -2 where the loaded token disagrees
+ * with the token the kernels' epilogue would store to). `labels` (same shape,
+ * may be NULL) receives each slot's shift-region label 3*r_y + r_x.
+ * SWIN_ERR_UNSUPPORTED unless swin_wattn_path(desc) == 1. */
+int swin_wattn_layout_map(const swin_wattn_desc* desc, void* ids, int32_t* map, int32_t* labels,
+                          void* stream);
 
 /* Synchronises `stream`, then reads the device status word of `workspace`
  * (SWIN_OK or SWIN_ERR_TIMEOUT) into *device_status and clears it. */

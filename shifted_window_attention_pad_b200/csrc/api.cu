@@ -30,6 +30,8 @@ static int check_desc(const swin_wattn_desc* d) {
   if (d->heads < 1 || d->head_dim < 8 || d->head_dim > 256 || (d->head_dim & 7))
     return SWIN_ERR_INVALID_ARG;
   if (d->dtype != SWIN_DTYPE_F32 && d->dtype != SWIN_DTYPE_BF16) return SWIN_ERR_UNSUPPORTED;
+  if (d->valid_h < 0 || d->valid_h > d->H || d->valid_w < 0 || d->valid_w > d->W)
+    return SWIN_ERR_INVALID_ARG;
   const long long Hp = (d->H + d->win_h - 1) / d->win_h * (long long)d->win_h;
   const long long Wp = (d->W + d->win_w - 1) / d->win_w * (long long)d->win_w;
   // Token ids of the index map are int32; grid offsets stay far inside int64.
@@ -59,6 +61,20 @@ static size_t need_workspace(const swin_wattn_desc* d, const Geo& g) {
 static int check_ws(const swin_wattn_desc* d, const Geo& g, void* ws, size_t bytes) {
   if (!ws || ((uintptr_t)ws & 255u)) return SWIN_ERR_WORKSPACE;
   if (bytes < need_workspace(d, g)) return SWIN_ERR_WORKSPACE;
+  return SWIN_OK;
+}
+
+int check_bwd_args(const swin_wattn_desc* d, const void* q, const void* k, const void* v,
+                   const float* bias_table, const void* dout, const void* dq, const void* dk,
+                   const void* dv, const float* dbias_table) {
+  const int rc = check_desc(d);
+  if (rc) return rc;
+  const void* ptrs[] = {q, k, v, bias_table, dout, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return SWIN_ERR_INVALID_ARG;
+  // dbias_table is not written when the exact sums are left in the workspace
+  if (!(d->flags & SWIN_FLAG_DBIAS_SUMS) && !dbias_table) return SWIN_ERR_INVALID_ARG;
+  if (dbias_table && !aligned16(dbias_table)) return SWIN_ERR_INVALID_ARG;
   return SWIN_OK;
 }
 
@@ -107,26 +123,80 @@ int swin_wattn_fwd(const swin_wattn_desc* desc, const void* q, const void* k, co
 int swin_wattn_bwd(const swin_wattn_desc* desc, const void* q, const void* k, const void* v,
                    const float* bias_table, const void* dout, void* dq, void* dk, void* dv,
                    float* dbias_table, void* workspace, size_t workspace_bytes, void* stream) {
-  int rc = check_desc(desc);
+  int rc = check_bwd_args(desc, q, k, v, bias_table, dout, dq, dk, dv, dbias_table);
   if (rc) return rc;
-  if (!q || !k || !v || !bias_table || !dout || !dq || !dk || !dv || !dbias_table)
-    return SWIN_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, bias_table, dout, dq, dk, dv, dbias_table};
-  for (const void* p : ptrs)
-    if (!aligned16(p)) return SWIN_ERR_INVALID_ARG;
   const Geo g = make_geo(*desc);
   rc = check_ws(desc, g, workspace, workspace_bytes);
   if (rc) return rc;
   cudaStream_t st = (cudaStream_t)stream;
   const int path = choose_path(desc, g);
+  if (path == 0 && (desc->flags & SWIN_FLAG_DBIAS_SUMS)) return SWIN_ERR_UNSUPPORTED;
   if (path == 1)
     return cuda_status(fast_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
                                      workspace, desc->flags, st));
   if (path == 2)
     return cuda_status(tiled_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
-                                      workspace, st));
+                                      workspace, desc->flags, st));
   return cuda_status(generic_backward(g, desc->dtype, q, k, v, bias_table, dout, dq, dk, dv,
                                       dbias_table, workspace, st));
+}
+
+// Band geometry: the description is the band's own; the shift wraps into
+// the halo tensor, whose rows the band must be able to hold a window of.
+static int band_geo(const swin_wattn_desc* desc, const swin_wattn_halo* halo, Geo& g) {
+  if (!halo) return SWIN_ERR_INVALID_ARG;
+  g = make_geo(*desc);
+  if (choose_path(desc, g) != 1) return SWIN_ERR_UNSUPPORTED;
+  if (halo->interior && (desc->H % desc->win_h)) return SWIN_ERR_INVALID_ARG;
+  if (desc->H < desc->shift_h) return SWIN_ERR_INVALID_ARG;
+  if (desc->valid_h && desc->valid_h < desc->H && halo->interior) return SWIN_ERR_INVALID_ARG;
+  g.band = 1;
+  g.seam_h = halo->interior ? 0 : desc->shift_h;
+  return SWIN_OK;
+}
+
+int swin_wattn_fwd_band(const swin_wattn_desc* desc, const swin_wattn_halo* halo, const void* q,
+                        const void* k, const void* v, const float* bias_table, void* out,
+                        float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_desc(desc);
+  if (rc) return rc;
+  if (!q || !k || !v || !bias_table || !out) return SWIN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(bias_table) || (lse && !aligned16(lse)))
+    return SWIN_ERR_INVALID_ARG;
+  Geo g;
+  rc = band_geo(desc, halo, g);
+  if (rc) return rc;
+  if (desc->shift_h > 0) {
+    const void* hp[] = {halo->q, halo->k, halo->v, halo->out};
+    for (const void* p : hp)
+      if (!p || !aligned16(p)) return SWIN_ERR_INVALID_ARG;
+    if (lse && (!halo->lse || !aligned16(halo->lse))) return SWIN_ERR_INVALID_ARG;
+  }
+  rc = check_ws(desc, g, workspace, workspace_bytes);
+  if (rc) return rc;
+  return cuda_status(fast_forward(g, q, k, v, bias_table, out, lse, workspace, desc->flags,
+                                  (cudaStream_t)stream, halo));
+}
+
+int swin_wattn_bwd_band(const swin_wattn_desc* desc, const swin_wattn_halo* halo, const void* q,
+                        const void* k, const void* v, const float* bias_table, const void* dout,
+                        void* dq, void* dk, void* dv, float* dbias_table, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  int rc = check_bwd_args(desc, q, k, v, bias_table, dout, dq, dk, dv, dbias_table);
+  if (rc) return rc;
+  Geo g;
+  rc = band_geo(desc, halo, g);
+  if (rc) return rc;
+  if (desc->shift_h > 0) {
+    const void* hp[] = {halo->q, halo->k, halo->v, halo->dout, halo->dq, halo->dk, halo->dv};
+    for (const void* p : hp)
+      if (!p || !aligned16(p)) return SWIN_ERR_INVALID_ARG;
+  }
+  rc = check_ws(desc, g, workspace, workspace_bytes);
+  if (rc) return rc;
+  return cuda_status(fast_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
+                                   workspace, desc->flags, (cudaStream_t)stream, halo));
 }
 
 int swin_wattn_index_map(const swin_wattn_desc* desc, int32_t* map, void* stream) {
@@ -134,6 +204,39 @@ int swin_wattn_index_map(const swin_wattn_desc* desc, int32_t* map, void* stream
   if (rc) return rc;
   if (!map) return SWIN_ERR_INVALID_ARG;
   return cuda_status(index_map(make_geo(*desc), map, (cudaStream_t)stream));
+}
+
+int swin_wattn_dbias_sums(const swin_wattn_desc* desc, size_t* offset, size_t* bytes) {
+  const int rc = check_desc(desc);
+  if (rc) return rc;
+  if (!offset || !bytes) return SWIN_ERR_INVALID_ARG;
+  const Geo g = make_geo(*desc);
+  if (choose_path(desc, g) == 0) return SWIN_ERR_UNSUPPORTED;
+  *offset = dbias_fixed_offset(g);
+  *bytes = dbias_fixed_bytes(g);
+  return SWIN_OK;
+}
+
+int swin_wattn_dbias_finish(const swin_wattn_desc* desc, const void* workspace,
+                            float* dbias_table, void* stream) {
+  const int rc = check_desc(desc);
+  if (rc) return rc;
+  if (!dbias_table || !aligned16(dbias_table)) return SWIN_ERR_INVALID_ARG;
+  if (!workspace || ((uintptr_t)workspace & 255u)) return SWIN_ERR_WORKSPACE;
+  const Geo g = make_geo(*desc);
+  if (choose_path(desc, g) == 0) return SWIN_ERR_UNSUPPORTED;
+  const long long* acc = (const long long*)((const char*)workspace + dbias_fixed_offset(g));
+  return cuda_status(finish_dbias(g, acc, dbias_table, (cudaStream_t)stream));
+}
+
+int swin_wattn_layout_map(const swin_wattn_desc* desc, void* ids, int32_t* map,
+                          int32_t* labels, void* stream) {
+  const int rc = check_desc(desc);
+  if (rc) return rc;
+  if (!ids || !map || !aligned16(ids)) return SWIN_ERR_INVALID_ARG;
+  const Geo g = make_geo(*desc);
+  if (choose_path(desc, g) != 1) return SWIN_ERR_UNSUPPORTED;
+  return cuda_status(fast_layout_map(g, ids, map, labels, (cudaStream_t)stream));
 }
 
 int swin_wattn_poll_status(void* workspace, int* device_status, void* stream) {

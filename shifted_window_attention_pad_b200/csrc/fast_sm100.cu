@@ -26,18 +26,19 @@
 //    from per-slot coordinates (no mask tensor), runs the softmax in registers
 //    (a whole window row is in the tile, so no running rescale is needed), writes
 //    P (and dS) to shared memory for the next MMAs, and stores outputs straight
-//    to their grid rows. The bias-table gradient is summed in fixed point
-//    (units of 2^-16): a tile's bins are int32 shared-memory reductions, folded
-//    per tile into one int64 table in global memory with global reductions.
-//    Integer sums are exact and do not depend on the order in which threads or
-//    CTAs land, so the result is bitwise repeatable; a last small kernel
-//    converts it to fp32.
+//    to their grid rows. The bias-table gradient is summed exactly in integers
+//    (dbias_fixed.cuh): per tile, a bound on |dS| sets the unit 2^-E of int32
+//    shared-memory bins, and the tile's bins are folded into wide integer sums
+//    in global memory. Integer sums do not depend on the order in which
+//    threads or CTAs land, so the result is bitwise repeatable, and the unit
+//    follows the magnitude of the gradients, so the relative error does not
+//    depend on their scale; a last small kernel converts the sums to fp32.
 //  * Warp roles: warps 0-3 and 4-7 two softmax/epilogue warpgroups taking
-//    alternate tiles, warp 8 TMA producer, warp 9 issues S (and dP) and owns
-//    TMEM, warp 10 issues PV (or the gradient products), warp 11 (backward)
-//    TMA-stores the staged gradients. Persistent grid of one CTA per SM; tiles
-//    go round-robin, head fastest, so the SMs stream neighbouring bytes
-//    together.
+//    alternate tiles, warp 8 TMA producer (which also prefetches the tiles
+//    of the steps ahead into L2), warp 9 issues S (and dP) and owns TMEM,
+//    warp 10 issues PV (or the gradient products). Persistent grid of one
+//    CTA per SM; tiles go round-robin, head fastest, so the SMs stream
+//    neighbouring bytes together.
 //  * Every mbarrier wait is bounded (%globaltimer); a wait that runs out records
 //    a timeout in the workspace status word and the kernel drains and returns.
 #include <cuda.h>
@@ -48,6 +49,7 @@
 
 #include <mutex>
 
+#include "dbias_fixed.cuh"
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -62,8 +64,7 @@ constexpr int kNumWg = 2;         // warpgroups 0 (warps 0-3) and 1 (warps 4-7) 
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;       // issues S (and dP); allocates and frees TMEM
 constexpr int kMma2Warp = 10;     // issues PV (forward) or the gradient products (backward)
-constexpr int kStoreWarp = 11;    // backward: TMA-stores the staged gradients
-constexpr int kThreads = 384;
+constexpr int kThreads = 352;
 constexpr int kMaxMaps = 9;       // box shapes: {full, seam part 1, seam part 2}^2
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestLimitNs = 1000000ull;
@@ -71,7 +72,6 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct FastParams {
   CUtensorMap maps[4][kMaxMaps];  // [q, k, v, dout][ky * 3 + kx]
-  CUtensorMap omaps[3][kMaxMaps]; // outputs: forward [out]; backward [dq, dk, dv]
   Geo g;
   long long n_groups;             // tiles per head: ceil(n_win / G)
   long long n_tiles;              // n_groups * heads
@@ -82,20 +82,36 @@ struct FastParams {
   void* out1;                     // backward: dk
   void* out2;                     // backward: dv
   float* lse;                     // forward, optional
-  long long* dt_fixed;            // backward: bias gradient [heads][bins_pad], units of 2^-16
+  void* out0h;                    // row band: outputs of the halo rows (same roles)
+  void* out1h;
+  void* out2h;
+  float* lse_h;
+  long long* dt_acc;              // backward: exact bias-gradient sums [heads][bins_pad][kLimbStride]
   int* status;                    // device status word (workspace header)
   int test_timeout;
 };
 
 // ---- shared-memory layout (same arithmetic on host and device) ------------------
+// A TMA box carries at most 64 channels (128 bytes, the swizzle span), so a
+// head_dim of 128 is loaded as two channel halves, each a [128 rows][64]
+// region of its own; smaller head_dims are one region of [128 rows][HD].
+template <int HD>
+struct TileGeom {
+  static constexpr int kBoxEl = HD > 64 ? 64 : HD;            // channels of one box
+  static constexpr int kHalves = HD / kBoxEl;
+  static constexpr uint32_t kRowBytes = kBoxEl * 2;           // a row inside one region
+  static constexpr uint32_t kHalfBytes = kRows * kRowBytes;   // one region
+  static constexpr int kStepsPerHalf = kBoxEl / 16;           // K steps of 16 per region
+};
+
 struct Layout {
   uint32_t tiles, ptile, bias, colinfo, bins_w, bars, misc, total;
 };
 
 // NS stages of NTEN input tiles, then PBYTES of P / dS operand blocks, the
-// bias rows of the stages, per warpgroup two buffers of key words and the
-// tile's bias-gradient bins (two fixed-point int32 parts), mbarriers and two
-// words (TMEM base, abort flag).
+// bias rows of the stages, per warpgroup two buffers of key words, the tile's
+// int32 bias-gradient bins and four per-warp bounds, mbarriers and two words
+// (TMEM base, abort flag).
 template <int HD, int NS, int NTEN, uint32_t PBYTES>
 __host__ __device__ inline Layout make_layout(int bins_pad) {
   constexpr uint32_t tile_bytes = kRows * HD * 2;
@@ -105,7 +121,7 @@ __host__ __device__ inline Layout make_layout(int bins_pad) {
   L.bias = L.ptile + PBYTES;
   L.colinfo = L.bias + ((NS * bins_pad * 4 + 15) & ~15);
   L.bins_w = L.colinfo + kNumWg * 2 * kRows * 4;
-  L.bars = (L.bins_w + kNumWg * bins_pad * 8 + 7) & ~7u;
+  L.bars = (L.bins_w + kNumWg * (bins_pad + 4) * 4 + 7) & ~7u;
   L.misc = L.bars + 8 * 32;
   L.total = L.misc + 16;
   return L;
@@ -178,7 +194,9 @@ __device__ inline void row_slot(const Geo& g, int wy, int wx, int r, int& iy, in
 
 // Everything the softmax warpgroup needs to know about its own row.
 struct RowInfo {
-  bool valid;
+  bool valid;       // a real token (inside the valid extent)
+  bool stored;      // inside the stored grid: its outputs are written
+  bool halo;        // row band: a row of the halo tensor (token counts in its [B, sh, W])
   int label;        // shift region 0..8
   int bias_base;    // (iy + wh - 1)(2 ww - 1) + ix + ww - 1
   int key_off;      // iy (2 ww - 1) + ix : subtract from a query's base to index the table
@@ -188,6 +206,8 @@ struct RowInfo {
 __device__ inline RowInfo row_info(const Geo& g, long long win, int r) {
   RowInfo ri;
   ri.valid = false;
+  ri.stored = false;
+  ri.halo = false;
   ri.label = 15;
   ri.bias_base = 0;
   ri.key_off = 0;
@@ -198,11 +218,18 @@ __device__ inline RowInfo row_info(const Geo& g, long long win, int r) {
   row_slot(g, wy, wx, r, iy, ix);
   const int yr = wy * g.wh + iy, xr = wx * g.ww + ix;
   const int y = (yr + g.sh) % g.Hp, x = (xr + g.sw) % g.Wp;
-  ri.valid = y < g.H && x < g.W;
-  ri.label = 3 * region_1d(yr, g.Hp, g.wh, g.sh) + region_1d(xr, g.Wp, g.ww, g.sw);
+  ri.stored = y < g.H && x < g.W;
+  ri.valid = y < g.Hv && x < g.Wv;
+  ri.label = 3 * region_1d(yr, g.Hp, g.wh, g.seam_h) + region_1d(xr, g.Wp, g.ww, g.sw);
   ri.bias_base = (iy + g.wh - 1) * (2 * g.ww - 1) + ix + g.ww - 1;
   ri.key_off = iy * (2 * g.ww - 1) + ix;
   ri.token = ((long long)b * g.H + y) * g.W + x;
+  if (g.band && yr + g.sh >= g.Hp) {   // wrapped row: source row y < sh of the halo tensor
+    ri.halo = true;
+    ri.stored = x < g.W;
+    ri.valid = x < g.Wv;
+    ri.token = ((long long)b * g.sh + y) * g.W + x;
+  }
   return ri;
 }
 
@@ -220,8 +247,9 @@ __device__ inline void issue_tile_loads(const FastParams& p, long long t, uint8_
   const int G = kRows / g.N;
   const long long group = t / g.heads;
   const int h = (int)(t - group * g.heads);
-  constexpr uint32_t row_bytes = HD * 2;
-  constexpr uint32_t tile_bytes = kRows * row_bytes;
+  using T = TileGeom<HD>;
+  constexpr uint32_t row_bytes = T::kRowBytes;
+  constexpr uint32_t tile_bytes = kRows * HD * 2;
   for (int gw = 0; gw < G; ++gw) {
     const long long win = group * G + gw;
     const uint32_t row0 = gw * g.N;
@@ -232,32 +260,31 @@ __device__ inline void issue_tile_loads(const FastParams& p, long long t, uint8_
       const int n = plan_window(g, wy, wx, sb);
       for (int i = 0; i < n; ++i)
         for (int tt = 0; tt < NTEN; ++tt)
-          tma_load_5d(tiles + tt * tile_bytes + (row0 + sb[i].row_off) * row_bytes,
-                      &p.maps[tt][sb[i].map_id], full, 0, h, sb[i].x, sb[i].y, b);
+          for (int hf = 0; hf < T::kHalves; ++hf)
+            tma_load_5d(tiles + tt * tile_bytes + hf * T::kHalfBytes +
+                            (row0 + sb[i].row_off) * row_bytes,
+                        &p.maps[tt][sb[i].map_id], full, hf * T::kBoxEl, h, sb[i].x, sb[i].y, b);
     } else {
       // No such window: a box wholly above the grid reads zeros and keeps the
       // transaction count uniform.
       for (int tt = 0; tt < NTEN; ++tt)
-        tma_load_5d(tiles + tt * tile_bytes + row0 * row_bytes, &p.maps[tt][0], full, 0, h, 0,
-                    -g.wh, 0);
+        for (int hf = 0; hf < T::kHalves; ++hf)
+          tma_load_5d(tiles + tt * tile_bytes + hf * T::kHalfBytes + row0 * row_bytes,
+                      &p.maps[tt][0], full, hf * T::kBoxEl, h, 0, -g.wh, 0);
     }
   }
-  bulk_load(bias_dst, p.bias_t + (size_t)h * p.bins_pad, p.bins_pad * 4, full);
+  if (bias_dst) bulk_load(bias_dst, p.bias_t + (size_t)h * p.bins_pad, p.bins_pad * 4, full);
 }
 
-// One elected thread: TMA-stores the staged output rows of tile `t` with the
-// same sub-box decomposition as the loads, for NOUT tensors. Window gw of
-// tensor tt is staged at staged + tt * tile_stride + gw * win_stride, rows of
-// HD bf16 back to back in sub-box order. Sub-boxes wholly in the padding are
-// skipped; the others are clipped to the grid by the TMA unit.
-template <int HD, int NOUT>
-__device__ inline void issue_tile_stores(const FastParams& p, long long t, const uint8_t* staged,
-                                         uint32_t tile_stride, uint32_t win_stride) {
+// Producer: asks the TMA unit to bring the boxes of tile `t` into L2 ahead of
+// their shared-memory loads, so that those find the tile in L2 instead of
+// waiting for HBM. No barrier is involved and nothing lands in shared memory.
+template <int HD, int NTEN>
+__device__ inline void issue_tile_prefetch(const FastParams& p, long long t) {
   const Geo& g = p.g;
   const int G = kRows / g.N;
   const long long group = t / g.heads;
   const int h = (int)(t - group * g.heads);
-  constexpr uint32_t row_bytes = HD * 2;
   for (int gw = 0; gw < G; ++gw) {
     const long long win = group * G + gw;
     if (win >= g.n_win) continue;
@@ -266,74 +293,35 @@ __device__ inline void issue_tile_stores(const FastParams& p, long long t, const
     SubBox sb[4];
     const int n = plan_window(g, wy, wx, sb);
     for (int i = 0; i < n; ++i) {
-      if (sb[i].y >= g.H || sb[i].x >= g.W) continue;
-      for (int tt = 0; tt < NOUT; ++tt)
-        tma_store_5d(&p.omaps[tt][sb[i].map_id],
-                     staged + tt * tile_stride + gw * win_stride + sb[i].row_off * row_bytes, 0,
-                     h, sb[i].x, sb[i].y, b);
+      if (sb[i].y >= g.H || sb[i].x >= g.W) continue;   // wholly in the padding
+      for (int tt = 0; tt < NTEN; ++tt)
+        for (int hf = 0; hf < TileGeom<HD>::kHalves; ++hf)
+          tma_prefetch_5d(&p.maps[tt][sb[i].map_id], hf * TileGeom<HD>::kBoxEl, h, sb[i].x,
+                          sb[i].y, b);
     }
   }
-  bulk_commit_group();
 }
 
-// The same for the three backward outputs staged in the operand-block area
-// (dV at bwd_stage(0), dQ at bwd_stage(1), dK at bwd_stage(2)).
-__host__ __device__ constexpr uint32_t bwd_stage(int part);
-template <int HD>
-__device__ inline void issue_tile_stores3(const FastParams& p, long long t, const uint8_t* staged) {
-  const Geo& g = p.g;
-  const int G = kRows / g.N;
-  const long long group = t / g.heads;
-  const int h = (int)(t - group * g.heads);
-  constexpr uint32_t row_bytes = HD * 2;
-  for (int gw = 0; gw < G; ++gw) {
-    const long long win = group * G + gw;
-    if (win >= g.n_win) continue;
-    int b, wy, wx;
-    window_coords(g, win, b, wy, wx);
-    SubBox sb[4];
-    const int n = plan_window(g, wy, wx, sb);
-    for (int i = 0; i < n; ++i) {
-      if (sb[i].y >= g.H || sb[i].x >= g.W) continue;
-      const uint32_t r = (gw * g.N + sb[i].row_off) * row_bytes;
-      tma_store_5d(&p.omaps[0][sb[i].map_id], staged + bwd_stage(1) + r, 0, h, sb[i].x, sb[i].y, b);
-      tma_store_5d(&p.omaps[1][sb[i].map_id], staged + bwd_stage(2) + r, 0, h, sb[i].x, sb[i].y, b);
-      tma_store_5d(&p.omaps[2][sb[i].map_id], staged + bwd_stage(0) + r, 0, h, sb[i].x, sb[i].y, b);
-    }
-  }
-  bulk_commit_group();
-}
-
-// Stages one output row of HD values (times `mul`, rounded to bf16) at
-// row_addr, with the tensor maps' swizzle (128-byte for HD = 64, 64-byte for
-// HD = 32: 16-byte chunk index XOR address bits 7.., on a 1024-aligned buffer).
-template <int HD>
-__device__ inline void stage_row(uint32_t row_addr, const float* v, float mul) {
-#pragma unroll
-  for (int c = 0; c < HD / 8; ++c) {
-    const uint32_t off = row_addr + c * 16;
-    const uint32_t swz = HD == 64 ? ((off >> 7) & 7) : ((off >> 7) & 3);
-    st_shared_v4(off ^ (swz << 4), pack_bf16(v[c * 8 + 0] * mul, v[c * 8 + 1] * mul),
-                 pack_bf16(v[c * 8 + 2] * mul, v[c * 8 + 3] * mul),
-                 pack_bf16(v[c * 8 + 4] * mul, v[c * 8 + 5] * mul),
-                 pack_bf16(v[c * 8 + 6] * mul, v[c * 8 + 7] * mul));
-  }
-}
-
-// K-major operand, rows of HD bf16 (128-byte swizzle for HD = 64, 64-byte for 32),
-// advanced by k16 steps of 16 elements along K.
+// K-major operand, rows of HD bf16 (128-byte swizzle for HD >= 64, 64-byte for
+// 32), advanced by k16 steps of 16 elements along K; with two channel
+// regions (HD = 128) steps 4-7 move to the second region.
 template <int HD>
 __device__ inline uint64_t desc_kmajor_tile(uint32_t base, int k16) {
-  constexpr uint32_t row_bytes = HD * 2;
-  constexpr uint32_t sw = HD == 64 ? kSwizzle128 : kSwizzle64;
-  return smem_desc(base + k16 * 32, 16, 8 * row_bytes, sw);
+  using T = TileGeom<HD>;
+  constexpr uint32_t sw = HD >= 64 ? kSwizzle128 : kSwizzle64;
+  return smem_desc(base + (k16 / T::kStepsPerHalf) * T::kHalfBytes +
+                       (k16 % T::kStepsPerHalf) * 32,
+                   16, 8 * T::kRowBytes, sw);
 }
-// MN-major operand (the HD columns are N), K = tile rows, 16 rows per step.
+// MN-major operand (the HD columns are N), K = tile rows, 16 rows per step;
+// with two channel regions (HD = 128) the second 64 columns of N are the next
+// region, one leading byte offset away.
 template <int HD>
 __device__ inline uint64_t desc_mnmajor_tile(uint32_t base, int k16) {
-  constexpr uint32_t row_bytes = HD * 2;
-  constexpr uint32_t sw = HD == 64 ? kSwizzle128 : kSwizzle64;
-  return smem_desc(base + k16 * 16 * row_bytes, 8 * row_bytes, 8 * row_bytes, sw);
+  using T = TileGeom<HD>;
+  constexpr uint32_t sw = HD >= 64 ? kSwizzle128 : kSwizzle64;
+  return smem_desc(base + k16 * 16 * T::kRowBytes,
+                   T::kHalves > 1 ? T::kHalfBytes : 8 * T::kRowBytes, 8 * T::kRowBytes, sw);
 }
 // P / dS tile: 128 rows x 128 columns bf16 as two 16 KB regions of 64 columns,
 // 128-byte swizzle. As K-major A (M = rows, K = columns):
@@ -393,7 +381,7 @@ __device__ inline bool window_plain(const Geo& g, long long win) {
   window_coords(g, win, b, wy, wx);
   if (g.sh > 0 && wy == g.nWy - 1) return false;
   if (g.sw > 0 && wx == g.nWx - 1) return false;
-  return wy * g.wh + g.sh + g.wh <= g.H && wx * g.ww + g.sw + g.ww <= g.W;
+  return wy * g.wh + g.sh + g.wh <= g.Hv && wx * g.ww + g.sw + g.ww <= g.Wv;
 }
 
 template <int WW>
@@ -403,6 +391,8 @@ __device__ inline RowInfo plain_row_info(const Geo& g, long long win, int r) {
   const int iy = r / (WW > 0 ? WW : 1), ix = r % (WW > 0 ? WW : 1);
   RowInfo ri;
   ri.valid = true;
+  ri.stored = true;
+  ri.halo = false;
   ri.label = 0;
   ri.bias_base = (iy + WW - 1) * (2 * WW - 1) + ix + WW - 1;
   ri.key_off = iy * (2 * WW - 1) + ix;
@@ -469,10 +459,21 @@ __device__ inline float exp_sum(float* x, float m) {
 // while one waits on TMEM loads or an MMA the other computes (two warps per
 // scheduler). One thread issues S of each tile as soon as its data and TMEM
 // slot are ready, another PV as soon as its P is written.
-// Four TMEM slots of 128 columns (S, then O in the first HD), one P tile per
-// warpgroup, three input stages.
-constexpr int kFwdStages = 3;
-constexpr int kFwdSlots = 4;
+// HD <= 64: four TMEM slots of 128 columns (S, then O in the first HD), one
+// P tile per warpgroup in shared memory, three input stages.
+// HD = 128: three 96 KB stages and the P tiles do not fit in shared memory,
+// so P stays in TMEM: two slots of 256 columns, S in the first 128 (P
+// overwrites its first 64 as packed bf16 pairs, the A operand of O = P V),
+// O in the last 128; two input stages.
+template <int HD>
+struct FwdCfg {
+  static constexpr bool kTmemP = HD > 64;
+  static constexpr int kStages = kTmemP ? 2 : 3;
+  static constexpr int kSlots = kTmemP ? 2 : 4;
+  static constexpr uint32_t kSlotCols = kTmemP ? 256 : 128;
+  static constexpr uint32_t kOCol = kTmemP ? 128 : 0;    // O inside its slot
+  static constexpr uint32_t kPBytes = kTmemP ? 0 : kNumWg * 32768;
+};
 constexpr int kFwdPBufs = kNumWg;
 
 
@@ -486,10 +487,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   constexpr int N = 64, G = kRows / N;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  constexpr int NS = kFwdStages, NT = kFwdSlots;
+  using C = FwdCfg<HD>;
+  constexpr int NS = C::kStages, NT = C::kSlots;
+  constexpr uint32_t SC = C::kSlotCols;
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   const Geo& g = p.g;
-  const Layout L = make_layout<HD, NS, 3, kFwdPBufs * 32768>(p.bins_pad);
+  const Layout L = make_layout<HD, NS, 3, C::kPBytes>(p.bins_pad);
   uint8_t* tiles = smem + L.tiles;
   uint8_t* ptile = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
@@ -524,8 +527,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     for (int tt = 0; tt < 3; ++tt)
       for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
   // P tiles start at zero: rows never write the columns of the other window.
-  for (uint32_t i = threadIdx.x; i < kFwdPBufs * 32768 / 16; i += kThreads)
-    reinterpret_cast<uint4*>(ptile)[i] = make_uint4(0, 0, 0, 0);
+  if constexpr (C::kPBytes > 0)
+    for (uint32_t i = threadIdx.x; i < C::kPBytes / 16; i += kThreads)
+      reinterpret_cast<uint4*>(ptile)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async();
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
@@ -538,6 +542,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
+      const long long ahead = (long long)NS * gridDim.x;
+      for (long long t = blockIdx.x; t < p.n_tiles && t < blockIdx.x + ahead; t += gridDim.x)
+        issue_tile_prefetch<HD, 3>(p, t);
       long long k = 0;
       for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
         const int s = (int)(k % NS);
@@ -545,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (!mbar_wait(&empty[s], ph ^ 1, abort, p.status, kWaitLimitNs)) break;
         mbar_arrive_expect_tx(&full[s], 3 * tile_bytes + p.bins_pad * 4);
         issue_tile_loads<HD, 3>(p, t, tiles + s * 3 * tile_bytes, bias + s * p.bins_pad, &full[s]);
+        if (t + ahead < p.n_tiles) issue_tile_prefetch<HD, 3>(p, t + ahead);
       }
       if (*abort) {  // let copies already in flight land before the CTA leaves
         const long long first = k > NS ? k - NS : 0;
@@ -566,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         const uint32_t k_s = smem_u32(tiles + (s * 3 + 1) * tile_bytes);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk)
-          umma_ss(tmem + sl * 128, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk),
+          umma_ss(tmem + sl * SC, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk),
                   idesc_s, kk);
         umma_commit(&s_full[sl]);
       }
@@ -584,11 +592,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           break;
         tc_fence_after();
         const uint32_t v_s = smem_u32(tiles + (s * 3 + 2) * tile_bytes);
-        const uint32_t p_s = smem_u32(ptile + (k % kFwdPBufs) * 32768);
+        if constexpr (C::kTmemP) {
+          // A = P from TMEM: 16 keys per step are 8 columns of bf16 pairs
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)
-          umma_ss(tmem + sl * 128, desc_p_kmajor(p_s, kk), desc_mnmajor_tile<HD>(v_s, kk),
-                  idesc_o, kk);
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            umma_ts(tmem + sl * SC + C::kOCol, tmem + sl * SC + kk * 8,
+                    desc_mnmajor_tile<HD>(v_s, kk), idesc_o, kk);
+        } else {
+          const uint32_t p_s = smem_u32(ptile + (k % kFwdPBufs) * 32768);
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            umma_ss(tmem + sl * SC, desc_p_kmajor(p_s, kk), desc_mnmajor_tile<HD>(v_s, kk),
+                    idesc_o, kk);
+        }
         umma_commit(&o_full[sl]);
         umma_commit(&empty[s]);
       }
@@ -598,13 +614,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       }
     }
   } else if (warp < kNumWg * 4) {
-    // Softmax / epilogue warpgroups: thread = tile row = TMEM lane. (Warp 11
-    // has no role in the forward and goes straight to the final barrier.)
+    // Softmax / epilogue warpgroups: thread = tile row = TMEM lane.
     const int wg = warp >> 2;
     const int row = threadIdx.x & (kWg - 1);
     const int gw = row / N, lr = row - gw * N;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t p_s = smem_u32(ptile + wg * 32768);
+    const uint32_t p_s = C::kTmemP ? 0u : smem_u32(ptile + wg * 32768);
     long long k = wg;
     for (long long t = blockIdx.x + wg * (long long)gridDim.x; t < p.n_tiles;
          t += kNumWg * (long long)gridDim.x, k += kNumWg) {
@@ -623,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
       tc_fence_after();
       float x[N];
-      tmem_load_cols<N>(tmem + lane_base + sl * 128 + gw * N, x);
+      tmem_load_cols<N>(tmem + lane_base + sl * SC + gw * N, x);
       tmem_wait_ld();
       const float* brow = bias + s * p.bins_pad;
       float m;
@@ -638,8 +653,24 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
         for (int j = 0; j < N; ++j) x[j] = 0.f;
       }
-      store_p_row<N>(p_s, row, gw * N, x);
-      fence_proxy_async();
+      if constexpr (C::kTmemP) {
+        // this row's P as bf16 pairs over the tile's 128 keys: the other
+        // window's 64 keys are zeros
+        uint32_t w0[32], w1[32];   // columns 0-31 (keys 0-63), 32-63 (keys 64-127)
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const uint32_t w = pack_bf16(x[2 * c], x[2 * c + 1]);
+          w0[c] = gw ? 0u : w;
+          w1[c] = gw ? w : 0u;
+        }
+        __syncwarp();
+        tmem_st32u(tmem + lane_base + sl * SC + 0, w0);
+        tmem_st32u(tmem + lane_base + sl * SC + 32, w1);
+        tmem_wait_st();
+      } else {
+        store_p_row<N>(p_s, row, gw * N, x);
+        fence_proxy_async();
+      }
       tc_fence_before();
       mbar_arrive(&p_full[sl]);
       // epilogue: O row from TMEM, normalised, straight to its grid token
@@ -647,16 +678,26 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       mbar_wait(&o_full[sl], pht, abort, p.status, kWaitLimitNs);
       tc_fence_after();
       {
-        float o[HD];
-        tmem_load_cols<HD>(tmem + lane_base + sl * 128, o);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&t_empty[sl]);
-        if (me.valid && !*abort)
-          store_row_bf16<HD>((__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD, o, 1.f / l);
+        // (rows beyond the valid extent hold P = 0, so O = 0 is stored there)
+        __nv_bfloat16* dst = (__nv_bfloat16*)(me.halo ? p.out0h : p.out0) +
+                             (me.token * g.heads + h) * HD;
+        constexpr int OC = HD > 64 ? 64 : HD;   // columns per TMEM read
+#pragma unroll
+        for (int c0 = 0; c0 < HD; c0 += OC) {
+          float o[OC];
+          tmem_load_cols<OC>(tmem + lane_base + sl * SC + C::kOCol + c0, o);
+          tmem_wait_ld();
+          if (c0 + OC == HD) {
+            tc_fence_before();
+            mbar_arrive(&t_empty[sl]);
+          }
+          if (me.stored && !*abort) store_row_bf16<OC>(dst + c0, o, 1.f / l);
+        }
       }
-      if (me.valid && !*abort && p.lse)
-        p.lse[me.token * g.heads + h] = (m + __log2f(l)) * 0.69314718055994531f;
+      float* lse_out = me.halo ? p.lse_h : p.lse;
+      if (me.stored && !*abort && lse_out)
+        lse_out[me.token * g.heads + h] =
+            me.valid ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
     }
   }
   tc_fence_before();
@@ -686,24 +727,33 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 //
 // Two warpgroups take alternate tiles, each with its own TMEM slot of 256
 // columns (S | dP, then dV | dQ | dK). The operand blocks are shared: tile k
-// writes them once the gradient products of tile k-1 have completed. One thread
-// issues S and dP of each tile as soon as its data and slot are ready, another
-// the gradient products as soon as its blocks are written.
-constexpr int kBwdStages = 2;
-constexpr int kBwdSlots = 2;
+// writes them as soon as the gradient products of tile k-1 have completed
+// (nothing else lives there), and each warpgroup stores its gradient rows
+// straight from registers to their grid tokens. One thread issues S and dP of
+// each tile as soon as its data and slot are ready, another the gradient
+// products as soon as its blocks are written; the producer also asks for the
+// tiles two steps ahead to be brought into L2.
+//
+// Bias-table gradient: per tile, a bound on |dS| (max P of the row times
+// max|dP| + |D|, maximised over the tile's rows) sets the exponent of an exact
+// fixed-point sum in int32 shared bins; the tile's bins are then added into
+// the wide integer sums of the workspace (dbias_fixed.cuh).
+// HD <= 64: two input stages, two TMEM slots of 256 columns (S | dP, then
+// dV | dQ | dK at 0 / 64 / 128), the two softmax warpgroups on alternate
+// tiles. HD = 128: a stage of four 32 KB tiles leaves room for one (the L2
+// prefetch keeps its refill short), and the three 128-column gradients need
+// 384 columns, so one slot (dV | dQ | dK at 0 / 128 / 256 over S | dP) and
+// one softmax warpgroup.
+template <int HD>
+struct BwdCfg {
+  static constexpr bool kWide = HD > 64;
+  static constexpr int kStages = kWide ? 1 : 2;
+  static constexpr int kSlots = kWide ? 1 : 2;
+  static constexpr int kWarpgroups = kWide ? 1 : kNumWg;
+  static constexpr uint32_t kGradCols = kWide ? 128 : 64;   // dV, dQ, dK spacing
+};
 constexpr uint32_t kBlk = 8192;
 enum { kP0h = 0, kP0l, kS0h, kZ1, kS1h, kS0l, kZ2, kS1l, kP1h, kP1l, kNumBlk };
-// Fixed point of the bias-gradient sums, in units of 2^-16: a dS below 64 in
-// magnitude goes whole into the low int32 part; larger ones (|dS| < 2^22) are
-// split into an integer high part and a low remainder. A tile's bins hold at
-// most 128 terms, so neither part can overflow; the global table is int64.
-constexpr double kFixInv = 1.52587890625e-05;  // 2^-16
-// Output staging in the operand-block area, clear of the zero blocks Z1
-// (24-32 KB) and Z2 (48-56 KB): dV at 0, dQ at 32 KB, dK at 56 KB, each
-// 128 rows of HD bf16.
-__host__ __device__ constexpr uint32_t bwd_stage(int part) {
-  return part == 0 ? 0u : (part == 1 ? 32768u : 57344u);
-}
 
 __device__ inline uint64_t desc_blk_kmajor(uint32_t base, int blk0, int blk1, int k16) {
   // keys [0,64) read the run starting at blk0, keys [64,128) the run at blk1
@@ -740,10 +790,10 @@ __device__ inline void store_split_cols_part(uint32_t blk_hi, uint32_t blk_lo, i
   }
 }
 
-// x (|x| < 2^22) rounded to the nearest integer with the float adder:
-// adding 1.5 * 2^23 leaves round(x) in the low mantissa bits.
-__device__ inline int round_int_fma(float x) {
-  return __float_as_int(x + 12582912.0f) - 0x4B400000;
+__device__ inline float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
 }
 
 template <int HD, int WW>
@@ -751,7 +801,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   constexpr int N = 64, G = kRows / N;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  constexpr int NS = kBwdStages, NT = kBwdSlots;
+  using C = BwdCfg<HD>;
+  constexpr int NS = C::kStages, NT = C::kSlots, NWG = C::kWarpgroups;
+  constexpr uint32_t GC = C::kGradCols;
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   const Geo& g = p.g;
   const int bp = p.bins_pad;
@@ -760,7 +812,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* blocks = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
   uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
-  int* bins = (int*)(smem + L.bins_w);   // [wg][hi, lo][bins_pad]
+  int* bins = (int*)(smem + L.bins_w);           // [wg][bins_pad] tile bins
+  float* tbound = (float*)(bins + kNumWg * bp);  // [wg][4] per-warp |dS| bounds
   uint64_t* bars = (uint64_t*)(smem + L.bars);
   uint64_t* full = bars;
   uint64_t* empty = full + NS;
@@ -770,8 +823,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint64_t* t_empty = grad_full + NT;
   uint64_t* drain = t_empty + NT;   // [2]: one per MMA-issuing thread
   uint64_t* never = drain + 2;
-  uint64_t* blk_free = never + 1;   // operand-block area free of staged outputs
-  uint64_t* staged = blk_free + 1;  // a tile's gradients are staged in the block area
   uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
   volatile int* abort = (volatile int*)(smem + L.misc + 4);
 
@@ -786,8 +837,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     mbar_init(never, 1);
-    mbar_init(blk_free, 1);
-    mbar_init(staged, kWg);
     *abort = 0;
     fence_mbar_init();
   }
@@ -798,10 +847,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     reinterpret_cast<uint4*>(blocks + kZ1 * kBlk)[i] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(blocks + kZ2 * kBlk)[i] = make_uint4(0, 0, 0, 0);
   }
-  for (int i = threadIdx.x; i < kNumWg * 2 * bp; i += kThreads) bins[i] = 0;
+  for (int i = threadIdx.x; i < kNumWg * bp; i += kThreads) bins[i] = 0;
   fence_proxy_async();
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, NT * 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -811,6 +860,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
+      const long long ahead = (long long)(NS + 1) * gridDim.x;
+      for (long long t = blockIdx.x; t < p.n_tiles && t < blockIdx.x + ahead; t += gridDim.x)
+        issue_tile_prefetch<HD, 4>(p, t);
       long long k = 0;
       for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
         const int s = (int)(k % NS);
@@ -818,6 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         if (!mbar_wait(&empty[s], ph ^ 1, abort, p.status, kWaitLimitNs)) break;
         mbar_arrive_expect_tx(&full[s], 4 * tile_bytes + bp * 4);
         issue_tile_loads<HD, 4>(p, t, tiles + s * 4 * tile_bytes, bias + s * bp, &full[s]);
+        if (t + ahead < p.n_tiles) issue_tile_prefetch<HD, 4>(p, t + ahead);
       }
       if (*abort) {
         const long long first = k > NS ? k - NS : 0;
@@ -872,7 +925,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
                                desc_blk_mnmajor(bb, kS0h, kZ1, kS1h, 4)};
       const uint64_t aKl[2] = {desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, 0),
                                desc_blk_mnmajor(bb, kS0l, kZ2, kS1l, 4)};
-      constexpr uint32_t kStepMN = 2048 >> 4, kStepK = 32 >> 4, kStepB = (16 * HD * 2) >> 4;
+      constexpr uint32_t kStepMN = 2048 >> 4, kStepK = 32 >> 4;
+      constexpr uint32_t kStepB = (16 * TileGeom<HD>::kRowBytes) >> 4;
       for (long long k = 0; k < n_local; ++k) {
         const int s = (int)(k % NS), sl = (int)(k % NT);
         if (!mbar_wait(&pds_full[sl], (uint32_t)((k / NT) & 1), abort, p.status, kWaitLimitNs))
@@ -891,14 +945,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk) {  // dQ = dS K
           const uint32_t a = (kk & 3) * kStepK, b = kk * kStepB;
-          umma_ss(d + 64, aQh[kk >> 2] + a, bK + b, idesc_q, kk);
-          umma_ss(d + 64, aQl[kk >> 2] + a, bK + b, idesc_q, 1);
+          umma_ss(d + GC, aQh[kk >> 2] + a, bK + b, idesc_q, kk);
+          umma_ss(d + GC, aQl[kk >> 2] + a, bK + b, idesc_q, 1);
         }
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk) {  // dK = dS^T Q
           const uint32_t a = (kk & 3) * kStepMN, b = kk * kStepB;
-          umma_ss(d + 128, aKh[kk >> 2] + a, bQ + b, idesc_t, kk);
-          umma_ss(d + 128, aKl[kk >> 2] + a, bQ + b, idesc_t, 1);
+          umma_ss(d + 2 * GC, aKh[kk >> 2] + a, bQ + b, idesc_t, kk);
+          umma_ss(d + 2 * GC, aKl[kk >> 2] + a, bQ + b, idesc_t, 1);
         }
         umma_commit(&grad_full[sl]);
         umma_commit(&empty[s]);
@@ -908,17 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         mbar_drain(&drain[1], 0, kTestLimitNs * 100);
       }
     }
-  } else if (warp == kStoreWarp) {
-    if (lane == 0) {   // staged gradients of every tile -> global, then free the block area
-      for (long long k = 0, t = blockIdx.x; k < n_local; ++k, t += gridDim.x) {
-        if (!mbar_wait(staged, (uint32_t)(k & 1), abort, p.status, kWaitLimitNs)) break;
-        if (!*abort) issue_tile_stores3<HD>(p, t, blocks);
-        bulk_wait_read0();
-        mbar_arrive(blk_free);
-      }
-      bulk_wait0();
-    }
-  } else if (warp < kNumWg * 4) {
+  } else if (warp < NWG * 4) {
     const int wg = warp >> 2;
     const int row = threadIdx.x & (kWg - 1);
     const int gw = row / N, lr = row - gw * N;
@@ -927,11 +971,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const uint32_t bb = smem_u32(blocks);
     const uint32_t blk_ph = bb + (gw ? kP1h : kP0h) * kBlk, blk_pl = bb + (gw ? kP1l : kP0l) * kBlk;
     const uint32_t blk_sh = bb + (gw ? kS1h : kS0h) * kBlk, blk_sl = bb + (gw ? kS1l : kS0l) * kBlk;
-    int* bins_hi = bins + wg * 2 * bp;
-    int* bins_lo = bins_hi + bp;
+    int* tb = bins + wg * bp;
+    float* bnd = tbound + wg * 4;
+    __nv_bfloat16* const outs[3] = {(__nv_bfloat16*)p.out2, (__nv_bfloat16*)p.out0,
+                                    (__nv_bfloat16*)p.out1};   // TMEM order: dV, dQ, dK
+    __nv_bfloat16* const outs_h[3] = {(__nv_bfloat16*)p.out2h, (__nv_bfloat16*)p.out0h,
+                                      (__nv_bfloat16*)p.out1h};
     long long k = wg;
     for (long long t = blockIdx.x + wg * (long long)gridDim.x; t < p.n_tiles;
-         t += kNumWg * (long long)gridDim.x, k += kNumWg) {
+         t += NWG * (long long)gridDim.x, k += NWG) {
       const int s = (int)(k % NS), sl = (int)(k % NT);
       const uint32_t phs = (uint32_t)((k / NS) & 1), pht = (uint32_t)((k / NT) & 1);
       const long long group = t / g.heads;
@@ -939,7 +987,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const long long win = group * G + gw;
       const bool plain = WW > 0 && window_plain(g, win);
       const RowInfo me = plain ? plain_row_info<WW>(g, win, lr) : row_info(g, win, lr);
-      uint32_t* ci = colinfo + (wg * 2 + ((k / kNumWg) & 1)) * kRows;
+      uint32_t* ci = colinfo + (wg * 2 + ((k / NWG) & 1)) * kRows;
       ci[row] = key_word(me);
       if (named_sync_or(1 + wg, kWg, *abort)) break;
       if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
@@ -961,8 +1009,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         m = logits_plain<N, (WW > 0 ? WW : 8)>(x, brow + me.bias_base, p.scale_log2);
       else
         m = logits_general<N>(x, brow, cw, me.bias_base, me.label, p.scale_log2);
+      float inv = 0.f;   // max_j P_ij (= 1 / row sum); 0 on pad rows
       if (me.valid) {
-        const float inv = 1.f / exp_sum<N>(x, m);
+        inv = 1.f / exp_sum<N>(x, m);
 #pragma unroll
         for (int j = 0; j < N; ++j) x[j] *= inv;
       } else {
@@ -972,22 +1021,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       // TMEM loads are warp-collective: every lane runs them, valid row or not
       // (x = 0 on invalid rows, so D = 0 and dS = 0 there).
       float dd[4] = {0.f, 0.f, 0.f, 0.f};
+      float mdp = 0.f;
       {
         float dp[N];
         tmem_load_cols<N>(dp_col, dp);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < N; ++j) dd[j & 3] = fmaf(x[j], dp[j], dd[j & 3]);
+        for (int j = 0; j < N; ++j) {
+          dd[j & 3] = fmaf(x[j], dp[j], dd[j & 3]);
+          mdp = fmaxf(mdp, fabsf(dp[j]));
+        }
       }
       const float D = (dd[0] + dd[1]) + (dd[2] + dd[3]);
       __syncwarp();
 #pragma unroll
       for (int c = 0; c < N / 32; ++c) tmem_st32(s_col + 32 * c, x + 32 * c);
+      // |dS_ij| = P_ij |dP_ij - D| <= max_j P_ij * (max_j |dP_ij| + |D|)
+      {
+        const float wb = warp_max(inv * (mdp + fabsf(D)));
+        if (lane == 0) bnd[warp & 3] = wb;
+      }
+      named_sync(3 + wg, kWg);
+      const float tile_bound = fmaxf(fmaxf(bnd[0], bnd[1]), fmaxf(bnd[2], bnd[3]));
+      const bool finite = tile_bound <= 3.0e38f;   // false for NaN and infinity
+      const int E = tile_exponent(finite ? tile_bound : 0.f);
+      const float qs = exp2_int(E);
       tmem_wait_st();
-      // Large |dS| rows take the two-part fixed-point form (rare).
-      float amax = 0.f;
-      int* bqh = bins_hi + me.bias_base;
-      int* bql = bins_lo + me.bias_base;
+      int* bq = tb + me.bias_base;
 #pragma unroll 1
       for (int c = 0; c < N / 32; ++c) {
         float ds[32], pc[32];
@@ -996,29 +1056,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         tmem_ld32(s_col + 32 * c, pc);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          ds[j] = pc[j] * (ds[j] - D);   // dS (0 off the row)
-          amax = fmaxf(amax, fabsf(ds[j]));
-        }
-        if (me.valid) {
-          // bias-gradient bins, fixed point: integer adds commute, so the sum
-          // is exact and independent of the order the lanes land in
-          if (amax < 64.f) {
+        for (int j = 0; j < 32; ++j) ds[j] = pc[j] * (ds[j] - D);   // dS (0 off the row)
+        if (me.valid && finite) {
+          // bias-gradient bins: integers in units of 2^-E; integer adds
+          // commute, so the sums do not depend on the order the lanes land in
+          // (unrolled: a runtime index would put ds in local memory)
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(32 * c + j)
-                                    : (int)(lds_u32(cw + 32 * c + j) & 0xFFFF);
-              red_add_s32(bql - off, round_int_fma(ds[j] * 65536.0f));
-            }
-          } else {   // (unrolled: a runtime index would put ds in local memory)
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(32 * c + j)
-                                    : (int)(lds_u32(cw + 32 * c + j) & 0xFFFF);
-              const float hf = rintf(ds[j]);
-              red_add_s32(bqh - off, __float2int_rn(hf));
-              red_add_s32(bql - off, round_int_fma((ds[j] - hf) * 65536.0f));
-            }
+          for (int j = 0; j < 32; ++j) {
+            const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(32 * c + j)
+                                  : (int)(lds_u32(cw + 32 * c + j) & 0xFFFF);
+            red_add_s32(bq - off, round_to_int(ds[j] * qs));
           }
         }
 #pragma unroll
@@ -1027,10 +1074,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         tmem_st32(dp_col + 32 * c, ds);
       }
       tmem_wait_st();
-      // The operand blocks are free once the previous tile's outputs, staged
-      // there, have been read out by its TMA stores.
+      // The operand blocks are free once the previous tile's gradient
+      // products have completed (grad_full of the other slot; this warpgroup
+      // saw that barrier's phase before, two tiles ago, so the parity names
+      // exactly the phase of tile k-1).
       if (k > 0)
-        mbar_wait(blk_free, (uint32_t)((k - 1) & 1), abort, p.status, kWaitLimitNs);
+        mbar_wait(&grad_full[(k - 1) % NT], (uint32_t)(((k - 1) / NT) & 1), abort, p.status,
+                  kWaitLimitNs);
 #pragma unroll 1
       for (int c = 0; c < N / 32; ++c) {
         float pc[32], ds[32];
@@ -1044,60 +1094,120 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&pds_full[sl]);
-      // Move this tile's bins into the global int64 table.
-      named_sync(3 + wg, kWg);
+      // This tile's bins into the workspace's exact sums.
+      named_sync(5 + wg, kWg);
+      long long* acc = p.dt_acc + (size_t)h * bp * kLimbStride;
       for (int b = row; b < g.bins; b += kWg) {
-        const long long v = ((long long)bins_hi[b] << 16) + bins_lo[b];   // units of 2^-16
-        bins_hi[b] = bins_lo[b] = 0;
-        if (v != 0) red_add_global_s64(p.dt_fixed + h * bp + b, v);
+        const int v = tb[b];
+        tb[b] = 0;
+        if (!finite) flag_nonfinite(acc + (size_t)b * kLimbStride);
+        else if (v != 0) add_fixed(acc + (size_t)b * kLimbStride, v, E);
       }
-      // epilogue: dV, dQ, dK rows from TMEM, staged in the operand-block area
-      // (free of readers once the gradient products are done); warp 11
-      // TMA-stores them to grid order and then frees the area for the next tile.
+      // epilogue: dV, dQ, dK rows from TMEM straight to their grid tokens
       mbar_wait(&grad_full[sl], pht, abort, p.status, kWaitLimitNs);
       tc_fence_after();
+      constexpr int OC = HD > 64 ? 64 : HD;   // columns per TMEM read
 #pragma unroll
       for (int part = 0; part < 3; ++part) {
-        float o[HD];
-        tmem_load_cols<HD>(tmem + lane_base + sl * 256 + part * 64, o);
-        tmem_wait_ld();
-        if (part == 2) {
-          tc_fence_before();
-          mbar_arrive(&t_empty[sl]);
+#pragma unroll
+        for (int c0 = 0; c0 < HD; c0 += OC) {
+          float o[OC];
+          tmem_load_cols<OC>(tmem + lane_base + sl * 256 + part * GC + c0, o);
+          tmem_wait_ld();
+          if (part == 2 && c0 + OC == HD) {
+            tc_fence_before();
+            mbar_arrive(&t_empty[sl]);
+          }
+          if (me.stored && !*abort)   // zero rows beyond the valid extent
+            store_row_bf16<OC>((me.halo ? outs_h[part] : outs[part]) +
+                                   (me.token * g.heads + h) * HD + c0, o, 1.f);
         }
-        stage_row<HD>(bb + bwd_stage(part) + (gw * N + lr) * (HD * 2), o, 1.f);
       }
-      fence_proxy_async();
-      mbar_arrive(staged);   // warp 11 stores them and frees the block area
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, NT * 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
-// Bias table transposed to [heads][bins_pad] and scaled by log2(e); clears
-// the fixed-point bias-gradient table when one is given.
-__global__ void bias_prep_kernel(const float* __restrict__ table, int bins, int heads,
-                                 int bins_pad, float* __restrict__ out,
-                                 long long* __restrict__ dt_fixed) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= heads * bins_pad) return;
-  const int h = i / bins_pad, b = i - h * bins_pad;
-  out[i] = b < bins ? table[b * heads + h] * kLog2e : 0.f;
-  if (dt_fixed) dt_fixed[i] = 0;
+// ================================================================================
+// Layout stage as the kernels above run it, for bit-exact checks
+// ================================================================================
+// ids[token, h, :] holds (token + 1) in its first two 16-bit words and h in
+// the third; all else is zero, so a pad slot (TMA zero fill) reads id 0.
+__global__ void layout_ids_kernel(Geo g, uint16_t* ids) {
+  const long long rows = (long long)g.B * g.H * g.W * g.heads;
+  for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < rows;
+       r += (long long)gridDim.x * blockDim.x) {
+    const long long token = r / g.heads;
+    const int h = (int)(r - token * g.heads);
+    uint16_t* row = ids + r * g.hd;
+    const unsigned long long id = (unsigned long long)token + 1;
+    for (int e = 0; e < g.hd; ++e)
+      row[e] = e == 0 ? (uint16_t)(id & 0xFFFF) : e == 1 ? (uint16_t)(id >> 16) : e == 2 ? (uint16_t)h : 0;
+  }
 }
 
-// dtable[bin][h] = fixed-point sum [h][bin] * 2^-16.
-__global__ void dbias_finish_kernel(const long long* __restrict__ dt_fixed, int bins, int heads,
-                                    int bins_pad, float* __restrict__ dtable) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= bins * heads) return;
-  const int b = i / heads, h = i - b * heads;
-  dtable[i] = (float)((double)dt_fixed[h * bins_pad + b] * kFixInv);
+// One CTA per tile: the producer's TMA boxes of tile t land in shared memory
+// exactly as in the forward and backward; thread r reads tile row r and
+// writes, at the slot that row_slot gives for it, the token it holds (-1 for
+// a zero-filled pad row) and the row's shift-region label. A disagreement
+// with row_info (validity, token) or with the plain-window row info, or a
+// row whose head word is not the tile's head, is written as -2.
+template <int HD>
+__global__ void __launch_bounds__(kRows) layout_map_kernel(const __grid_constant__ FastParams p,
+                                                           int32_t* map, int32_t* labels) {
+  constexpr uint32_t row_bytes = TileGeom<HD>::kRowBytes;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tile = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t full;
+  __shared__ int status;
+  __shared__ int abort_flag;
+  const Geo& g = p.g;
+  const long long t = blockIdx.x;
+  if (threadIdx.x == 0) {
+    mbar_init(&full, 1);
+    status = 0;
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&full, kRows * HD * 2);
+    issue_tile_loads<HD, 1>(p, t, tile, nullptr, &full);
+  }
+  const bool ok = mbar_wait(&full, 0, (volatile int*)&abort_flag, &status, kWaitLimitNs);
+  if (!ok) mbar_drain(&full, 0, kWaitLimitNs);
+  const int G = kRows / g.N;
+  const int r = threadIdx.x, gw = r / g.N, lr = r - gw * g.N;
+  const long long group = t / g.heads;
+  const int h = (int)(t - group * g.heads);
+  const long long win = group * G + gw;
+  if (win >= g.n_win || h != g.heads - 1) return;   // the last head exercises the head coordinate
+  const uint32_t row_addr = smem_u32(tile) + r * row_bytes;
+  const uint32_t swz = HD >= 64 ? ((row_addr >> 7) & 7) : ((row_addr >> 7) & 3);
+  const uint16_t* w = (const uint16_t*)(tile + r * row_bytes + (swz << 4));
+  const unsigned id = (unsigned)w[0] | ((unsigned)w[1] << 16);
+  int b, wy, wx, iy, ix;
+  window_coords(g, win, b, wy, wx);
+  row_slot(g, wy, wx, lr, iy, ix);
+  const RowInfo ri = row_info(g, win, lr);
+  int32_t out = (id == 0 || !ri.valid) ? -1 : (int32_t)(id - 1);
+  if (!ok || (id != 0) != ri.stored || (ri.stored && (long long)(id - 1) != ri.token) ||
+      (id != 0 && w[2] != (uint16_t)h))
+    out = -2;
+  if (g.wh == 8 && g.ww == 8 && window_plain(g, win)) {
+    const RowInfo pi = plain_row_info<8>(g, win, lr);
+    if (pi.token != ri.token || pi.bias_base != ri.bias_base || pi.key_off != ri.key_off ||
+        pi.label != ri.label || !ri.valid)
+      out = -2;
+  }
+  const long long at = win * g.N + iy * g.ww + ix;
+  map[at] = out;
+  if (labels) labels[at] = ri.label;
 }
 
 // ================================================================================
@@ -1124,41 +1234,45 @@ EncodeTiledFn encode_fn() {
 
 int box_len(int kind, int w, int s) { return kind == 0 ? w : (kind == 1 ? w - s : s); }
 
-// The 5-D map [hd, heads, W, H, B] of one tensor with box [hd, 1, bx, by, 1].
-bool encode_map(CUtensorMap* m, const void* base, const Geo& g, int by, int bx) {
+// The 5-D map [hd, heads, W, rows, B] of one tensor with box [hd, 1, bx, by, 1].
+bool encode_map(CUtensorMap* m, const void* base, const Geo& g, int rows, int by, int bx) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[5] = {(cuuint64_t)g.hd, (cuuint64_t)g.heads, (cuuint64_t)g.W,
-                              (cuuint64_t)g.H, (cuuint64_t)g.B};
+                              (cuuint64_t)rows, (cuuint64_t)g.B};
   const cuuint64_t es = 2;
   const cuuint64_t strides[4] = {g.hd * es, (cuuint64_t)g.heads * g.hd * es,
                                  (cuuint64_t)g.W * g.heads * g.hd * es,
-                                 (cuuint64_t)g.H * g.W * g.heads * g.hd * es};
-  const cuuint32_t box[5] = {(cuuint32_t)g.hd, 1, (cuuint32_t)bx, (cuuint32_t)by, 1};
+                                 (cuuint64_t)rows * g.W * g.heads * g.hd * es};
+  // at most 64 channels (128 bytes) per box: head_dim 128 is two boxes
+  const cuuint32_t box[5] = {(cuuint32_t)(g.hd > 64 ? 64 : g.hd), 1, (cuuint32_t)bx,
+                             (cuuint32_t)by, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUtensorMapSwizzle sw =
-      g.hd == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+      g.hd >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The nine box shapes of one tensor into dst[0..8].
-bool encode_map_set(CUtensorMap* dst, const void* base, const Geo& g) {
+// The nine box shapes of one tensor into dst[0..8]. The wrapped row part
+// (ky = 2: source rows 0 .. sh-1) reads `halo` ([B, sh, W, heads, hd]) in a
+// row band, the tensor itself otherwise.
+bool encode_map_set(CUtensorMap* dst, const void* base, const void* halo, const Geo& g) {
   for (int ky = 0; ky < 3; ++ky)
     for (int kx = 0; kx < 3; ++kx) {
       int by = box_len(ky, g.wh, g.sh), bx = box_len(kx, g.ww, g.sw);
       if (by <= 0) by = g.wh;  // shape unused when the axis has no shift
       if (bx <= 0) bx = g.ww;
-      if (!encode_map(&dst[ky * 3 + kx], base, g, by, bx)) return false;
+      const bool from_halo = g.band && ky == 2 && g.sh > 0;
+      if (!encode_map(&dst[ky * 3 + kx], from_halo ? halo : base, g, from_halo ? g.sh : g.H, by,
+                      bx))
+        return false;
     }
   return true;
 }
-bool encode_maps(FastParams& p, int which, const void* base) {
-  return encode_map_set(p.maps[which], base, p.g);
-}
-bool encode_omaps(FastParams& p, int which, const void* base) {
-  return encode_map_set(p.omaps[which], base, p.g);
+bool encode_maps(FastParams& p, int which, const void* base, const void* halo = nullptr) {
+  return encode_map_set(p.maps[which], base, halo, p.g);
 }
 
 int num_sms() {
@@ -1173,17 +1287,23 @@ constexpr size_t kSmemLimit = 227 * 1024;
 
 template <int HD>
 size_t fwd_smem(const Geo& g) {
-  return make_layout<HD, kFwdStages, 3, kFwdPBufs * 32768>(bins_padded(g.bins)).total + 1024;
+  using C = FwdCfg<HD>;
+  return make_layout<HD, C::kStages, 3, C::kPBytes>(bins_padded(g.bins)).total + 1024;
 }
 template <int HD>
 size_t bwd_smem(const Geo& g) {
-  return make_layout<HD, kBwdStages, 4, kNumBlk * kBlk>(bins_padded(g.bins)).total + 1024;
+  return make_layout<HD, BwdCfg<HD>::kStages, 4, kNumBlk * kBlk>(bins_padded(g.bins)).total +
+         1024;
+}
+size_t fwd_smem_any(const Geo& g) {
+  return g.hd == 128 ? fwd_smem<128>(g) : g.hd == 64 ? fwd_smem<64>(g) : fwd_smem<32>(g);
+}
+size_t bwd_smem_any(const Geo& g) {
+  return g.hd == 128 ? bwd_smem<128>(g) : g.hd == 64 ? bwd_smem<64>(g) : bwd_smem<32>(g);
 }
 
 bool smem_ok(const Geo& g) {
-  const size_t f = g.hd == 64 ? fwd_smem<64>(g) : fwd_smem<32>(g);
-  const size_t b = g.hd == 64 ? bwd_smem<64>(g) : bwd_smem<32>(g);
-  return f <= kSmemLimit && b <= kSmemLimit;
+  return fwd_smem_any(g) <= kSmemLimit && bwd_smem_any(g) <= kSmemLimit;
 }
 
 
@@ -1210,20 +1330,11 @@ cudaError_t launch(K kernel, const FastParams& p, size_t smem, cudaStream_t st) 
   return cudaGetLastError();
 }
 
-cudaError_t prep_bias(const Geo& g, const float* table, float* bias_t, long long* dt_fixed,
-                      cudaStream_t st) {
-  const int n = g.heads * bins_padded(g.bins);
-  bias_prep_kernel<<<(n + 255) / 256, 256, 0, st>>>(table, g.bins, g.heads, bins_padded(g.bins),
-                                                    bias_t, dt_fixed);
-  note_launch();
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 bool fast_supported(const Geo& g, int dtype) {
   if (dtype != SWIN_DTYPE_BF16) return false;
-  if (g.hd != 64 && g.hd != 32) return false;
+  if (g.hd != 64 && g.hd != 32 && g.hd != 128) return false;
   if (g.N != 64) return false;
   // Every sub-box must be a whole number of 8-row swizzle atoms.
   const int ylen[3] = {g.wh, g.wh - g.sh, g.sh};
@@ -1238,60 +1349,104 @@ bool fast_supported(const Geo& g, int dtype) {
 }
 
 // Workspace: header (status word), bias table [heads][bins_pad] fp32, and the
-// fixed-point bias gradient [heads][bins_pad] int64.
+// exact bias-gradient sums [heads][bins_pad][kLimbStride] int64.
 size_t fast_workspace(const Geo& g) {
   const int bp = bins_padded(g.bins);
-  return kWsHeader + align256((size_t)g.heads * bp * 4) + align256((size_t)g.heads * bp * 8);
+  return kWsHeader + align256((size_t)g.heads * bp * 4) + align256(dbias_fixed_bytes(g));
 }
 
 cudaError_t fast_forward(const Geo& g, const void* q, const void* k, const void* v,
                          const float* table, void* out, float* lse, void* ws, int flags,
-                         cudaStream_t st) {
+                         cudaStream_t st, const swin_wattn_halo* halo) {
   float* bias_t = (float*)((char*)ws + kWsHeader);
   static thread_local FastParams p;
   fill_common(p, g, bias_t, (int*)ws, flags);
   p.out0 = out;
   p.lse = lse;
-  if (!encode_maps(p, 0, q) || !encode_maps(p, 1, k) || !encode_maps(p, 2, v))
+  if (g.band) {
+    p.out0h = halo->out;
+    p.lse_h = lse ? halo->lse : nullptr;
+  }
+  if (!encode_maps(p, 0, q, g.band ? halo->q : nullptr) ||
+      !encode_maps(p, 1, k, g.band ? halo->k : nullptr) ||
+      !encode_maps(p, 2, v, g.band ? halo->v : nullptr))
     return cudaErrorInvalidValue;
   cudaError_t e = prep_bias(g, table, bias_t, nullptr, st);
   if (e != cudaSuccess) return e;
   const bool w8 = g.wh == 8 && g.ww == 8;
+  const size_t smem = fwd_smem_any(g);
+  if (g.hd == 128)
+    return w8 ? launch(fwd_kernel<128, 8>, p, smem, st) : launch(fwd_kernel<128, 0>, p, smem, st);
   if (g.hd == 64)
-    return w8 ? launch(fwd_kernel<64, 8>, p, fwd_smem<64>(g), st)
-              : launch(fwd_kernel<64, 0>, p, fwd_smem<64>(g), st);
-  return w8 ? launch(fwd_kernel<32, 8>, p, fwd_smem<32>(g), st)
-            : launch(fwd_kernel<32, 0>, p, fwd_smem<32>(g), st);
+    return w8 ? launch(fwd_kernel<64, 8>, p, smem, st) : launch(fwd_kernel<64, 0>, p, smem, st);
+  return w8 ? launch(fwd_kernel<32, 8>, p, smem, st) : launch(fwd_kernel<32, 0>, p, smem, st);
 }
 
 cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void* v,
                           const float* table, const void* dout, void* dq, void* dk, void* dv,
-                          float* dtable, void* ws, int flags, cudaStream_t st) {
+                          float* dtable, void* ws, int flags, cudaStream_t st,
+                          const swin_wattn_halo* halo) {
   float* bias_t = (float*)((char*)ws + kWsHeader);
-  long long* dt_fixed =
-      (long long*)((char*)ws + kWsHeader + align256((size_t)g.heads * bins_padded(g.bins) * 4));
+  long long* dt_acc = (long long*)((char*)ws + dbias_fixed_offset(g));
   static thread_local FastParams p;
   fill_common(p, g, bias_t, (int*)ws, flags);
   p.out0 = dq;
   p.out1 = dk;
   p.out2 = dv;
-  p.dt_fixed = dt_fixed;
-  if (!encode_maps(p, 0, q) || !encode_maps(p, 1, k) || !encode_maps(p, 2, v) ||
-      !encode_maps(p, 3, dout) || !encode_omaps(p, 0, dq) || !encode_omaps(p, 1, dk) ||
-      !encode_omaps(p, 2, dv))
+  p.dt_acc = dt_acc;
+  if (g.band) {
+    p.out0h = halo->dq;
+    p.out1h = halo->dk;
+    p.out2h = halo->dv;
+  }
+  if (!encode_maps(p, 0, q, g.band ? halo->q : nullptr) ||
+      !encode_maps(p, 1, k, g.band ? halo->k : nullptr) ||
+      !encode_maps(p, 2, v, g.band ? halo->v : nullptr) ||
+      !encode_maps(p, 3, dout, g.band ? halo->dout : nullptr))
     return cudaErrorInvalidValue;
-  cudaError_t e = prep_bias(g, table, bias_t, dt_fixed, st);
+  cudaError_t e = prep_bias(g, table, bias_t, dt_acc, st);
   if (e != cudaSuccess) return e;
-  const size_t smem = g.hd == 64 ? bwd_smem<64>(g) : bwd_smem<32>(g);
+  const size_t smem = bwd_smem_any(g);
   const bool w8 = g.wh == 8 && g.ww == 8;
-  if (g.hd == 64)
+  if (g.hd == 128)
+    e = w8 ? launch(bwd_kernel<128, 8>, p, smem, st) : launch(bwd_kernel<128, 0>, p, smem, st);
+  else if (g.hd == 64)
     e = w8 ? launch(bwd_kernel<64, 8>, p, smem, st) : launch(bwd_kernel<64, 0>, p, smem, st);
   else
     e = w8 ? launch(bwd_kernel<32, 8>, p, smem, st) : launch(bwd_kernel<32, 0>, p, smem, st);
   if (e != cudaSuccess) return e;
-  const int n = g.bins * g.heads;
-  dbias_finish_kernel<<<(n + 255) / 256, 256, 0, st>>>(dt_fixed, g.bins, g.heads,
-                                                       bins_padded(g.bins), dtable);
+  if (flags & SWIN_FLAG_DBIAS_SUMS) return cudaSuccess;   // the caller finishes the sums
+  return finish_dbias(g, dt_acc, dtable, st);
+}
+
+cudaError_t fast_layout_map(const Geo& g, void* ids, int32_t* map, int32_t* labels,
+                            cudaStream_t st) {
+  static thread_local FastParams p;
+  fill_common(p, g, nullptr, nullptr, 0);
+  if (!encode_maps(p, 0, ids)) return cudaErrorInvalidValue;
+  const long long rows = (long long)g.B * g.H * g.W * g.heads;
+  const int blocks = (int)((rows + 255) / 256 < 4096 ? (rows + 255) / 256 : 4096);
+  layout_ids_kernel<<<blocks, 256, 0, st>>>(g, (uint16_t*)ids);
+  note_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = (size_t)kRows * g.hd * 2 + 1024;
+  if (g.hd == 128) {
+    e = cudaFuncSetAttribute(layout_map_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    layout_map_kernel<128><<<(unsigned)p.n_tiles, kRows, smem, st>>>(p, map, labels);
+  } else if (g.hd == 64) {
+    e = cudaFuncSetAttribute(layout_map_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    layout_map_kernel<64><<<(unsigned)p.n_tiles, kRows, smem, st>>>(p, map, labels);
+  } else {
+    e = cudaFuncSetAttribute(layout_map_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    layout_map_kernel<32><<<(unsigned)p.n_tiles, kRows, smem, st>>>(p, map, labels);
+  }
   note_launch();
   return cudaGetLastError();
 }

@@ -26,7 +26,9 @@ __device__ __forceinline__ void st(float* p, float x) { *p = x; }
 __device__ __forceinline__ void st(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
 
 // Per-window slot table staged in shared memory: element offset of the token's
-// row for head h (or -1 for a pad slot), region label, slot coordinates.
+// row for head h (or -1 for a slot outside the stored grid), region label (a
+// distinct negative value -1 - slot for a token beyond the valid extent, so it
+// pairs with nothing), slot coordinates.
 struct SlotTab {
   long long* off;
   int* label;
@@ -42,13 +44,18 @@ __device__ SlotTab stage_slots(const Geo& g, long long win, int h, unsigned char
   t.ix = t.iy + g.N;
   for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
     const SlotInfo s = slot_info(g, win, i);
-    t.off[i] = s.valid ? (token_of(g, s) * g.heads + h) * g.hd : -1;
-    t.label[i] = s.label;
+    t.off[i] = s.stored ? (token_of(g, s) * g.heads + h) * g.hd : -1;
+    t.label[i] = s.valid ? s.label : -1 - i;
     t.iy[i] = s.iy;
     t.ix[i] = s.ix;
   }
   __syncthreads();
   return t;
+}
+
+// Key j is allowed for query i: both real tokens in the same shift region.
+__device__ __forceinline__ bool allowed(const SlotTab& t, int i, int j) {
+  return t.label[i] >= 0 && t.label[i] == t.label[j];
 }
 
 __host__ size_t slot_smem(const Geo& g) { return (size_t)g.N * (sizeof(long long) + 3 * sizeof(int)); }
@@ -83,10 +90,15 @@ __global__ void generic_fwd_kernel(Geo g, const T* __restrict__ q, const T* __re
   float acc[kMaxHd];
   for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
     if (t.off[i] < 0) continue;
+    if (t.label[i] < 0) {   // stored token beyond the valid extent: zeros
+      for (int e = 0; e < g.hd; ++e) st(out + t.off[i] + e, 0.f);
+      if (lse) lse[t.off[i] / g.hd] = 0.f;
+      continue;
+    }
     const T* qi = q + t.off[i];
     float m = -INFINITY;
     for (int j = 0; j < g.N; ++j) {
-      if (t.off[j] < 0 || t.label[j] != t.label[i]) continue;
+      if (!allowed(t, i, j)) continue;
       const float a = scale * dot(qi, k + t.off[j], g.hd) +
                       table[rel_index(g, t.iy[i], t.ix[i], t.iy[j], t.ix[j]) * g.heads + h];
       m = fmaxf(m, a);
@@ -94,7 +106,7 @@ __global__ void generic_fwd_kernel(Geo g, const T* __restrict__ q, const T* __re
     for (int e = 0; e < g.hd; ++e) acc[e] = 0.f;
     float l = 0.f;
     for (int j = 0; j < g.N; ++j) {
-      if (t.off[j] < 0 || t.label[j] != t.label[i]) continue;
+      if (!allowed(t, i, j)) continue;
       const float a = scale * dot(qi, k + t.off[j], g.hd) +
                       table[rel_index(g, t.iy[i], t.ix[i], t.iy[j], t.ix[j]) * g.heads + h];
       const float p = expf(a - m);
@@ -115,13 +127,13 @@ __device__ void row_stats(const Geo& g, const SlotTab& t, int i, int h, const T*
   const T* qi = q + t.off[i];
   m = -INFINITY;
   for (int j = 0; j < g.N; ++j) {
-    if (t.off[j] < 0 || t.label[j] != t.label[i]) continue;
+    if (!allowed(t, i, j)) continue;
     m = fmaxf(m, scale * dot(qi, k + t.off[j], g.hd) +
                      table[rel_index(g, t.iy[i], t.ix[i], t.iy[j], t.ix[j]) * g.heads + h]);
   }
   l = 0.f;
   for (int j = 0; j < g.N; ++j) {
-    if (t.off[j] < 0 || t.label[j] != t.label[i]) continue;
+    if (!allowed(t, i, j)) continue;
     l += expf(scale * dot(qi, k + t.off[j], g.hd) +
               table[rel_index(g, t.iy[i], t.ix[i], t.iy[j], t.ix[j]) * g.heads + h] - m);
   }
@@ -142,8 +154,10 @@ __global__ void generic_bwd_rows_kernel(Geo g, const T* __restrict__ q, const T*
   float acc[kMaxHd];
   for (int i = threadIdx.x; i < g.N; i += blockDim.x) {
     float* st3 = stats + ((win * g.heads + h) * g.N + i) * 3;
-    if (t.off[i] < 0) {
+    if (t.off[i] < 0 || t.label[i] < 0) {
       st3[0] = 0.f; st3[1] = 1.f; st3[2] = 0.f;
+      if (t.off[i] >= 0)
+        for (int e = 0; e < g.hd; ++e) st(dq + t.off[i] + e, 0.f);
       continue;
     }
     float m, l;
@@ -152,7 +166,7 @@ __global__ void generic_bwd_rows_kernel(Geo g, const T* __restrict__ q, const T*
     const T* doi = dout + t.off[i];
     float D = 0.f;
     for (int j = 0; j < g.N; ++j) {
-      if (t.off[j] < 0 || t.label[j] != t.label[i]) continue;
+      if (!allowed(t, i, j)) continue;
       const float p = expf(scale * dot(qi, k + t.off[j], g.hd) +
                            table[rel_index(g, t.iy[i], t.ix[i], t.iy[j], t.ix[j]) * g.heads + h] -
                            m) / l;
@@ -160,7 +174,7 @@ __global__ void generic_bwd_rows_kernel(Geo g, const T* __restrict__ q, const T*
     }
     for (int e = 0; e < g.hd; ++e) acc[e] = 0.f;
     for (int j = 0; j < g.N; ++j) {
-      if (t.off[j] < 0 || t.label[j] != t.label[i]) continue;
+      if (!allowed(t, i, j)) continue;
       const float p = expf(scale * dot(qi, k + t.off[j], g.hd) +
                            table[rel_index(g, t.iy[i], t.ix[i], t.iy[j], t.ix[j]) * g.heads + h] -
                            m) / l;
@@ -188,10 +202,17 @@ __global__ void generic_bwd_cols_kernel(Geo g, const T* __restrict__ q, const T*
   for (int j = threadIdx.x; j < g.N; j += blockDim.x) {
     if (t.off[j] < 0) continue;
     for (int e = 0; e < g.hd; ++e) ak[e] = av[e] = 0.f;
+    if (t.label[j] < 0) {   // stored token beyond the valid extent: zeros
+      for (int e = 0; e < g.hd; ++e) {
+        st(dk + t.off[j] + e, 0.f);
+        st(dv + t.off[j] + e, 0.f);
+      }
+      continue;
+    }
     const T* kj = k + t.off[j];
     const T* vj = v + t.off[j];
     for (int i = 0; i < g.N; ++i) {
-      if (t.off[i] < 0 || t.label[i] != t.label[j]) continue;
+      if (!allowed(t, j, i)) continue;
       const float* st3 = stats + ((win * g.heads + h) * g.N + i) * 3;
       const T* qi = q + t.off[i];
       const T* doi = dout + t.off[i];
@@ -234,7 +255,7 @@ __global__ void generic_dbias_partial_kernel(Geo g, const T* __restrict__ q,
         const int jy = t.iy[i] - dy, jx = t.ix[i] - dx;
         if (jy < 0 || jy >= g.wh || jx < 0 || jx >= g.ww) continue;
         const int j = jy * g.ww + jx;
-        if (t.off[i] < 0 || t.off[j] < 0 || t.label[i] != t.label[j]) continue;
+        if (!allowed(t, i, j)) continue;
         const float* st3 = stats + ((win * g.heads + h) * g.N + i) * 3;
         const float p = expf(scale * dot(q + t.off[i], k + t.off[j], g.hd) + table[bin * g.heads + h] -
                              st3[0]) / st3[1];

@@ -16,15 +16,24 @@ namespace swin {
 
 struct Geo {
   int B, H, W, wh, ww, sh, sw, heads, hd;
+  int Hv, Wv;               // valid extent: tokens at y >= Hv or x >= Wv are padding
   int Hp, Wp, nWy, nWx, N;  // padded grid, windows per axis, tokens per window
   long long n_win;          // B * nWy * nWx
   int bins;                 // (2 wh - 1) (2 ww - 1)
+  // Row band of a larger grid (tcgen05 kernels only): the rows the shift
+  // wraps to (source rows 0 .. sh-1 of the last window row) live in a
+  // separate halo tensor [B, sh, W, heads, hd] (the next band's first rows),
+  // and their outputs go to a halo output tensor of that shape.
+  int band;
+  int seam_h;               // shift of the row shift-region split (0: none; sh otherwise)
 };
 
 inline Geo make_geo(const swin_wattn_desc& d) {
   Geo g;
   g.B = d.B; g.H = d.H; g.W = d.W; g.wh = d.win_h; g.ww = d.win_w;
   g.sh = d.shift_h; g.sw = d.shift_w; g.heads = d.heads; g.hd = d.head_dim;
+  g.Hv = d.valid_h > 0 ? d.valid_h : d.H;
+  g.Wv = d.valid_w > 0 ? d.valid_w : d.W;
   g.Hp = (d.H + d.win_h - 1) / d.win_h * d.win_h;
   g.Wp = (d.W + d.win_w - 1) / d.win_w * d.win_w;
   g.nWy = g.Hp / d.win_h;
@@ -32,6 +41,8 @@ inline Geo make_geo(const swin_wattn_desc& d) {
   g.N = d.win_h * d.win_w;
   g.n_win = (long long)d.B * g.nWy * g.nWx;
   g.bins = (2 * d.win_h - 1) * (2 * d.win_w - 1);
+  g.band = 0;
+  g.seam_h = d.shift_h;
   return g;
 }
 
@@ -46,7 +57,8 @@ struct SlotInfo {
   int b, y, x;     // source grid position (y < Hp, x < Wp)
   int iy, ix;      // slot coordinates inside the window
   int label;       // 3 * row region + column region
-  bool valid;      // y < H and x < W
+  bool valid;      // a real token: y < Hv and x < Wv
+  bool stored;     // in the tensor: y < H and x < W (outputs are written)
 };
 
 // Window `win` (flattened over b, wy, wx) and slot -> source token. Rolled
@@ -63,12 +75,13 @@ __host__ __device__ inline SlotInfo slot_info(const Geo& g, long long win, int s
   const int yr = wy * g.wh + s.iy, xr = wx * g.ww + s.ix;
   s.y = (yr + g.sh) % g.Hp;
   s.x = (xr + g.sw) % g.Wp;
-  s.valid = s.y < g.H && s.x < g.W;
-  s.label = 3 * region_1d(yr, g.Hp, g.wh, g.sh) + region_1d(xr, g.Wp, g.ww, g.sw);
+  s.stored = s.y < g.H && s.x < g.W;
+  s.valid = s.y < g.Hv && s.x < g.Wv;
+  s.label = 3 * region_1d(yr, g.Hp, g.wh, g.seam_h) + region_1d(xr, g.Wp, g.ww, g.sw);
   return s;
 }
 
-// Linear token index (b*H + y)*W + x of a valid slot.
+// Linear token index (b*H + y)*W + x of a stored slot.
 __host__ __device__ inline long long token_of(const Geo& g, const SlotInfo& s) {
   return ((long long)s.b * g.H + s.y) * g.W + s.x;
 }

@@ -55,11 +55,12 @@ extern "C" int swin_wattn_bwd_noalloc(const swin_wattn_desc* desc, const void* q
                                       const void* v, const float* bias_table, const void* dout,
                                       void* dq, void* dk, void* dv, float* dbias_table,
                                       void* stream) {
-  const int path = swin_wattn_path(desc);   // validates the description
-  if (path < 0) return path;
-  if (path != 1) return SWIN_ERR_UNSUPPORTED;   // only the tcgen05 kernels run here
+  // Every argument is checked before anything is queued on the stream.
+  int rc = check_bwd_args(desc, q, k, v, bias_table, dout, dq, dk, dv, dbias_table);
+  if (rc) return rc;
+  if (swin_wattn_path(desc) != 1) return SWIN_ERR_UNSUPPORTED;   // only the tcgen05 kernels run here
   size_t need = 0;
-  int rc = swin_wattn_workspace_size(desc, &need);
+  rc = swin_wattn_workspace_size(desc, &need);
   if (rc) return rc;
   if (need > (size_t)SWIN_NOALLOC_SCRATCH_BYTES) return SWIN_ERR_WORKSPACE;
   void* scratch = nullptr;

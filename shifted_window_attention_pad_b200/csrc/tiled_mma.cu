@@ -31,15 +31,18 @@
 //     split into bf16 high and low parts so the products keep about 16 bits;
 //     dS^T goes to shared memory and, after a CTA barrier, the warps compute
 //     dQ = dS K for the chunk's 64 queries.
-//   The bias-table gradient is summed per tile in fixed point (int32 shared
-//   bins, units of 2^-16) and folded into the workspace's int64 table, so the
-//   result does not depend on the order of the additions.
+//   The bias-table gradient is summed exactly in integers (dbias_fixed.cuh):
+//   pass 1 also gives a bound on |dS| over the tile, which sets the unit 2^-E
+//   of the tile's int32 shared bins; the bins are then folded into the
+//   workspace's wide integer sums. The result does not depend on the order of
+//   the additions, and its relative error not on the scale of the gradients.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
 
 #include "../../include/swin_wattn.h"
+#include "dbias_fixed.cuh"
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -50,7 +53,6 @@ using namespace ptx;
 
 constexpr float kLog2eT = 1.4426950408889634f;
 constexpr float kLn2T = 0.6931471805599453f;
-constexpr double kFixInvT = 1.52587890625e-05;  // 2^-16
 constexpr size_t kSmemLimitT = 227 * 1024;
 
 struct TiledParams {
@@ -68,7 +70,7 @@ struct TiledParams {
   uint16_t* dq;
   uint16_t* dk;
   uint16_t* dv;
-  long long* dt_fixed;  // [heads][bins_pad], units of 2^-16
+  long long* dt_acc;    // exact bias-gradient sums [heads][bins_pad][kLimbStride]
 };
 
 // ---- shared-memory layout of one tile --------------------------------------
@@ -76,7 +78,7 @@ struct TiledParams {
 // backward: the dS^T buffer of one 64-query chunk, high and low parts, as
 // [NP keys][64 queries] bf16; per-slot source offsets and info words; row
 // statistics (backward: log-sum-exp and D per query); the head's bias row;
-// fixed-point bins (backward).
+// backward: int32 bias-gradient bins and the tile's bound on |dS|.
 struct TLay {
   uint32_t q, k, v, dout, dsh, dsl, off, info, stat, bias, bins, total;
 };
@@ -107,7 +109,7 @@ __host__ __device__ inline TLay tlayout(bool bwd, int bins_pad) {
   L.bias = o;
   o += (uint32_t)bins_pad * 4;
   L.bins = o;
-  o += bwd ? (uint32_t)bins_pad * 8 : 0;
+  o += bwd ? (uint32_t)bins_pad * 4 + 16 : 0;
   L.total = o;
   return L;
 }
@@ -166,11 +168,6 @@ __device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint3
   lo = pack_bf16(x - __uint_as_float(a), y - __uint_as_float(b));
 }
 
-// x (|x| < 2^22) rounded to the nearest integer with the float adder.
-__device__ __forceinline__ int round_int_add(float x) {
-  return __float_as_int(x + 12582912.0f) - 0x4B400000;
-}
-
 // Slot info word: bits 0-15 the slot's position iy * (2 ww - 1) + ix, bits
 // 16-19 its label as a key (15: pad or past the window, matches nothing), bits
 // 20-23 its label as a query (14: no output). Allowed pair <=> key label ==
@@ -207,12 +204,11 @@ __device__ __forceinline__ bool tile_setup(const TiledParams& p, uint8_t* smem, 
       const SlotInfo s = slot_info(g, win, tid);
       const uint32_t pos = (uint32_t)(s.iy * (2 * g.ww - 1) + s.ix);
       plain = s.valid && s.label == slot_info(g, win, 0).label;
-      if (s.valid) {
-        w = pos | ((uint32_t)s.label << 16) | ((uint32_t)s.label << 20);
-        o = (token_of(g, s) * g.heads + h) * HD;
-      } else {
-        w = pos | (15u << 16) | (14u << 20);
-      }
+      // a stored token beyond the valid extent keeps its address (its
+      // outputs are written, as zeros) but matches no query and no key
+      w = s.valid ? pos | ((uint32_t)s.label << 16) | ((uint32_t)s.label << 20)
+                  : pos | (15u << 16) | (14u << 20);
+      if (s.stored) o = (token_of(g, s) * g.heads + h) * HD;
     }
     info[tid] = w;
     off[tid] = o;
@@ -220,8 +216,8 @@ __device__ __forceinline__ bool tile_setup(const TiledParams& p, uint8_t* smem, 
   float* bias = (float*)(smem + L.bias);
   for (int b = tid; b < p.bins_pad; b += blockDim.x) bias[b] = p.bias_t[(size_t)h * p.bins_pad + b];
   if (BWD) {
-    int* bins = (int*)(smem + L.bins);
-    for (int b = tid; b < 2 * p.bins_pad; b += blockDim.x) bins[b] = 0;
+    int* bins = (int*)(smem + L.bins);   // bins, then the tile's |dS| bound (float bits)
+    for (int b = tid; b <= p.bins_pad; b += blockDim.x) bins[b] = 0;
   }
   plain = __syncthreads_and(plain);
   constexpr int CH = HD / 8;
@@ -354,8 +350,8 @@ __device__ __forceinline__ void fwd_tile(const TiledParams& p, uint8_t* smem, co
     if (o1 >= 0) *(uint32_t*)(p.out + o1 + col) = pack_bf16(o[n][2] * i1, o[n][3] * i1);
   }
   if (p.lse && t4 == 0) {
-    if (o0 >= 0) p.lse[o0 / HD] = (m0 + log2f(l0)) * kLn2T;
-    if (o1 >= 0) p.lse[o1 / HD] = (m1 + log2f(l1)) * kLn2T;
+    if (o0 >= 0) p.lse[o0 / HD] = l0 > 0.f ? (m0 + log2f(l0)) * kLn2T : 0.f;
+    if (o1 >= 0) p.lse[o1 / HD] = l1 > 0.f ? (m1 + log2f(l1)) * kLn2T : 0.f;
   }
 }
 
@@ -376,20 +372,13 @@ __global__ void __launch_bounds__(NP * 2 / PARTS, 256 * PARTS / NP)
 }
 
 // ---- backward -----------------------------------------------------------------
-// Adds dS (one value of the tile) to the fixed-point bins of bias index b:
-// |dS| < 64 goes whole into the low int32 part; larger values (|dS| < 2^22)
-// are split into an integer high part and a low remainder. A tile adds at
-// most NP <= 256 terms to one bin, so neither part can overflow.
+// Adds dS (one value of the tile) to the int32 bin of bias index b, in units
+// of 2^-E (qs = 2^E): every term is below 2^22 units and a bin takes at most
+// NP <= 256 terms, so the sum cannot overflow.
 template <bool PLAIN>
-__device__ __forceinline__ void bin_add(int* bins_hi, int* bins_lo, int b, float ds) {
+__device__ __forceinline__ void bin_add(int* bins, int b, float ds, float qs) {
   if (!PLAIN && ds == 0.f) return;   // masked pairs of seam and pad windows
-  if (fabsf(ds) < 64.f) {
-    red_add_s32(bins_lo + b, round_int_add(ds * 65536.0f));
-  } else {
-    const float hf = rintf(ds);
-    red_add_s32(bins_hi + b, __float2int_rn(hf));
-    red_add_s32(bins_lo + b, round_int_add((ds - hf) * 65536.0f));
-  }
+  red_add_s32(bins + b, round_to_int(ds * qs));
 }
 
 template <int HD, int NP, int QS, bool PLAIN>
@@ -408,8 +397,8 @@ __device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, co
   const float* bias = (const float*)(smem + L.bias);
   float* st_lse = (float*)(smem + L.stat);   // log2 of the row sum of 2^logit
   float* st_d = st_lse + NP;                 // D = sum_j P_ij dP_ij
-  int* bins_hi = (int*)(smem + L.bins);
-  int* bins_lo = bins_hi + p.bins_pad;
+  int* bins = (int*)(smem + L.bins);
+  unsigned* bound_bits = (unsigned*)(bins + p.bins_pad);   // tile max of the row bounds
   const int C0 = (g.wh - 1) * (2 * g.ww - 1) + g.ww - 1;
   const float sc = p.scale_log2;
 
@@ -426,6 +415,7 @@ __device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, co
     const int qp0 = (int)(qw0 & 0xFFFFu) + C0, qp1 = (int)(qw1 & 0xFFFFu) + C0;
     const uint32_t ql0 = (qw0 >> 20) & 15u, ql1 = (qw1 >> 20) & 15u;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, d0 = 0.f, d1 = 0.f;
+    float x0 = 0.f, x1 = 0.f;   // max |dP| of the two rows
 #pragma unroll 1
     for (int kc = 0; kc < NP / 64; ++kc) {
       float s[8][4], dp[8][4];
@@ -456,6 +446,8 @@ __device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, co
         s[n][3] = logit<PLAIN>(s[n][3], kw.y, qp1, ql1, bias, sc);
         c0 = fmaxf(c0, fmaxf(s[n][0], s[n][1]));
         c1 = fmaxf(c1, fmaxf(s[n][2], s[n][3]));
+        x0 = fmaxf(x0, fmaxf(fabsf(dp[n][0]), fabsf(dp[n][1])));
+        x1 = fmaxf(x1, fmaxf(fabsf(dp[n][2]), fabsf(dp[n][3])));
       }
       c0 = fmaxf(c0, __shfl_xor_sync(0xffffffffu, c0, 1));
       c0 = fmaxf(c0, __shfl_xor_sync(0xffffffffu, c0, 2));
@@ -487,8 +479,15 @@ __device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, co
       l1 += __shfl_xor_sync(0xffffffffu, l1, x);
       d0 += __shfl_xor_sync(0xffffffffu, d0, x);
       d1 += __shfl_xor_sync(0xffffffffu, d1, x);
+      x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, x));
+      x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, x));
     }
     if (t4 == 0) {
+      // |dS_ij| = P_ij |dP_ij - D_i| <= (1 / l_i) (max_j |dP_ij| + |D_i|);
+      // non-negative floats order like their bit patterns (NaN above all)
+      const float b0 = l0 > 0.f ? (x0 + fabsf(d0 / l0)) / l0 : 0.f;
+      const float b1 = l1 > 0.f ? (x1 + fabsf(d1 / l1)) / l1 : 0.f;
+      atomicMax(bound_bits, __float_as_uint(fmaxf(b0, b1)));
       // P = 2^(logit - lse); rows without an allowed key (pad queries) get
       // lse = +inf, hence P = 0, in pass 2
       st_lse[r0 + g8] = l0 > 0.f ? m0 + log2f(l0) : INFINITY;
@@ -498,6 +497,10 @@ __device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, co
     }
   }
   __syncthreads();
+  const float tile_bound = __uint_as_float(*bound_bits);
+  const bool finite = tile_bound <= 3.0e38f;   // false for NaN and infinity
+  const int E = tile_exponent(finite ? tile_bound : 0.f);
+  const float qs = exp2_int(E);
 
   // ---- pass 2: key-major dV, dK; dS^T to shared; dQ per 64-query chunk ----
   const int kb = warp * 16;
@@ -558,7 +561,7 @@ __device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, co
           const float x = ok ? fmaf(st[n][e], sc, bias[bidx]) : -INFINITY;
           const float pe = ex2(x - lse);
           const float ds = pe * (dpt[n][e] - D);
-          if (ok) bin_add<PLAIN>(bins_hi, bins_lo, bidx, ds);
+          if (ok && finite) bin_add<PLAIN>(bins, bidx, ds, qs);
           st[n][e] = pe;
           dpt[n][e] = ds * p.dscale;
         }
@@ -679,11 +682,13 @@ __device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, co
       }
     }
   }
-  // the tile's bins into the global int64 table (the last loop barrier made
-  // every shared add visible)
+  // the tile's bins into the workspace's exact sums (the last loop barrier
+  // made every shared add visible)
+  long long* acc = p.dt_acc + (size_t)h * p.bins_pad * kLimbStride;
   for (int b = threadIdx.x; b < g.bins; b += blockDim.x) {
-    const long long v = ((long long)bins_hi[b] << 16) + bins_lo[b];
-    if (v != 0) red_add_global_s64(p.dt_fixed + (size_t)h * p.bins_pad + b, v);
+    const int v = bins[b];
+    if (!finite) flag_nonfinite(acc + (size_t)b * kLimbStride);
+    else if (v != 0) add_fixed(acc + (size_t)b * kLimbStride, v, E);
   }
 }
 
@@ -698,27 +703,6 @@ __global__ void __launch_bounds__(NP * 2, 256 / NP)
     bwd_tile<HD, NP, QS, true>(p, smem, L, h);
   else
     bwd_tile<HD, NP, QS, false>(p, smem, L, h);
-}
-
-// Bias table transposed to [heads][bins_pad] and scaled by log2(e); clears the
-// fixed-point bias-gradient table when one is given.
-__global__ void tiled_bias_prep_kernel(const float* __restrict__ table, int bins, int heads,
-                                       int bins_pad, float* __restrict__ out,
-                                       long long* __restrict__ dt_fixed) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= heads * bins_pad) return;
-  const int h = i / bins_pad, b = i - h * bins_pad;
-  out[i] = b < bins ? table[(size_t)b * heads + h] * kLog2eT : 0.f;
-  if (dt_fixed) dt_fixed[i] = 0;
-}
-
-// dtable[bin][h] = fixed-point sum [h][bin] * 2^-16.
-__global__ void tiled_dbias_finish_kernel(const long long* __restrict__ dt_fixed, int bins,
-                                          int heads, int bins_pad, float* __restrict__ dtable) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= bins * heads) return;
-  const int b = i / heads, h = i - b * heads;
-  dtable[i] = (float)((double)dt_fixed[(size_t)h * bins_pad + b] * kFixInvT);
 }
 
 int slots_for(int N) { return N <= 64 ? 64 : (N <= 128 ? 128 : 256); }
@@ -761,15 +745,6 @@ cudaError_t launch_tiled(K kernel, const TiledParams& p, int threads, size_t sme
   return cudaGetLastError();
 }
 
-cudaError_t prep(const Geo& g, const float* table, float* bias_t, long long* dt_fixed,
-                 cudaStream_t st) {
-  const int n = g.heads * bins_padded(g.bins);
-  tiled_bias_prep_kernel<<<(n + 255) / 256, 256, 0, st>>>(table, g.bins, g.heads,
-                                                          bins_padded(g.bins), bias_t, dt_fixed);
-  note_launch();
-  return cudaGetLastError();
-}
-
 }  // namespace
 
 bool tiled_supported(const Geo& g, int dtype) {
@@ -781,10 +756,10 @@ bool tiled_supported(const Geo& g, int dtype) {
 }
 
 // Workspace: header (status word), bias table [heads][bins_pad] fp32, and the
-// fixed-point bias gradient [heads][bins_pad] int64.
+// exact bias-gradient sums [heads][bins_pad][kLimbStride] int64.
 size_t tiled_workspace(const Geo& g) {
   const int bp = bins_padded(g.bins);
-  return kWsHeader + align256((size_t)g.heads * bp * 4) + align256((size_t)g.heads * bp * 8);
+  return kWsHeader + align256((size_t)g.heads * bp * 4) + align256(dbias_fixed_bytes(g));
 }
 
 cudaError_t tiled_forward(const Geo& g, const void* q, const void* k, const void* v,
@@ -797,7 +772,7 @@ cudaError_t tiled_forward(const Geo& g, const void* q, const void* k, const void
   p.v = (const uint16_t*)v;
   p.out = (uint16_t*)out;
   p.lse = lse;
-  cudaError_t e = prep(g, table, bias_t, nullptr, st);
+  cudaError_t e = prep_bias(g, table, bias_t, nullptr, st);
   if (e != cudaSuccess) return e;
   const int NP = slots_for(g.N);
   const size_t smem = tiled_smem_any(g, false);
@@ -813,10 +788,9 @@ cudaError_t tiled_forward(const Geo& g, const void* q, const void* k, const void
 
 cudaError_t tiled_backward(const Geo& g, const void* q, const void* k, const void* v,
                            const float* table, const void* dout, void* dq, void* dk, void* dv,
-                           float* dtable, void* ws, cudaStream_t st) {
+                           float* dtable, void* ws, int flags, cudaStream_t st) {
   float* bias_t = (float*)((char*)ws + kWsHeader);
-  long long* dt_fixed =
-      (long long*)((char*)ws + kWsHeader + align256((size_t)g.heads * bins_padded(g.bins) * 4));
+  long long* dt_acc = (long long*)((char*)ws + dbias_fixed_offset(g));
   TiledParams p;
   fill_params(p, g, bias_t);
   p.q = (const uint16_t*)q;
@@ -826,8 +800,8 @@ cudaError_t tiled_backward(const Geo& g, const void* q, const void* k, const voi
   p.dq = (uint16_t*)dq;
   p.dk = (uint16_t*)dk;
   p.dv = (uint16_t*)dv;
-  p.dt_fixed = dt_fixed;
-  cudaError_t e = prep(g, table, bias_t, dt_fixed, st);
+  p.dt_acc = dt_acc;
+  cudaError_t e = prep_bias(g, table, bias_t, dt_acc, st);
   if (e != cudaSuccess) return e;
   const int NP = slots_for(g.N);
   const size_t smem = tiled_smem_any(g, true);
@@ -841,11 +815,8 @@ cudaError_t tiled_backward(const Geo& g, const void* q, const void* k, const voi
     else e = launch_tiled(tiled_bwd_kernel<32, 256, kQS>, p, 512, smem, st);
   }
   if (e != cudaSuccess) return e;
-  const int n = g.bins * g.heads;
-  tiled_dbias_finish_kernel<<<(n + 255) / 256, 256, 0, st>>>(dt_fixed, g.bins, g.heads,
-                                                             bins_padded(g.bins), dtable);
-  note_launch();
-  return cudaGetLastError();
+  if (flags & SWIN_FLAG_DBIAS_SUMS) return cudaSuccess;   // the caller finishes the sums
+  return finish_dbias(g, dt_acc, dtable, st);
 }
 
 }  // namespace swin

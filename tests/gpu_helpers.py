@@ -20,7 +20,7 @@ BF16_TOL = 2e-2
 
 def oracle_shape(desc):
     return oracle.Shape(desc.B, desc.H, desc.W, desc.win_h, desc.win_w, desc.shift_h,
-                        desc.shift_w, desc.heads, desc.head_dim)
+                        desc.shift_w, desc.heads, desc.head_dim, desc.valid_h, desc.valid_w)
 
 
 def run_gpu(desc, inp, want_lse=True, backward=True):
@@ -84,9 +84,23 @@ def err_f32(gpu, ref):
 FP32_OUTPUTS = ("lse", "dT")
 
 
-def compare(gpu, ref, dtype, names=("o", "lse", "dq", "dk", "dv", "dT")):
+# Every comparison of a run, for the table the test session prints at its end
+# (the margin of each output against its bar, per case).
+RECORDED = []
+
+
+def compare(gpu, ref, dtype, names=("o", "lse", "dq", "dk", "dv", "dT"), label=None):
     """Returns {name: error} against the workload's bar. lse and dT are stored
     in fp32 on every path, so no storage rounding is discounted for them."""
+    errs = _compare(gpu, ref, dtype, names)
+    if label is None:
+        import os
+        label = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0].split("::")[-1]
+    RECORDED.append((label, dtype, errs))
+    return errs
+
+
+def _compare(gpu, ref, dtype, names):
     errs = {}
     for n in names:
         if n in gpu and gpu[n] is not None and n in ref and ref[n] is not None:

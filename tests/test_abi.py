@@ -59,7 +59,8 @@ def test_path_selection_on_the_workloads(L):
 
 @pytest.mark.parametrize("win,hd,want", [((7, 7), 64, 2), ((8, 12), 32, 2), ((16, 16), 64, 2),
                                          ((12, 12), 32, 2), ((16, 17), 64, 0), ((32, 32), 64, 0),
-                                         ((16, 16), 128, 0), ((8, 8), 64, 1)])
+                                         ((16, 16), 128, 0), ((8, 8), 64, 1), ((8, 8), 128, 1),
+                                         ((4, 16), 128, 1), ((7, 7), 128, 0)])
 def test_tiled_path_covers_windows_up_to_256_tokens(L, win, hd, want):
     d = sb.make_desc(1, 40, 52, win, (win[0] // 2, win[1] // 2), 2, hd, "bf16")
     assert sb.swin_wattn_path(d) == want
@@ -115,8 +116,9 @@ def _a256(x):
                                   "tiny-16x16-w4"])
 def test_workspace_size_follows_the_documented_layout(L, name):
     """Tensor-core families: 256-byte header, the transposed bias table
-    [heads][bins padded to 4] fp32 and the fixed-point bias gradient
-    [heads][bins padded] int64, each region 256-byte aligned. Portable
+    [heads][bins padded to 4] fp32 and the exact bias-gradient sums
+    [heads][bins padded][9 limbs + 1 flag] int64, each region 256-byte
+    aligned. Portable
     kernels: header, per-row partials (3 floats per window slot and head) and
     per-window bias-gradient partials."""
     wl = WORKLOADS[name]
@@ -124,7 +126,7 @@ def test_workspace_size_follows_the_documented_layout(L, name):
     bins = (2 * wl.win - 1) ** 2
     bp = (bins + 3) // 4 * 4
     if sb.swin_wattn_path(d) in (1, 2):
-        want = 256 + _a256(wl.heads * bp * 4) + _a256(wl.heads * bp * 8)
+        want = 256 + _a256(wl.heads * bp * 4) + _a256(wl.heads * bp * 10 * 8)
     else:
         hp = -(-wl.H // wl.win) * wl.win
         wp = -(-wl.W // wl.win) * wl.win

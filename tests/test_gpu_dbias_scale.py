@@ -1,0 +1,88 @@
+"""The bias-table gradient at the magnitudes a training step feeds it.
+
+A loss averaged over many tokens hands this op output gradients far below 1,
+so dT must keep its relative accuracy at any scale of dO. These tests scale dO
+by 1e-3, 1e-6 and 1e3 (the inputs, not the outputs: the oracle runs on the
+same scaled bf16 values) and hold every output to the same RMS-relative bar
+on both tensor-core kernel families, check that repeated calls give the same
+bits, and that a NaN in one head's dO reaches that head's dT only."""
+import numpy as np
+import pytest
+import torch
+
+from shifted_window_attention_pad_b200 import WORKLOADS, binding as sb
+from shifted_window_attention_pad_b200.synth import make_inputs
+from shifted_window_attention_pad_b200.workloads import Workload
+
+from gpu_helpers import BF16_TOL, compare, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from shifted_window_attention_pad_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+def _table(win, heads, seed):
+    nb = (2 * win[0] - 1) * (2 * win[1] - 1)
+    return torch.from_numpy(np.random.Generator(np.random.PCG64(seed)).standard_normal(
+        (nb, heads)).astype(np.float32) * 0.02)
+
+
+# (name, description, inputs): the ragged workload on the tcgen05 kernels and a
+# padded 16 x 16-window grid on the warp-MMA kernels
+def _cases():
+    wl = WORKLOADS["ragged-90x180-w8"]
+    yield "tcgen05-ragged", sb.desc_for(wl), make_inputs(wl), 1
+    d = sb.make_desc(1, 40, 52, 16, 8, 2, 64, "bf16")
+    w16 = Workload("w16", 1, 40, 52, 16, 8, 2, 64, "bf16", 41)
+    inp = make_inputs(w16)
+    yield "warp-mma-40x52-w16", d, inp, 2
+
+
+CASES = list(_cases())
+
+
+@pytest.mark.parametrize("scale", [1e-3, 1e-6, 1e3])
+@pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
+def test_gradients_keep_their_relative_accuracy_at_any_scale_of_dout(case, scale):
+    name, d, inp, path = case
+    assert sb.swin_wattn_path(d) == path
+    inp = dict(inp)
+    inp["dout"] = (inp["dout"].to(torch.float32) * scale).to(torch.bfloat16)
+    gpu = run_gpu(d, inp, want_lse=False)
+    ref = run_oracle(d, inp)
+    errs = compare(gpu, ref, "bf16", names=("dq", "dk", "dv", "dT"))
+    print(name, scale, errs)
+    assert set(errs) == {"dq", "dk", "dv", "dT"}
+    for n, e in errs.items():
+        assert e <= BF16_TOL, (name, scale, n, e)
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
+def test_small_gradient_backward_is_bitwise_repeatable(case):
+    name, d, inp, _ = case
+    inp = dict(inp)
+    inp["dout"] = (inp["dout"].to(torch.float32) * 1e-5).to(torch.bfloat16)
+    a = run_gpu(d, inp, want_lse=False)
+    b = run_gpu(d, inp, want_lse=False)
+    for n in ("dq", "dk", "dv", "dT"):
+        assert torch.equal(a[n], b[n]), (name, n)
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: c[0])
+def test_nan_in_one_head_reaches_only_that_heads_bias_gradient(case):
+    """Heads are independent: a NaN in head 0's dO makes head 0's dT NaN and
+    leaves every other head's dT bitwise as it was."""
+    name, d, inp, _ = case
+    clean = run_gpu(d, inp, want_lse=False, backward=True)
+    bad = dict(inp)
+    do = inp["dout"].clone()
+    do[0, 3, 5, 0, 7] = float("nan")
+    bad["dout"] = do
+    dirty = run_gpu(d, bad, want_lse=False, backward=True)
+    assert torch.isnan(dirty["dT"][:, 0]).any(), name
+    assert torch.equal(clean["dT"][:, 1:], dirty["dT"][:, 1:]), name

@@ -50,6 +50,83 @@ def test_index_map_bit_exact_sweep(H, W, w, s):
     assert np.array_equal(gpu.astype(np.int64), oracle.index_map(oracle_shape(d)))
 
 
+# The same bit-exact bar for the layout stage as the tcgen05 kernels run it:
+# their TMA boxes (seam windows split into sub-boxes), the row order those
+# boxes leave in shared memory and the per-row token and region each kernel
+# derives. Every description here runs on those kernels (path 1).
+FAST_LAYOUT = ([(1, H, W, (8, 8), (s, s), 3, hd) for (H, W) in [(1, 1), (5, 7), (16, 16), (17, 40),
+                                                                (40, 3), (90, 180)]
+                for s in (4, 0) for hd in (32, 64, 128)] +
+               [(2, 18, 30, win, sh, 2, 64) for (win, sh) in [((4, 16), (2, 8)), ((16, 4), (8, 2)),
+                                                                ((2, 32), (1, 16)), ((4, 16), (0, 0))]])
+
+
+def _check_layout(d):
+    assert sb.swin_wattn_path(d) == 1
+    m, lab = sb.swin_wattn_layout_map(d)
+    torch.cuda.synchronize()
+    s = oracle_shape(d)
+    ref = oracle.index_map(s)
+    got = m.cpu().numpy().reshape(ref.shape).astype(np.int64)
+    assert not np.any(got == -2)
+    assert np.array_equal(got, ref)
+    rl = oracle.region_labels(s)
+    lab = lab.cpu().numpy().reshape(d.B, -1, d.win_h * d.win_w)
+    for b in range(d.B):
+        assert np.array_equal(lab[b], rl)
+
+
+@pytest.mark.parametrize("case", FAST_LAYOUT, ids=lambda c: "%dx%dx%d-w%dx%d-s%dx%d-hd%d" % (
+    c[0], c[1], c[2], *c[3], *c[4], c[6]))
+def test_tcgen05_layout_stage_bit_exact(case):
+    B, H, W, win, shift, heads, hd = case
+    _check_layout(sb.make_desc(B, H, W, win, shift, heads, hd, "bf16"))
+
+
+@pytest.mark.parametrize("name", ["ragged-90x180-w8", "twelfth-degree-256x544-w8",
+                                  "small-patch-2x512x1088-w8"])
+def test_tcgen05_layout_stage_bit_exact_on_workloads(name):
+    _check_layout(sb.desc_for(WORKLOADS[name]))
+
+
+@pytest.mark.parametrize("valid", [(256, 540), (251, 537)])
+def test_tcgen05_layout_stage_with_a_valid_extent(valid):
+    """The 1/12-degree token grid whose last columns (or rows) cover only
+    padded field pixels: those slots read as padding."""
+    wl = WORKLOADS["twelfth-degree-256x544-w8"]
+    _check_layout(sb.make_desc(1, wl.H, wl.W, 8, 4, 2, 64, "bf16", valid=valid))
+
+
+# ---------------------------------------------------------------------------
+# Valid extent: stored tokens over padded field pixels (all kernel families)
+# ---------------------------------------------------------------------------
+VALID = [
+    (1, Workload("valid-tcgen05", 2, 40, 56, 8, 4, 3, 64, "bf16", 71, valid=(37, 50))),
+    (2, Workload("valid-warp-mma", 1, 40, 52, 16, 8, 2, 64, "bf16", 72, valid=(35, 47))),
+    (0, Workload("valid-portable", 1, 13, 18, 4, 2, 2, 16, "f32", 73, valid=(11, 15))),
+    (1, Workload("valid-1/12-degree-field", 1, 256, 544, 8, 4, 4, 64, "bf16", 74,
+                 valid=sb.field_valid_extent(2041, 4320, 8))),
+]
+
+
+@pytest.mark.parametrize("case", VALID, ids=lambda c: c[1].name)
+def test_valid_extent_parity(case):
+    path, wl = case
+    d = sb.desc_for(wl)
+    assert sb.swin_wattn_path(d) == path
+    inp = make_inputs(wl)
+    gpu = run_gpu(d, inp)
+    ref = run_oracle(d, inp)
+    vh, vw = wl.valid
+    for n in ("o", "lse", "dq", "dk", "dv"):
+        g = gpu[n].cpu()
+        assert torch.all(g[:, vh:] == 0) and torch.all(g[:, :, vw:] == 0), n
+    errs = compare(gpu, ref, wl.dtype)
+    print(wl.name, errs)
+    for n, e in errs.items():
+        assert e <= tol(wl.dtype), (wl.name, n, e)
+
+
 # ---------------------------------------------------------------------------
 # Parity on the five workloads
 # ---------------------------------------------------------------------------
@@ -285,3 +362,65 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     ref = run_oracle(d_ok, inp)
     for n, e in compare(gpu, ref, "bf16").items():
         assert e <= BF16_TOL, (n, e)
+
+
+# ---------------------------------------------------------------------------
+# head_dim 128 on the tcgen05 kernels (TERRA page, Table V: every model size
+# uses 128-channel heads): two channel halves per TMA box, P kept in TMEM as
+# the A operand of P V, a one-stage, one-slot backward
+# ---------------------------------------------------------------------------
+HD128 = [
+    Workload("hd128-ragged-90x180", 1, 90, 180, 8, 4, 2, 128, "bf16", 81),
+    Workload("hd128-batch2-20x28", 2, 20, 28, 8, 4, 3, 128, "bf16", 82),
+    Workload("hd128-noshift-24x40", 1, 24, 40, 8, 0, 2, 128, "bf16", 83),
+    Workload("hd128-tiny-5x6", 1, 5, 6, 8, 4, 1, 128, "bf16", 84),
+]
+
+
+@pytest.mark.parametrize("wl", HD128, ids=lambda w: w.name)
+def test_head_dim_128_parity(wl):
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    assert sb.swin_wattn_path(d) == 1
+    errs = compare(run_gpu(d, inp), run_oracle(d, inp), "bf16")
+    print(wl.name, errs)
+    assert set(errs) == {"o", "lse", "dq", "dk", "dv", "dT"}
+    for n, e in errs.items():
+        assert e <= BF16_TOL, (wl.name, n, e)
+
+
+@pytest.mark.parametrize("win,shift", [((4, 16), (2, 8)), ((16, 4), (8, 2))])
+def test_head_dim_128_non_square_windows(win, shift):
+    B, H, W, heads, hd = 1, 18, 30, 2, 128
+    d = sb.make_desc(B, H, W, win, shift, heads, hd, "bf16")
+    assert sb.swin_wattn_path(d) == 1
+    wl = Workload("ns128", B, H, W, win[0], shift[0], heads, hd, "bf16", 85)
+    inp = make_inputs(wl, shape_override=(B, H, W, heads, hd))
+    nb = (2 * win[0] - 1) * (2 * win[1] - 1)
+    inp["table"] = torch.from_numpy(
+        np.random.Generator(np.random.PCG64(6)).standard_normal((nb, heads)).astype(np.float32) * 0.02)
+    errs = compare(run_gpu(d, inp), run_oracle(d, inp), "bf16")
+    for n, e in errs.items():
+        assert e <= BF16_TOL, (win, n, e)
+
+
+def test_head_dim_128_table5_grid_two_heads():
+    """The 1/12-degree token grid with Table V's head size: 256 x 544 tokens,
+    8 heads x 128 (d = 1024). The whole problem runs on the GPU; heads 0 and 5
+    are checked against the oracle in full, and the backward repeats bitwise."""
+    wl = Workload("table5-256x544-8x128", 1, 256, 544, 8, 4, 8, 128, "bf16", 86)
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    assert sb.swin_wattn_path(d) == 1
+    gpu = run_gpu(d, inp, want_lse=False)
+    again = run_gpu(d, inp, want_lse=False)
+    for n in ("o", "dq", "dk", "dv", "dT"):
+        assert torch.equal(gpu[n], again[n]), n
+    for h in (0, 5):
+        sub = {n: inp[n][:, :, :, h:h + 1].contiguous() for n in ("q", "k", "v", "dout")}
+        sub["table"] = inp["table"][:, h:h + 1].contiguous()
+        ds = sb.make_desc(wl.B, wl.H, wl.W, wl.win, wl.shift, 1, wl.head_dim, wl.dtype)
+        g = {n: gpu[n][:, :, :, h:h + 1] for n in ("o", "dq", "dk", "dv")}
+        g["dT"] = gpu["dT"][:, h:h + 1]
+        for n, e in compare(g, run_oracle(ds, sub), "bf16").items():
+            assert e <= BF16_TOL, (h, n, e)
