@@ -67,6 +67,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=BENCH_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (and its second buffer set): profiler captures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0,
                     help="CPU seconds for the oracle baseline sample")
@@ -362,6 +364,10 @@ def run_ours(args):
     fwd_achieved = wl.alg_bytes_fwd() / (fwd_ms / 1e3) / 1e9
     step_gbs = (wl.alg_bytes_fwd() + wl.alg_bytes_bwd()) * K / secs / 1e9
 
+    if args.no_e2e:
+        return _finish(args, wl, desc, rank, world, ms, K, fwd_ms, bwd_ms, value, tflops, hbm,
+                       peak_src, achieved, fwd_achieved, step_gbs, bwd_bytes, launches, clocks,
+                       None, flush, in_bytes)
     # End to end through the public API with pinned host buffers: every step
     # uploads its own inputs and downloads its own results inside the timed
     # region. Two device buffer sets and three streams (upload, compute,
@@ -418,6 +424,16 @@ def run_ours(args):
         raise RuntimeError("device-side timeout in the end-to-end steps")
     h2d = sum(t.numel() * t.element_size() for t in h_in.values())
     d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    e2e = {"value": wl.tokens * E * world / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    return _finish(args, wl, desc, rank, world, ms, K, fwd_ms, bwd_ms, value, tflops, hbm,
+                   peak_src, achieved, fwd_achieved, step_gbs, bwd_bytes, launches, clocks, e2e,
+                   flush, in_bytes)
+
+
+def _finish(args, wl, desc, rank, world, ms, K, fwd_ms, bwd_ms, value, tflops, hbm, peak_src,
+            achieved, fwd_achieved, step_gbs, bwd_bytes, launches, clocks, e2e, flush, in_bytes):
+    from shifted_window_attention_pad_b200 import binding as sb
 
     clk = clocks.summary()
     if world > 1:
@@ -453,8 +469,7 @@ def run_ours(args):
                          "peak_source": peak_src, "traffic": traffic,
                          "alg_bytes_per_launch": bwd_bytes},
             "cpu_baseline": cpu,
-            "e2e": {"value": wl.tokens * E * world / (e2e_ms / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk,
         }

@@ -34,8 +34,7 @@
 //    follows the magnitude of the gradients, so the relative error does not
 //    depend on their scale; a last small kernel converts the sums to fp32.
 //  * Warp roles: warps 0-3 and 4-7 two softmax/epilogue warpgroups taking
-//    alternate tiles, warp 8 TMA producer (which also prefetches the tiles
-//    of the steps ahead into L2), warp 9 issues S (and dP) and owns TMEM,
+//    alternate tiles, warp 8 TMA producer, warp 9 issues S (and dP) and owns TMEM,
 //    warp 10 issues PV (or the gradient products). Persistent grid of one
 //    CTA per SM; tiles go round-robin, head fastest, so the SMs stream
 //    neighbouring bytes together.
@@ -109,9 +108,9 @@ struct Layout {
 };
 
 // NS stages of NTEN input tiles, then PBYTES of P / dS operand blocks, the
-// bias rows of the stages, per warpgroup two buffers of key words, the tile's
-// int32 bias-gradient bins and four per-warp bounds, mbarriers and two words
-// (TMEM base, abort flag).
+// bias rows of the stages, per warpgroup two buffers of key words, the int32
+// bias-gradient bins of its two windows and four per-warp bounds, mbarriers
+// and two words (TMEM base, abort flag).
 template <int HD, int NS, int NTEN, uint32_t PBYTES>
 __host__ __device__ inline Layout make_layout(int bins_pad) {
   constexpr uint32_t tile_bytes = kRows * HD * 2;
@@ -121,7 +120,7 @@ __host__ __device__ inline Layout make_layout(int bins_pad) {
   L.bias = L.ptile + PBYTES;
   L.colinfo = L.bias + ((NS * bins_pad * 4 + 15) & ~15);
   L.bins_w = L.colinfo + kNumWg * 2 * kRows * 4;
-  L.bars = (L.bins_w + kNumWg * (bins_pad + 4) * 4 + 7) & ~7u;
+  L.bars = (L.bins_w + kNumWg * (2 * bins_pad + 4) * 4 + 7) & ~7u;
   L.misc = L.bars + 8 * 32;
   L.total = L.misc + 16;
   return L;
@@ -274,32 +273,6 @@ __device__ inline void issue_tile_loads(const FastParams& p, long long t, uint8_
     }
   }
   if (bias_dst) bulk_load(bias_dst, p.bias_t + (size_t)h * p.bins_pad, p.bins_pad * 4, full);
-}
-
-// Producer: asks the TMA unit to bring the boxes of tile `t` into L2 ahead of
-// their shared-memory loads, so that those find the tile in L2 instead of
-// waiting for HBM. No barrier is involved and nothing lands in shared memory.
-template <int HD, int NTEN>
-__device__ inline void issue_tile_prefetch(const FastParams& p, long long t) {
-  const Geo& g = p.g;
-  const int G = kRows / g.N;
-  const long long group = t / g.heads;
-  const int h = (int)(t - group * g.heads);
-  for (int gw = 0; gw < G; ++gw) {
-    const long long win = group * G + gw;
-    if (win >= g.n_win) continue;
-    int b, wy, wx;
-    window_coords(g, win, b, wy, wx);
-    SubBox sb[4];
-    const int n = plan_window(g, wy, wx, sb);
-    for (int i = 0; i < n; ++i) {
-      if (sb[i].y >= g.H || sb[i].x >= g.W) continue;   // wholly in the padding
-      for (int tt = 0; tt < NTEN; ++tt)
-        for (int hf = 0; hf < TileGeom<HD>::kHalves; ++hf)
-          tma_prefetch_5d(&p.maps[tt][sb[i].map_id], hf * TileGeom<HD>::kBoxEl, h, sb[i].x,
-                          sb[i].y, b);
-    }
-  }
 }
 
 // K-major operand, rows of HD bf16 (128-byte swizzle for HD >= 64, 64-byte for
@@ -542,9 +515,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
-      const long long ahead = (long long)NS * gridDim.x;
-      for (long long t = blockIdx.x; t < p.n_tiles && t < blockIdx.x + ahead; t += gridDim.x)
-        issue_tile_prefetch<HD, 3>(p, t);
       long long k = 0;
       for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
         const int s = (int)(k % NS);
@@ -552,7 +522,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (!mbar_wait(&empty[s], ph ^ 1, abort, p.status, kWaitLimitNs)) break;
         mbar_arrive_expect_tx(&full[s], 3 * tile_bytes + p.bins_pad * 4);
         issue_tile_loads<HD, 3>(p, t, tiles + s * 3 * tile_bytes, bias + s * p.bins_pad, &full[s]);
-        if (t + ahead < p.n_tiles) issue_tile_prefetch<HD, 3>(p, t + ahead);
       }
       if (*abort) {  // let copies already in flight land before the CTA leaves
         const long long first = k > NS ? k - NS : 0;
@@ -731,8 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 // (nothing else lives there), and each warpgroup stores its gradient rows
 // straight from registers to their grid tokens. One thread issues S and dP of
 // each tile as soon as its data and slot are ready, another the gradient
-// products as soon as its blocks are written; the producer also asks for the
-// tiles two steps ahead to be brought into L2.
+// products as soon as its blocks are written.
 //
 // Bias-table gradient: per tile, a bound on |dS| (max P of the row times
 // max|dP| + |D|, maximised over the tile's rows) sets the exponent of an exact
@@ -740,8 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 // the wide integer sums of the workspace (dbias_fixed.cuh).
 // HD <= 64: two input stages, two TMEM slots of 256 columns (S | dP, then
 // dV | dQ | dK at 0 / 64 / 128), the two softmax warpgroups on alternate
-// tiles. HD = 128: a stage of four 32 KB tiles leaves room for one (the L2
-// prefetch keeps its refill short), and the three 128-column gradients need
+// tiles. HD = 128: a stage of four 32 KB tiles leaves room for one, and the
+// three 128-column gradients need
 // 384 columns, so one slot (dV | dQ | dK at 0 / 128 / 256 over S | dP) and
 // one softmax warpgroup.
 template <int HD>
@@ -812,8 +780,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* blocks = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
   uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
-  int* bins = (int*)(smem + L.bins_w);           // [wg][bins_pad] tile bins
-  float* tbound = (float*)(bins + kNumWg * bp);  // [wg][4] per-warp |dS| bounds
+  int* bins = (int*)(smem + L.bins_w);               // [wg][window][bins_pad] bins
+  float* tbound = (float*)(bins + kNumWg * 2 * bp);  // [wg][4] per-warp |dS| bounds
   uint64_t* bars = (uint64_t*)(smem + L.bars);
   uint64_t* full = bars;
   uint64_t* empty = full + NS;
@@ -847,7 +815,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     reinterpret_cast<uint4*>(blocks + kZ1 * kBlk)[i] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(blocks + kZ2 * kBlk)[i] = make_uint4(0, 0, 0, 0);
   }
-  for (int i = threadIdx.x; i < kNumWg * bp; i += kThreads) bins[i] = 0;
+  for (int i = threadIdx.x; i < kNumWg * 2 * bp; i += kThreads) bins[i] = 0;
   fence_proxy_async();
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
@@ -860,9 +828,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
-      const long long ahead = (long long)(NS + 1) * gridDim.x;
-      for (long long t = blockIdx.x; t < p.n_tiles && t < blockIdx.x + ahead; t += gridDim.x)
-        issue_tile_prefetch<HD, 4>(p, t);
       long long k = 0;
       for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
         const int s = (int)(k % NS);
@@ -870,7 +835,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         if (!mbar_wait(&empty[s], ph ^ 1, abort, p.status, kWaitLimitNs)) break;
         mbar_arrive_expect_tx(&full[s], 4 * tile_bytes + bp * 4);
         issue_tile_loads<HD, 4>(p, t, tiles + s * 4 * tile_bytes, bias + s * bp, &full[s]);
-        if (t + ahead < p.n_tiles) issue_tile_prefetch<HD, 4>(p, t + ahead);
       }
       if (*abort) {
         const long long first = k > NS ? k - NS : 0;
@@ -971,7 +935,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const uint32_t bb = smem_u32(blocks);
     const uint32_t blk_ph = bb + (gw ? kP1h : kP0h) * kBlk, blk_pl = bb + (gw ? kP1l : kP0l) * kBlk;
     const uint32_t blk_sh = bb + (gw ? kS1h : kS0h) * kBlk, blk_sl = bb + (gw ? kS1l : kS0l) * kBlk;
-    int* tb = bins + wg * bp;
+    int* tb = bins + wg * 2 * bp;   // [window][bins_pad]
     float* bnd = tbound + wg * 4;
     __nv_bfloat16* const outs[3] = {(__nv_bfloat16*)p.out2, (__nv_bfloat16*)p.out0,
                                     (__nv_bfloat16*)p.out1};   // TMEM order: dV, dQ, dK
@@ -1036,18 +1000,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       __syncwarp();
 #pragma unroll
       for (int c = 0; c < N / 32; ++c) tmem_st32(s_col + 32 * c, x + 32 * c);
-      // |dS_ij| = P_ij |dP_ij - D| <= max_j P_ij * (max_j |dP_ij| + |D|)
+      // |dS_ij| = P_ij |dP_ij - D| <= max_j P_ij * (max_j |dP_ij| + |D|); a NaN
+      // becomes +inf here, since fmaxf would drop it
       {
-        const float wb = warp_max(inv * (mdp + fabsf(D)));
+        float rb = inv * (mdp + fabsf(D));
+        if (!(rb <= 3.0e38f)) rb = INFINITY;
+        const float wb = warp_max(rb);
         if (lane == 0) bnd[warp & 3] = wb;
       }
       named_sync(3 + wg, kWg);
-      const float tile_bound = fmaxf(fmaxf(bnd[0], bnd[1]), fmaxf(bnd[2], bnd[3]));
-      const bool finite = tile_bound <= 3.0e38f;   // false for NaN and infinity
-      const int E = tile_exponent(finite ? tile_bound : 0.f);
+      // Each window has its own unit (warps 2gw and 2gw+1 hold its rows), so
+      // its integer sums do not depend on which window shares its tile.
+      const float win_bound = fmaxf(bnd[2 * gw], bnd[2 * gw + 1]);
+      const bool finite = win_bound <= 3.0e38f;   // false for NaN and infinity
+      const int E = tile_exponent(finite ? win_bound : 0.f);
       const float qs = exp2_int(E);
       tmem_wait_st();
-      int* bq = tb + me.bias_base;
+      int* bq = tb + gw * bp + me.bias_base;
 #pragma unroll 1
       for (int c = 0; c < N / 32; ++c) {
         float ds[32], pc[32];
@@ -1094,14 +1063,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&pds_full[sl]);
-      // This tile's bins into the workspace's exact sums.
+      // Both windows' bins into the workspace's exact sums, each in its unit.
       named_sync(5 + wg, kWg);
       long long* acc = p.dt_acc + (size_t)h * bp * kLimbStride;
-      for (int b = row; b < g.bins; b += kWg) {
-        const int v = tb[b];
-        tb[b] = 0;
-        if (!finite) flag_nonfinite(acc + (size_t)b * kLimbStride);
-        else if (v != 0) add_fixed(acc + (size_t)b * kLimbStride, v, E);
+      for (int i = row; i < 2 * g.bins; i += kWg) {
+        const int w2 = i >= g.bins;
+        const int b = i - (w2 ? g.bins : 0);
+        const float wbd = fmaxf(bnd[2 * w2], bnd[2 * w2 + 1]);
+        const bool fin = wbd <= 3.0e38f;
+        const int v = tb[w2 * bp + b];
+        tb[w2 * bp + b] = 0;
+        if (!fin) flag_nonfinite(acc + (size_t)b * kLimbStride);
+        else if (v != 0) add_fixed(acc + (size_t)b * kLimbStride, v, tile_exponent(wbd));
       }
       // epilogue: dV, dQ, dK rows from TMEM straight to their grid tokens
       mbar_wait(&grad_full[sl], pht, abort, p.status, kWaitLimitNs);

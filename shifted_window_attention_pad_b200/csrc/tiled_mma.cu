@@ -485,8 +485,10 @@ __device__ __forceinline__ void bwd_tile(const TiledParams& p, uint8_t* smem, co
     if (t4 == 0) {
       // |dS_ij| = P_ij |dP_ij - D_i| <= (1 / l_i) (max_j |dP_ij| + |D_i|);
       // non-negative floats order like their bit patterns (NaN above all)
-      const float b0 = l0 > 0.f ? (x0 + fabsf(d0 / l0)) / l0 : 0.f;
-      const float b1 = l1 > 0.f ? (x1 + fabsf(d1 / l1)) / l1 : 0.f;
+      float b0 = l0 > 0.f ? (x0 + fabsf(d0 / l0)) / l0 : 0.f;
+      float b1 = l1 > 0.f ? (x1 + fabsf(d1 / l1)) / l1 : 0.f;
+      if (!(b0 <= 3.0e38f)) b0 = INFINITY;   // NaN -> +inf: fmaxf would drop a NaN
+      if (!(b1 <= 3.0e38f)) b1 = INFINITY;
       atomicMax(bound_bits, __float_as_uint(fmaxf(b0, b1)));
       // P = 2^(logit - lse); rows without an allowed key (pad queries) get
       // lse = +inf, hence P = 0, in pass 2

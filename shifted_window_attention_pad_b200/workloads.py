@@ -82,6 +82,9 @@ WORKLOADS = {
         Workload("small-patch-2x512x1088-w8", 2, 512, 1088, 8, 4, 12, 64, "bf16", 4,
                  "patch 4 -> 512x1088 tokens, d=768 = 12 heads x 64, 8x8 windows, shift 4, "
                  "batch 2 (two rollout steps)"),
+        Workload("profile-128x544-w8", 1, 128, 544, 8, 4, 16, 64, "bf16", 6,
+                 "half of the 1/12-degree token grid (128 x 544 tokens, 16 heads x 64): the "
+                 "same kernels on 0.57 GB of inputs, for profiler captures"),
         Workload("table5-256x544-8x128-w8", 1, 256, 544, 8, 4, 8, 128, "bf16", 5,
                  "the 1/12-degree token grid with the 128-channel heads of Table V: "
                  "d=1024 = 8 heads x 128, 8x8 windows, shift 4"),
