@@ -208,47 +208,54 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle legs (baseline and reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample_step(wl, rows, inp_np):
-    """One oracle forward + backward on the sample: head 0 of the workload's
-    first `rows` grid rows of image 0 (a problem of the same window, shift and
-    head size). Returns (tokens of the full workload the work stands for, s)."""
+def oracle_sample_step(wl, rows, nh, inp_np):
+    """One oracle forward + backward on the sample: heads 0..nh-1 of the
+    workload's first `rows` grid rows of image 0 (a problem of the same window,
+    shift and head size). Returns (tokens of the full workload the work stands
+    for, seconds)."""
     import oracle
-    s = oracle.make_shape(1, rows, wl.W, wl.win, wl.shift, 1, wl.head_dim)
-    q, k, v, do, T = inp_np
+    s = oracle.make_shape(1, rows, wl.W, wl.win, wl.shift, nh, wl.head_dim)
+    q, k, v, do = (np.ascontiguousarray(a[:1, :rows, :, :nh].to(torch.float64).numpy())
+                   for a in inp_np[:4])
+    T = np.ascontiguousarray(inp_np[4][:, :nh].to(torch.float64).numpy())
     t0 = time.perf_counter()
-    oracle.forward(s, q[:, :rows], k[:, :rows], v[:, :rows], T)
-    oracle.backward(s, q[:, :rows], k[:, :rows], v[:, :rows], T, do[:, :rows])
+    oracle.forward(s, q, k, v, T)
+    oracle.backward(s, q, k, v, T, do)
     dt = time.perf_counter() - t0
-    # work is uniform per (token, head): the sample stands for rows*W tokens of one head
-    return rows * wl.W / wl.heads, dt
+    # work is uniform per (token, head): the sample stands for rows*W*nh token-heads
+    return rows * wl.W * nh / wl.heads, dt
 
 
-def oracle_inputs(wl, rows):
+def oracle_inputs(wl):
+    """The workload's inputs (CPU tensors in their storage type; each sample
+    widens its own slice to fp64)."""
     inp = make_inputs(wl)
-    f = lambda t: np.ascontiguousarray(t[:1, :rows, :, :1].to(torch.float64).numpy())
-    return (f(inp["q"]), f(inp["k"]), f(inp["v"]), f(inp["dout"]),
-            np.ascontiguousarray(inp["table"][:, :1].to(torch.float64).numpy()))
+    return inp["q"], inp["k"], inp["v"], inp["dout"], inp["table"]
 
 
-def pick_rows(wl, budget_s):
-    """Largest multiple of the window (<= H) whose oracle step fits the budget,
-    from a calibration step on one window row."""
+def pick_sample(wl, budget_s):
+    """(rows, heads) of image 0 whose oracle step fits the budget: whole window
+    rows of head 0 first, then more heads of the whole grid, from a calibration
+    step on one window row of head 0."""
     import oracle
     rows0 = min(wl.win, wl.H)
-    inp = oracle_inputs(wl, wl.H)
-    _, dt = oracle_sample_step(wl, rows0, inp)
+    inp = oracle_inputs(wl)
+    _, dt = oracle_sample_step(wl, rows0, 1, inp)
     per_row = dt / rows0
-    rows = int(budget_s / max(per_row, 1e-9)) // wl.win * wl.win
-    return max(rows0, min(wl.H, rows)), inp, oracle.num_threads()
+    rows = max(rows0, min(wl.H, int(budget_s / max(per_row, 1e-9)) // wl.win * wl.win))
+    nh = 1
+    if rows == wl.H:
+        nh = max(1, min(wl.heads, int(budget_s / max(per_row * wl.H, 1e-9))))
+    return rows, nh, inp, oracle.num_threads()
 
 
 def cpu_baseline(wl, budget_s):
-    rows, inp, cores = pick_rows(wl, budget_s)
-    tok, dt = oracle_sample_step(wl, rows, inp)
+    rows, nh, inp, cores = pick_sample(wl, budget_s)
+    tok, dt = oracle_sample_step(wl, rows, nh, inp)
     return {"value": tok / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": "fp64 oracle fwd+bwd on head 0 of grid rows 0..%d (x %d cols) of image 0; "
-                      "%.1f s; scaled to tokens/s of the full %d-head workload" %
-                      (rows - 1, wl.W, dt, wl.heads)}
+            "sample": "fp64 oracle fwd+bwd on heads 0..%d of grid rows 0..%d (x %d cols) of "
+                      "image 0; %.1f s; scaled to tokens/s of the full %d-head workload" %
+                      (nh - 1, rows - 1, wl.W, dt, wl.heads)}
 
 
 def run_reference(args):
@@ -258,17 +265,18 @@ def run_reference(args):
     wl = WORKLOADS[args.workload]
     steps, warmup = args.steps, args.warmup
     per_step = max(0.5, min(20.0, 150.0 / max(1, steps + warmup)))
-    rows, inp, cores = pick_rows(wl, per_step)
+    rows, nh, inp, cores = pick_sample(wl, per_step)
     for _ in range(warmup):
-        oracle_sample_step(wl, rows, inp)
+        oracle_sample_step(wl, rows, nh, inp)
     tok_total, t_total = 0.0, 0.0
     for _ in range(steps):
-        tok, dt = oracle_sample_step(wl, rows, inp)
+        tok, dt = oracle_sample_step(wl, rows, nh, inp)
         tok_total += tok
         t_total += dt
     value = tok_total / t_total
-    sample = ("fp64 oracle fwd+bwd per step on head 0 of grid rows 0..%d (x %d cols) of image 0, "
-              "scaled to tokens/s of the full %d-head workload" % (rows - 1, wl.W, wl.heads))
+    sample = ("fp64 oracle fwd+bwd per step on heads 0..%d of grid rows 0..%d (x %d cols) of "
+              "image 0, scaled to tokens/s of the full %d-head workload" %
+              (nh - 1, rows - 1, wl.W, wl.heads))
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": steps, "warmup": warmup, "ms_per_step": 1e3 * t_total / max(1, steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
