@@ -63,7 +63,8 @@ constexpr int kNumWg = 2;         // warpgroups 0 (warps 0-3) and 1 (warps 4-7) 
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;       // issues S (and dP); allocates and frees TMEM
 constexpr int kMma2Warp = 10;     // issues PV (forward) or the gradient products (backward)
-constexpr int kThreads = 352;
+constexpr int kFoldWarp = 11;     // backward: folds each tile's bias-gradient bins into global sums
+constexpr int kThreads = 384;
 constexpr int kMaxMaps = 9;       // box shapes: {full, seam part 1, seam part 2}^2
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kTestLimitNs = 1000000ull;
@@ -108,9 +109,9 @@ struct Layout {
 };
 
 // NS stages of NTEN input tiles, then PBYTES of P / dS operand blocks, the
-// bias rows of the stages, per warpgroup two buffers of key words, the int32
-// bias-gradient bins of its two windows and four per-warp bounds, mbarriers
-// and two words (TMEM base, abort flag).
+// bias rows of the stages, per warpgroup two buffers of key words, int32
+// bias-gradient bins per warp (two warps hold a window's rows) and four
+// per-warp bounds, mbarriers and two words (TMEM base, abort flag).
 template <int HD, int NS, int NTEN, uint32_t PBYTES>
 __host__ __device__ inline Layout make_layout(int bins_pad) {
   constexpr uint32_t tile_bytes = kRows * HD * 2;
@@ -120,7 +121,7 @@ __host__ __device__ inline Layout make_layout(int bins_pad) {
   L.bias = L.ptile + PBYTES;
   L.colinfo = L.bias + ((NS * bins_pad * 4 + 15) & ~15);
   L.bins_w = L.colinfo + kNumWg * 2 * kRows * 4;
-  L.bars = (L.bins_w + kNumWg * (2 * bins_pad + 4) * 4 + 7) & ~7u;
+  L.bars = (L.bins_w + kNumWg * (4 * bins_pad + 4) * 4 + 7) & ~7u;
   L.misc = L.bars + 8 * 32;
   L.total = L.misc + 16;
   return L;
@@ -328,6 +329,63 @@ __device__ inline void store_row_bf16(void* dst, const float* v, float mul) {
                  pack_bf16(v[c * 8 + 6] * mul, v[c * 8 + 7] * mul));
 }
 
+// NCH chunks of 16 bytes of this lane's row, from NCH * 8 values times `mul`,
+// rounded to bf16.
+template <int NCH>
+__device__ inline void pack_chunks(const float* v, float mul, uint4 (&a)[NCH]) {
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+    a[c] = make_uint4(pack_bf16(v[c * 8 + 0] * mul, v[c * 8 + 1] * mul),
+                      pack_bf16(v[c * 8 + 2] * mul, v[c * 8 + 3] * mul),
+                      pack_bf16(v[c * 8 + 4] * mul, v[c * 8 + 5] * mul),
+                      pack_bf16(v[c * 8 + 6] * mul, v[c * 8 + 7] * mul));
+}
+
+// Warp-collective: the warp's 32 rows (one per lane, NCH chunks of 16 bytes
+// each, `dst` = this lane's row or nullptr for a row that is not stored) go
+// to global memory so that every store instruction writes whole rows. Lanes
+// hold rows and a row's chunks are contiguous in memory, so a plain store
+// per chunk would touch 32 separate rows per instruction. Instead, an
+// NCH x NCH transpose of the chunks inside each group of NCH lanes (log2 NCH
+// butterfly steps of shuffles) leaves lane g*NCH + c with chunk c of the
+// group's rows g*NCH + t, t = 0..NCH-1, and each of the NCH stores writes
+// 32 / NCH whole rows.
+template <int NCH>
+__device__ inline void store_rows_coalesced(uint4 (&a)[NCH], const void* dst) {
+  const int lane = threadIdx.x & 31;
+  const int p = lane & (NCH - 1);
+#pragma unroll
+  for (int d = NCH / 2; d >= 1; d >>= 1) {
+    const bool hi = (p & d) != 0;
+#pragma unroll
+    for (int q = 0; q < NCH; ++q) {
+      if (q & d) continue;   // the pair of positions (q, q + d)
+      uint4 v = hi ? a[q] : a[q + d];   // the position whose bit differs from the lane's
+      v.x = __shfl_xor_sync(0xffffffffu, v.x, d);
+      v.y = __shfl_xor_sync(0xffffffffu, v.y, d);
+      v.z = __shfl_xor_sync(0xffffffffu, v.z, d);
+      v.w = __shfl_xor_sync(0xffffffffu, v.w, d);
+      if (hi) a[q] = v; else a[q + d] = v;
+    }
+  }
+  const int g0 = lane & ~(NCH - 1);
+#pragma unroll
+  for (int t = 0; t < NCH; ++t) {
+    const unsigned long long rp =
+        __shfl_sync(0xffffffffu, (unsigned long long)dst, g0 + t);
+    if (rp) st_global_v4(reinterpret_cast<uint4*>(rp) + p, a[t].x, a[t].y, a[t].z, a[t].w);
+  }
+}
+
+// Warp-collective: rows of OC values (OC = 32 or 64, times `mul`) of the
+// warp's 32 lanes, coalesced as above.
+template <int OC>
+__device__ inline void store_rows_bf16(const float* v, float mul, const void* dst) {
+  uint4 a[OC / 8];
+  pack_chunks<OC / 8>(v, mul, a);
+  store_rows_coalesced<OC / 8>(a, dst);
+}
+
 // Warp-collective (.sync.aligned): every lane of the warp must reach it.
 template <int NCOL>
 __device__ inline void tmem_load_cols(uint32_t taddr, float* v) {
@@ -432,19 +490,20 @@ __device__ inline float exp_sum(float* x, float m) {
 // while one waits on TMEM loads or an MMA the other computes (two warps per
 // scheduler). One thread issues S of each tile as soon as its data and TMEM
 // slot are ready, another PV as soon as its P is written.
-// HD <= 64: four TMEM slots of 128 columns (S, then O in the first HD), one
-// P tile per warpgroup in shared memory, three input stages.
-// HD = 128: three 96 KB stages and the P tiles do not fit in shared memory,
-// so P stays in TMEM: two slots of 256 columns, S in the first 128 (P
-// overwrites its first 64 as packed bf16 pairs, the A operand of O = P V),
-// O in the last 128; two input stages.
+// P stays in TMEM: S of a tile fills the first 128 columns of its slot, P
+// overwrites S's first 64 columns as packed bf16 pairs (the A operand of
+// O = P V) once the softmax has read S, and O goes after them. HD <= 64:
+// four slots of 128 columns (S | then P in 0-63, O in 64-127) and four input
+// stages; HD = 128: two slots of 256 columns (O in 128-255) and two 96 KB
+// input stages. (P in shared memory instead, as before: three stages at
+// HD = 64 and 8 KB of P stores per row of tiles.)
 template <int HD>
 struct FwdCfg {
-  static constexpr bool kTmemP = HD > 64;
-  static constexpr int kStages = kTmemP ? 2 : 3;
-  static constexpr int kSlots = kTmemP ? 2 : 4;
-  static constexpr uint32_t kSlotCols = kTmemP ? 256 : 128;
-  static constexpr uint32_t kOCol = kTmemP ? 128 : 0;    // O inside its slot
+  static constexpr bool kTmemP = true;
+  static constexpr int kStages = HD > 64 ? 2 : 4;
+  static constexpr int kSlots = HD > 64 ? 2 : 4;
+  static constexpr uint32_t kSlotCols = HD > 64 ? 256 : 128;
+  static constexpr uint32_t kOCol = HD > 64 ? 128 : 64;    // O inside its slot
   static constexpr uint32_t kPBytes = kTmemP ? 0 : kNumWg * 32768;
 };
 constexpr int kFwdPBufs = kNumWg;
@@ -780,8 +839,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* blocks = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
   uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
-  int* bins = (int*)(smem + L.bins_w);               // [wg][window][bins_pad] bins
-  float* tbound = (float*)(bins + kNumWg * 2 * bp);  // [wg][4] per-warp |dS| bounds
+  int* bins = (int*)(smem + L.bins_w);               // [wg][warp][bins_pad] bins
+  float* tbound = (float*)(bins + kNumWg * 4 * bp);  // [wg][4] per-warp |dS| bounds
   uint64_t* bars = (uint64_t*)(smem + L.bars);
   uint64_t* full = bars;
   uint64_t* empty = full + NS;
@@ -791,6 +850,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint64_t* t_empty = grad_full + NT;
   uint64_t* drain = t_empty + NT;   // [2]: one per MMA-issuing thread
   uint64_t* never = drain + 2;
+  uint64_t* gradv_full = never + 1;          // [NT] dV products done
+  uint64_t* bins_full = gradv_full + NT;     // [wg] a tile's bins are complete
+  uint64_t* bins_empty = bins_full + kNumWg; // [wg] ... and folded into global sums
   uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
   volatile int* abort = (volatile int*)(smem + L.misc + 4);
 
@@ -801,7 +863,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     for (int i = 0; i < NT; ++i) {
       mbar_init(&sdp_full[i], 1); mbar_init(&pds_full[i], kWg);
       mbar_init(&grad_full[i], 1); mbar_init(&t_empty[i], kWg);
+      mbar_init(&gradv_full[i], 1);
     }
+    for (int i = 0; i < kNumWg; ++i) { mbar_init(&bins_full[i], kWg); mbar_init(&bins_empty[i], 32); }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     mbar_init(never, 1);
@@ -815,7 +879,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     reinterpret_cast<uint4*>(blocks + kZ1 * kBlk)[i] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(blocks + kZ2 * kBlk)[i] = make_uint4(0, 0, 0, 0);
   }
-  for (int i = threadIdx.x; i < kNumWg * 2 * bp; i += kThreads) bins[i] = 0;
+  for (int i = threadIdx.x; i < kNumWg * 4 * bp; i += kThreads) bins[i] = 0;
   fence_proxy_async();
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
@@ -906,6 +970,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           umma_ss(d + 0, aPh[kk >> 2] + a, bO + b, idesc_t, kk);
           umma_ss(d + 0, aPl[kk >> 2] + a, bO + b, idesc_t, 1);
         }
+        umma_commit(&gradv_full[sl]);   // its rows can leave while dQ and dK run
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk) {  // dQ = dS K
           const uint32_t a = (kk & 3) * kStepK, b = kk * kStepB;
@@ -926,6 +991,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         mbar_drain(&drain[1], 0, kTestLimitNs * 100);
       }
     }
+  } else if (warp == kFoldWarp) {
+    // Each tile's bins, per warp, into the workspace's exact sums: the two
+    // warps of a window add up (exact integers), in the window's own unit.
+    for (long long k = 0, t = blockIdx.x; k < n_local; ++k, t += gridDim.x) {
+      const int wgk = (int)(k % NWG);
+      if (!mbar_wait(&bins_full[wgk], (uint32_t)((k / NWG) & 1), abort, p.status, kWaitLimitNs))
+        break;
+      const int h = (int)(t - (t / g.heads) * g.heads);
+      int* tbk = bins + wgk * 4 * bp;
+      const float* bk = tbound + wgk * 4;
+      long long* acc = p.dt_acc + (size_t)h * bp * kLimbStride;
+      for (int i = lane; i < 2 * g.bins; i += 32) {
+        const int w2 = i >= g.bins;
+        const int b = i - (w2 ? g.bins : 0);
+        const float wbd = fmaxf(bk[2 * w2], bk[2 * w2 + 1]);
+        const bool fin = wbd <= 3.0e38f;
+        int* b0 = tbk + (2 * w2) * bp + b;
+        int* b1 = b0 + bp;
+        const int v = *b0 + *b1;
+        *b0 = 0;
+        *b1 = 0;
+        if (!fin) flag_nonfinite(acc + (size_t)b * kLimbStride);
+        else if (v != 0) add_fixed(acc + (size_t)b * kLimbStride, v, tile_exponent(wbd));
+      }
+      mbar_arrive(&bins_empty[wgk]);
+    }
   } else if (warp < NWG * 4) {
     const int wg = warp >> 2;
     const int row = threadIdx.x & (kWg - 1);
@@ -935,7 +1026,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const uint32_t bb = smem_u32(blocks);
     const uint32_t blk_ph = bb + (gw ? kP1h : kP0h) * kBlk, blk_pl = bb + (gw ? kP1l : kP0l) * kBlk;
     const uint32_t blk_sh = bb + (gw ? kS1h : kS0h) * kBlk, blk_sl = bb + (gw ? kS1l : kS0l) * kBlk;
-    int* tb = bins + wg * 2 * bp;   // [window][bins_pad]
+    int* tb = bins + (wg * 4 + (warp & 3)) * bp;   // this warp's bins
     float* bnd = tbound + wg * 4;
     __nv_bfloat16* const outs[3] = {(__nv_bfloat16*)p.out2, (__nv_bfloat16*)p.out0,
                                     (__nv_bfloat16*)p.out1};   // TMEM order: dV, dQ, dK
@@ -1000,6 +1091,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       __syncwarp();
 #pragma unroll
       for (int c = 0; c < N / 32; ++c) tmem_st32(s_col + 32 * c, x + 32 * c);
+      // The bins and bounds are free once the fold warp has taken this
+      // warpgroup's previous tile.
+      if (k >= NWG)
+        mbar_wait(&bins_empty[wg], (uint32_t)(((k / NWG) - 1) & 1), abort, p.status,
+                  kWaitLimitNs);
       // |dS_ij| = P_ij |dP_ij - D| <= max_j P_ij * (max_j |dP_ij| + |D|); a NaN
       // becomes +inf here, since fmaxf would drop it
       {
@@ -1016,7 +1112,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const int E = tile_exponent(finite ? win_bound : 0.f);
       const float qs = exp2_int(E);
       tmem_wait_st();
-      int* bq = tb + gw * bp + me.bias_base;
+      int* bq = tb + me.bias_base;
 #pragma unroll 1
       for (int c = 0; c < N / 32; ++c) {
         float ds[32], pc[32];
@@ -1043,6 +1139,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         tmem_st32(dp_col + 32 * c, ds);
       }
       tmem_wait_st();
+      mbar_arrive(&bins_full[wg]);   // the fold warp adds them to the global sums
       // The operand blocks are free once the previous tile's gradient
       // products have completed (grad_full of the other slot; this warpgroup
       // saw that barrier's phase before, two tiles ago, so the parity names
@@ -1063,25 +1160,26 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&pds_full[sl]);
-      // Both windows' bins into the workspace's exact sums, each in its unit.
-      named_sync(5 + wg, kWg);
-      long long* acc = p.dt_acc + (size_t)h * bp * kLimbStride;
-      for (int i = row; i < 2 * g.bins; i += kWg) {
-        const int w2 = i >= g.bins;
-        const int b = i - (w2 ? g.bins : 0);
-        const float wbd = fmaxf(bnd[2 * w2], bnd[2 * w2 + 1]);
-        const bool fin = wbd <= 3.0e38f;
-        const int v = tb[w2 * bp + b];
-        tb[w2 * bp + b] = 0;
-        if (!fin) flag_nonfinite(acc + (size_t)b * kLimbStride);
-        else if (v != 0) add_fixed(acc + (size_t)b * kLimbStride, v, tile_exponent(wbd));
+      // epilogue: dV (as soon as its products are done), then dQ and dK,
+      // from TMEM to their grid tokens in whole-row stores (zero rows beyond
+      // the valid extent)
+      constexpr int OC = HD > 64 ? 64 : HD;   // columns per TMEM read
+      const bool st_row = me.stored && !*abort;
+      const long long roff = (me.token * g.heads + h) * HD;
+      mbar_wait(&gradv_full[sl], pht, abort, p.status, kWaitLimitNs);
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < HD; c0 += OC) {
+        float o[OC];
+        tmem_load_cols<OC>(tmem + lane_base + sl * 256 + c0, o);
+        tmem_wait_ld();
+        store_rows_bf16<OC>(o, 1.f, st_row ? (const void*)((me.halo ? outs_h[0] : outs[0]) + roff + c0)
+                                           : nullptr);
       }
-      // epilogue: dV, dQ, dK rows from TMEM straight to their grid tokens
       mbar_wait(&grad_full[sl], pht, abort, p.status, kWaitLimitNs);
       tc_fence_after();
-      constexpr int OC = HD > 64 ? 64 : HD;   // columns per TMEM read
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {
+      for (int part = 1; part < 3; ++part) {
 #pragma unroll
         for (int c0 = 0; c0 < HD; c0 += OC) {
           float o[OC];
@@ -1091,9 +1189,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
             tc_fence_before();
             mbar_arrive(&t_empty[sl]);
           }
-          if (me.stored && !*abort)   // zero rows beyond the valid extent
-            store_row_bf16<OC>((me.halo ? outs_h[part] : outs[part]) +
-                                   (me.token * g.heads + h) * HD + c0, o, 1.f);
+          store_rows_bf16<OC>(o, 1.f, st_row ? (const void*)((me.halo ? outs_h[part] : outs[part]) +
+                                                              roff + c0)
+                                             : nullptr);
         }
       }
     }
