@@ -66,6 +66,13 @@ cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void
 cudaError_t fast_layout_map(const Geo& g, void* ids, int32_t* map, int32_t* labels,
                             cudaStream_t st);
 
+// ---- tcgen05 / TMA kernels for 256-token windows (bf16, head_dim 32 or 64);
+// workspace as fast_workspace --------------------------------------------------
+bool wide_supported(const Geo& g, int dtype);
+cudaError_t wide_forward(const Geo& g, const void* q, const void* k, const void* v,
+                         const float* table, void* out, float* lse, void* ws, int flags,
+                         cudaStream_t st);
+
 // ---- warp-level tensor-core kernels: one CTA per (window, head), windows of
 // up to 256 tokens (bf16, head_dim 32 or 64) ----------------------------------
 bool tiled_supported(const Geo& g, int dtype);

@@ -43,25 +43,28 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_path_selection_on_the_workloads(L):
-    """tcgen05 kernels (1) for bf16 64-token windows, warp-MMA kernels (2) for
-    the 256-token windows, portable kernels (0) for fp32."""
+    """tcgen05 kernels for bf16 64-token windows (1) and 256-token windows (3),
+    portable kernels (0) for fp32."""
     expect = {"tiny-16x16-w4": 0, "ragged-90x180-w8": 1, "twelfth-degree-256x544-w8": 1,
-              "downsampled-128x272-w16": 2, "small-patch-2x512x1088-w8": 1}
+              "downsampled-128x272-w16": 3, "small-patch-2x512x1088-w8": 1}
     for name, want in expect.items():
         assert sb.swin_wattn_path(sb.desc_for(WORKLOADS[name])) == want, name
     d = sb.desc_for(WORKLOADS["twelfth-degree-256x544-w8"], flags=sb.SWIN_FLAG_FORCE_GENERIC)
     assert sb.swin_wattn_path(d) == 0
     d = sb.desc_for(WORKLOADS["twelfth-degree-256x544-w8"], flags=sb.SWIN_FLAG_FORCE_TILED)
     assert sb.swin_wattn_path(d) == 2
+    d = sb.desc_for(WORKLOADS["downsampled-128x272-w16"], flags=sb.SWIN_FLAG_FORCE_TILED)
+    assert sb.swin_wattn_path(d) == 2
     d = sb.desc_for(WORKLOADS["tiny-16x16-w4"], flags=sb.SWIN_FLAG_FORCE_TILED)
     assert sb.swin_wattn_path(d) == 0      # fp32 has no tensor-core path
 
 
-@pytest.mark.parametrize("win,hd,want", [((7, 7), 64, 2), ((8, 12), 32, 2), ((16, 16), 64, 2),
+@pytest.mark.parametrize("win,hd,want", [((7, 7), 64, 2), ((8, 12), 32, 2), ((16, 16), 64, 3),
+                                         ((16, 16), 32, 3), ((8, 32), 64, 3), ((16, 8), 64, 2),
                                          ((12, 12), 32, 2), ((16, 17), 64, 0), ((32, 32), 64, 0),
                                          ((16, 16), 128, 0), ((8, 8), 64, 1), ((8, 8), 128, 1),
                                          ((4, 16), 128, 1), ((7, 7), 128, 0)])
-def test_tiled_path_covers_windows_up_to_256_tokens(L, win, hd, want):
+def test_tensor_core_paths_cover_windows_up_to_256_tokens(L, win, hd, want):
     d = sb.make_desc(1, 40, 52, win, (win[0] // 2, win[1] // 2), 2, hd, "bf16")
     assert sb.swin_wattn_path(d) == want
 
@@ -125,7 +128,7 @@ def test_workspace_size_follows_the_documented_layout(L, name):
     d = sb.desc_for(wl)
     bins = (2 * wl.win - 1) ** 2
     bp = (bins + 3) // 4 * 4
-    if sb.swin_wattn_path(d) in (1, 2):
+    if sb.swin_wattn_path(d) in (1, 2, 3):
         want = 256 + _a256(wl.heads * bp * 4) + _a256(wl.heads * bp * 10 * 8)
     else:
         hp = -(-wl.H // wl.win) * wl.win

@@ -32,15 +32,17 @@ def _table(win, heads, seed):
         (nb, heads)).astype(np.float32) * 0.02)
 
 
-# (name, description, inputs): the ragged workload on the tcgen05 kernels and a
-# padded 16 x 16-window grid on the warp-MMA kernels
+# (name, description, inputs, path): the ragged workload on the tcgen05 kernels
+# and a padded 16 x 16-window grid on the 256-token tcgen05 kernels and on the
+# warp-MMA kernels
 def _cases():
     wl = WORKLOADS["ragged-90x180-w8"]
     yield "tcgen05-ragged", sb.desc_for(wl), make_inputs(wl), 1
-    d = sb.make_desc(1, 40, 52, 16, 8, 2, 64, "bf16")
     w16 = Workload("w16", 1, 40, 52, 16, 8, 2, 64, "bf16", 41)
     inp = make_inputs(w16)
-    yield "warp-mma-40x52-w16", d, inp, 2
+    yield "tcgen05-40x52-w16", sb.make_desc(1, 40, 52, 16, 8, 2, 64, "bf16"), inp, 3
+    yield ("warp-mma-40x52-w16",
+           sb.make_desc(1, 40, 52, 16, 8, 2, 64, "bf16", flags=sb.SWIN_FLAG_FORCE_TILED), inp, 2)
 
 
 CASES = list(_cases())

@@ -102,7 +102,8 @@ def test_tcgen05_layout_stage_with_a_valid_extent(valid):
 # ---------------------------------------------------------------------------
 VALID = [
     (1, Workload("valid-tcgen05", 2, 40, 56, 8, 4, 3, 64, "bf16", 71, valid=(37, 50))),
-    (2, Workload("valid-warp-mma", 1, 40, 52, 16, 8, 2, 64, "bf16", 72, valid=(35, 47))),
+    (3, Workload("valid-tcgen05-w16", 1, 40, 52, 16, 8, 2, 64, "bf16", 72, valid=(35, 47))),
+    (2, Workload("valid-warp-mma", 1, 40, 52, 16, 8, 2, 64, "bf16", 75, valid=(33, 49))),
     (0, Workload("valid-portable", 1, 13, 18, 4, 2, 2, 16, "f32", 73, valid=(11, 15))),
     (1, Workload("valid-1/12-degree-field", 1, 256, 544, 8, 4, 4, 64, "bf16", 74,
                  valid=sb.field_valid_extent(2041, 4320, 8))),
@@ -112,7 +113,7 @@ VALID = [
 @pytest.mark.parametrize("case", VALID, ids=lambda c: c[1].name)
 def test_valid_extent_parity(case):
     path, wl = case
-    d = sb.desc_for(wl)
+    d = sb.desc_for(wl, flags=sb.SWIN_FLAG_FORCE_TILED if path == 2 else 0)
     assert sb.swin_wattn_path(d) == path
     inp = make_inputs(wl)
     gpu = run_gpu(d, inp)
@@ -233,9 +234,44 @@ TILED = [
 @pytest.mark.parametrize("case", TILED, ids=lambda c: "%dx%d-w%dx%d-hd%d" % (c[1], c[2], *c[3], c[6]))
 def test_tiled_path_parity(case):
     B, H, W, win, shift, heads, hd, seed = case
-    d = sb.make_desc(B, H, W, win, shift, heads, hd, "bf16")
+    # (256-token windows go to the tcgen05 kernels unless the warp-MMA ones are forced)
+    d = sb.make_desc(B, H, W, win, shift, heads, hd, "bf16", flags=sb.SWIN_FLAG_FORCE_TILED)
     assert sb.swin_wattn_path(d) == 2
     wl = Workload("tiled", B, H, W, win[0], shift[0], heads, hd, "bf16", seed)
+    inp = make_inputs(wl, shape_override=(B, H, W, heads, hd))
+    nb = (2 * win[0] - 1) * (2 * win[1] - 1)
+    inp["table"] = torch.from_numpy(np.random.Generator(np.random.PCG64(seed)).standard_normal(
+        (nb, heads)).astype(np.float32) * 0.02)
+    errs = compare(run_gpu(d, inp), run_oracle(d, inp), "bf16")
+    print(case, errs)
+    for n, e in errs.items():
+        assert e <= BF16_TOL, (case, n, e)
+
+
+# ---------------------------------------------------------------------------
+# tcgen05 kernels for 256-token windows (path 3)
+# ---------------------------------------------------------------------------
+# (B, H, W, window, shift, heads, head_dim, seed): a padded grid with both
+# seams, no shift, head_dim 32, batch > 1, a grid smaller than one window,
+# 8 x 32 windows (seam sub-boxes of 8 x 16 tokens), the 16 x 16 window row of
+# the downsampled grid
+WIDE = [
+    (1, 40, 52, (16, 16), (8, 8), 2, 64, 81),
+    (1, 32, 48, (16, 16), (0, 0), 2, 64, 82),
+    (2, 36, 30, (16, 16), (8, 8), 3, 32, 83),
+    (1, 11, 13, (16, 16), (8, 8), 2, 64, 84),
+    (1, 24, 70, (8, 32), (4, 16), 2, 64, 85),
+    (1, 16, 272, (16, 16), (8, 8), 4, 64, 86),
+]
+
+
+@pytest.mark.parametrize("case", WIDE, ids=lambda c: "%dx%dx%d-w%dx%d-s%d-hd%d" % (
+    c[0], c[1], c[2], *c[3], c[4][0], c[6]))
+def test_wide_path_parity(case):
+    B, H, W, win, shift, heads, hd, seed = case
+    d = sb.make_desc(B, H, W, win, shift, heads, hd, "bf16")
+    assert sb.swin_wattn_path(d) == 3
+    wl = Workload("wide", B, H, W, win[0], shift[0], heads, hd, "bf16", seed)
     inp = make_inputs(wl, shape_override=(B, H, W, heads, hd))
     nb = (2 * win[0] - 1) * (2 * win[1] - 1)
     inp["table"] = torch.from_numpy(np.random.Generator(np.random.PCG64(seed)).standard_normal(
