@@ -46,7 +46,7 @@ static int choose_path(const swin_wattn_desc* d, const Geo& g) {
   if (d->flags & SWIN_FLAG_FORCE_GENERIC) return 0;
   if (!(d->flags & SWIN_FLAG_FORCE_TILED)) {
     if (fast_supported(g, d->dtype)) return 1;
-    if (wide_supported(g, d->dtype) && tiled_supported(g, d->dtype)) return 3;
+    if (wide_supported(g, d->dtype)) return 3;
   }
   if (tiled_supported(g, d->dtype)) return 2;
   return 0;
@@ -140,7 +140,10 @@ int swin_wattn_bwd(const swin_wattn_desc* desc, const void* q, const void* k, co
   if (path == 1)
     return cuda_status(fast_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
                                      workspace, desc->flags, st));
-  if (path == 2 || path == 3)
+  if (path == 3)
+    return cuda_status(wide_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
+                                     workspace, desc->flags, st));
+  if (path == 2)
     return cuda_status(tiled_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
                                       workspace, desc->flags, st));
   return cuda_status(generic_backward(g, desc->dtype, q, k, v, bias_table, dout, dq, dk, dv,

@@ -447,6 +447,12 @@ __device__ inline float exp_sum(float* x, float m) {
   return (l[0] + l[1]) + (l[2] + l[3]);
 }
 
+__device__ inline float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
 // Number of tiles CTA `cta` takes in a grid of `grid` CTAs.
 __device__ inline long long local_tiles(long long n_tiles, long long cta, long long grid) {
   return cta < n_tiles ? (n_tiles - 1 - cta) / grid + 1 : 0;

@@ -378,12 +378,6 @@ __device__ inline void store_split_cols_part(uint32_t blk_hi, uint32_t blk_lo, i
   }
 }
 
-__device__ inline float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
 template <int HD, int WW>
 __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ FastParams p) {
   constexpr int N = 64, G = kRows / N;

@@ -72,6 +72,9 @@ bool wide_supported(const Geo& g, int dtype);
 cudaError_t wide_forward(const Geo& g, const void* q, const void* k, const void* v,
                          const float* table, void* out, float* lse, void* ws, int flags,
                          cudaStream_t st);
+cudaError_t wide_backward(const Geo& g, const void* q, const void* k, const void* v,
+                          const float* table, const void* dout, void* dq, void* dk, void* dv,
+                          float* dtable, void* ws, int flags, cudaStream_t st);
 
 // ---- warp-level tensor-core kernels: one CTA per (window, head), windows of
 // up to 256 tokens (bf16, head_dim 32 or 64) ----------------------------------

@@ -373,6 +373,520 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   }
 }
 
+// ================================================================================
+// Backward
+// ================================================================================
+// Per (window, head) item, with Q, K, V, dO of the window in shared memory:
+//  Phase 1, row statistics, query-major: for each 128-query half qt,
+//    S = Q_qt K^T and dP = dO_qt V^T over all 256 keys fill the 512 TMEM
+//    columns; warpgroup w reads keys 128 w .. 128 w + 127 of every row and
+//    keeps an online maximum M, l = sum 2^(x - M), d = sum 2^(x - M) dP and
+//    max |dP|; the two halves of a row are merged through shared memory into
+//    L = M + log2 l (log2 units) and D = d / l = sum_j P_ij dP_ij, and a bound
+//    (max_j |dP_ij| + |D|) / l >= |dS_ij| of the row. The largest bound of the
+//    window sets the unit 2^-E of its exact bias-gradient sums.
+//  Phase 2, gradients, key-major: for each block of 128 keys (kb) x 128
+//    queries (qt), S^T = K_kb Q_qt^T and dP^T = V_kb dO_qt^T (M = keys, so a
+//    thread holds one key and walks queries); P = 2^(x - L_i) and
+//    dS = P (dP - D_i) go back into their own columns as bf16 hi + lo pairs
+//    (the A operands, from TMEM, of dV_kb += P^T dO_qt and
+//    dK_kb += dS^T Q_qt), scale * dS also into shared memory as the MN-major
+//    A operand of dQ_qt += dS K_kb, and dS into the bias-gradient bins.
+//    Warpgroup w takes queries 64 w .. 64 w + 63 of the block.
+// TMEM: phase 1 S | dP at 0 | 256; phase 2 S^T | dP^T at 0 | 128, dV_kb at
+// 256, dK_kb at 320, dQ_0 at 384, dQ_1 at 448. dV and dK of a key half leave
+// after its two blocks, dQ after the last block.
+template <int HD>
+struct WideBwdCfg {
+  static constexpr uint32_t kRowBytes = HD * 2;
+  static constexpr uint32_t kTileBytes = kKeys * kRowBytes;
+  static constexpr int kStages = HD > 32 ? 1 : 2;
+  static constexpr uint32_t kOpBytes = 2 * 32768;   // scale * dS, hi and lo
+};
+constexpr uint32_t kColDP1 = 256;                    // phase 1 dP (S at 0)
+constexpr uint32_t kColDPT = 128;                    // phase 2 dP^T (S^T at 0)
+constexpr uint32_t kColDV = 256, kColDK = 320, kColDQ = 384;
+constexpr int kWideBwdWarps = 11;                    // 8 softmax, producer, MMA, bin fold
+constexpr int kWideFoldWarp = 10;
+
+struct WideBwdLayout {
+  uint32_t tiles, dsop, bias, colinfo, stats, xch, bins, wb, bars, misc, total;
+};
+
+template <int HD>
+__host__ __device__ inline WideBwdLayout wide_bwd_layout(int bins_pad) {
+  using C = WideBwdCfg<HD>;
+  WideBwdLayout L;
+  L.tiles = 0;
+  L.dsop = L.tiles + C::kStages * 4 * C::kTileBytes;
+  L.bias = L.dsop + C::kOpBytes;
+  L.colinfo = L.bias + ((C::kStages * bins_pad * 4 + 15) & ~15);
+  L.stats = L.colinfo + kKeys * 4;           // float2 {L, D} per query
+  L.xch = L.stats + kKeys * 8;               // [qt][4][128] partial statistics
+  L.bins = L.xch + 2 * 4 * kRows * 4;        // [2][bins_pad] int32 (item parity)
+  L.wb = L.bins + 2 * bins_pad * 4;          // [4] warp bounds, [2] E, [2] finite
+  L.bars = (L.wb + 64 + 7) & ~7u;
+  L.misc = L.bars + 8 * 32;
+  L.total = L.misc + 16;
+  return L;
+}
+
+// Scale * dS operand of dQ_qt += dS K_kb (M = 128 queries, K = 128 keys),
+// MN-major with 128-byte swizzle: 8 KB regions of 64 keys x 64 queries at
+// (key half * 2 + query half) * 8 KB, K step k16 = 16 keys.
+__device__ inline uint64_t desc_dsop(uint32_t base, int k16) {
+  return smem_desc(base + (k16 >> 2) * 16384 + (k16 & 3) * 2048, 8192, 1024, kSwizzle128);
+}
+
+// hi / lo bf16 pairs of 16 values: hw[c] = (hi(v[2c]), hi(v[2c+1])), hi = v
+// with the low 16 bits cleared; lw[c] the bf16 of the remainders.
+__device__ inline void split_pairs16(const float* v, uint32_t* hw, uint32_t* lw) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t a = __float_as_uint(v[2 * c]) & 0xFFFF0000u;
+    const uint32_t b = __float_as_uint(v[2 * c + 1]) & 0xFFFF0000u;
+    hw[c] = __byte_perm(a, b, 0x7632);
+    lw[c] = pack_bf16(v[2 * c] - __uint_as_float(a), v[2 * c + 1] - __uint_as_float(b));
+  }
+}
+
+// Phase 1 over 128 keys of one row (columns s_col.. of S and dp_col.. of dP,
+// keys k0base..): online maximum M, l, d and max |dP|.
+template <bool PLAIN, int WW>
+__device__ inline void wide_row_stats(uint32_t s_col, uint32_t dp_col, int k0base,
+                                      const float* brow, const uint32_t* ci, int bias_base,
+                                      int label, float c, float& M, float& l, float& d,
+                                      float& a) {
+  M = -INFINITY;
+  l = 0.f;
+  d = 0.f;
+  a = 0.f;
+#pragma unroll 1
+  for (int kc = 0; kc < kRows; kc += 32) {
+    float x[32], dp[32];
+    __syncwarp();
+    tmem_ld32(s_col + kc, x);
+    tmem_ld32(dp_col + kc, dp);
+    tmem_wait_ld();
+    const int k0 = k0base + kc;
+    float cm;
+    if constexpr (PLAIN)
+      cm = chunk_logits_plain<WW>(x, brow + bias_base, k0, c);
+    else
+      cm = logits_general<32>(x, brow, ci + k0, bias_base, label, c);
+    if (cm > M) {   // rescale the sums to the new maximum
+      const float f = ex2(M - cm);
+      l *= f;
+      d *= f;
+      M = cm;
+    }
+    const float Mz = M == -INFINITY ? 0.f : M;   // a chunk of masked keys adds zeros
+    float l0 = 0.f, l1 = 0.f, d0 = 0.f, d1 = 0.f, a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const float e0 = ex2(x[j] - Mz), e1 = ex2(x[j + 1] - Mz);
+      l0 += e0;
+      l1 += e1;
+      d0 = fmaf(e0, dp[j], d0);
+      d1 = fmaf(e1, dp[j + 1], d1);
+      a0 = fmaxf(a0, fabsf(dp[j]));
+      a1 = fmaxf(a1, fabsf(dp[j + 1]));
+    }
+    l += l0 + l1;
+    d += d0 + d1;
+    a = fmaxf(a, fmaxf(a0, a1));
+  }
+}
+
+// Phase 2, one chunk of 16 queries (i0 .. i0 + 15) of this thread's key: P
+// and dS from S^T and dP^T, their hi / lo pairs back to TMEM, scale * dS to the
+// dQ operand in shared memory, dS to the bias-gradient bins.
+template <bool PLAIN, int WW>
+__device__ inline void wide_grad_chunk(uint32_t st_col, uint32_t dpt_col, int i0,
+                                       const float2* stats, const uint32_t* ci,
+                                       const float* bk, int* bn, uint32_t keylab, bool bins_on,
+                                       float c, float qs, float dscale, uint32_t op_hi,
+                                       uint32_t op_lo) {
+  float s[16], dp[16];
+  __syncwarp();
+  tmem_ld16(st_col, s);
+  tmem_ld16(dpt_col, dp);
+  tmem_wait_ld();
+  float pv[16], dv[16];
+  const int ib = PLAIN ? plain_off<WW>(i0) : 0;   // i0 starts a window row
+#pragma unroll
+  for (int ii = 0; ii < 16; ++ii) {
+    const float2 st = stats[i0 + ii];
+    float x;
+    int off;
+    if constexpr (PLAIN) {
+      off = ib + plain_off<WW>(ii);
+      x = fmaf(s[ii], c, bk[off]);
+    } else {
+      const uint32_t w = ci[i0 + ii];
+      off = (int)(w & 0xFFFF);
+      x = (w >> 16) == keylab ? fmaf(s[ii], c, bk[off]) : -INFINITY;
+    }
+    const float P = ex2(x - st.x);
+    const float dS = P * (dp[ii] - st.y);
+    if (bins_on) red_add_s32(bn + off, round_to_int(dS * qs));
+    pv[ii] = P;
+    dv[ii] = dS * dscale;
+  }
+  uint32_t w[16];
+  split_pairs16(pv, w, w + 8);
+  __syncwarp();
+  tmem_st16u(st_col, w);
+  split_pairs16(dv, w, w + 8);
+  tmem_st16u(dpt_col, w);
+  st_shared_v4(op_hi, w[0], w[1], w[2], w[3]);
+  st_shared_v4(op_hi ^ 16u, w[4], w[5], w[6], w[7]);
+  st_shared_v4(op_lo, w[8], w[9], w[10], w[11]);
+  st_shared_v4(op_lo ^ 16u, w[12], w[13], w[14], w[15]);
+}
+
+// Rows of one accumulator (HD columns) to the grid tokens of `ri` (lane = row).
+template <int HD>
+__device__ inline void store_acc_rows(uint32_t taddr, const RowInfo& ri, bool ok,
+                                      __nv_bfloat16* out, int heads, int h) {
+  float o[HD];
+  tmem_load_cols<HD>(taddr, o);
+  tmem_wait_ld();
+  store_rows_bf16<HD>(o, 1.f, ri.stored && ok ? (const void*)(out + (ri.token * heads + h) * HD)
+                                               : nullptr);
+}
+
+template <int HD, int WW>
+__global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
+    wide_bwd_kernel(const __grid_constant__ FastParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  using C = WideBwdCfg<HD>;
+  constexpr int NS = C::kStages;
+  constexpr uint32_t tile_bytes = C::kTileBytes, RB = C::kRowBytes;
+  constexpr int kSoft = 2 * kWg;   // threads of the two softmax warpgroups
+  const Geo& g = p.g;
+  const int bp = p.bins_pad;
+  const WideBwdLayout L = wide_bwd_layout<HD>(bp);
+  uint8_t* tiles = smem + L.tiles;
+  float* bias = (float*)(smem + L.bias);
+  uint32_t* ci = (uint32_t*)(smem + L.colinfo);
+  float2* stats = (float2*)(smem + L.stats);
+  float* xch = (float*)(smem + L.xch);
+  int* bins = (int*)(smem + L.bins);
+  float* wbnd = (float*)(smem + L.wb);
+  int* wE = (int*)(smem + L.wb + 16);
+  int* wfin = wE + 2;
+  uint64_t* bars = (uint64_t*)(smem + L.bars);
+  uint64_t* full = bars;
+  uint64_t* empty = full + NS;
+  uint64_t* s1_full = empty + NS;
+  uint64_t* t1_empty = s1_full + 1;
+  uint64_t* s2_full = t1_empty + 1;
+  uint64_t* pds_full = s2_full + 1;
+  uint64_t* grad_done = pds_full + 1;
+  uint64_t* acc_free = grad_done + 1;
+  uint64_t* t_free = acc_free + 1;
+  uint64_t* bins_full = t_free + 1;    // [2]
+  uint64_t* bins_empty = bins_full + 2;
+  uint64_t* drain = bins_empty + 2;    // [1]
+  uint64_t* never = drain + 1;
+  uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
+  volatile int* abort = (volatile int*)(smem + L.misc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long n_local = local_tiles(p.n_tiles, blockIdx.x, gridDim.x);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(s1_full, 1);
+    mbar_init(t1_empty, kSoft);
+    mbar_init(s2_full, 1);
+    mbar_init(pds_full, kSoft);
+    mbar_init(grad_done, 1);
+    mbar_init(acc_free, kSoft);
+    mbar_init(t_free, kSoft);
+    for (int i = 0; i < 2; ++i) { mbar_init(&bins_full[i], kSoft); mbar_init(&bins_empty[i], 32); }
+    mbar_init(drain, 1);
+    mbar_init(never, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarp && lane == 0)
+    for (int tt = 0; tt < 4; ++tt)
+      for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
+  for (int i = threadIdx.x; i < 2 * bp; i += kWideBwdWarps * 32) bins[i] = 0;
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      long long k = 0;
+      for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
+        const int s = (int)(k % NS);
+        const uint32_t ph = (uint32_t)((k / NS) & 1);
+        if (!mbar_wait(&empty[s], ph ^ 1, abort, p.status, kWaitLimitNs)) break;
+        mbar_arrive_expect_tx(&full[s], 4 * tile_bytes + bp * 4);
+        issue_item_loads<HD, 4>(p, t, tiles + s * 4 * tile_bytes, bias + s * bp, &full[s]);
+      }
+      if (*abort) {
+        const long long first = k > NS ? k - NS : 0;
+        for (long long j = first; j < k; ++j)
+          mbar_drain(&full[j % NS], (uint32_t)((j / NS) & 1), kTestLimitNs * 100);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {   // every product, in dependency order
+      constexpr uint32_t id_s1 = idesc_bf16(kRows, kKeys, 0, 0);
+      constexpr uint32_t id_s2 = idesc_bf16(kRows, kRows, 0, 0);
+      constexpr uint32_t id_g = idesc_bf16(kRows, HD, 0, 1);   // dV, dK: A from TMEM
+      constexpr uint32_t id_q = idesc_bf16(kRows, HD, 1, 1);   // dQ: A MN-major in smem
+      const uint32_t op_hi = smem_u32(smem + L.dsop), op_lo = op_hi + 32768;
+      bool ok = true;
+      for (long long k = 0; k < n_local && ok; ++k) {
+        const int s = (int)(k % NS);
+        if (!mbar_wait(&full[s], (uint32_t)((k / NS) & 1), abort, p.status, kWaitLimitNs)) break;
+        const uint32_t q_s = smem_u32(tiles + (s * 4 + 0) * tile_bytes);
+        const uint32_t k_s = smem_u32(tiles + (s * 4 + 1) * tile_bytes);
+        const uint32_t v_s = smem_u32(tiles + (s * 4 + 2) * tile_bytes);
+        const uint32_t o_s = smem_u32(tiles + (s * 4 + 3) * tile_bytes);
+        // phase 1: S | dP of each query half
+        for (int qt = 0; qt < kHalves && ok; ++qt) {
+          ok = qt == 0 ? mbar_wait(t_free, (uint32_t)((k & 1) ^ 1), abort, p.status, kWaitLimitNs)
+                       : mbar_wait(t1_empty, 0, abort, p.status, kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk)
+            umma_ss(tmem, wdesc_kmajor<HD>(q_s + qt * kRows * RB, kk), wdesc_kmajor<HD>(k_s, kk),
+                    id_s1, kk);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk)
+            umma_ss(tmem + kColDP1, wdesc_kmajor<HD>(o_s + qt * kRows * RB, kk),
+                    wdesc_kmajor<HD>(v_s, kk), id_s1, kk);
+          umma_commit(s1_full);
+        }
+        if (!ok || !mbar_wait(t1_empty, 1, abort, p.status, kWaitLimitNs)) break;
+        // phase 2: blocks (kb, qt) = (0,0), (0,1), (1,0), (1,1)
+        for (int b = 0; b < 4 && ok; ++b) {
+          const int kb = b >> 1, qt = b & 1;
+          if (b > 0 && !(ok = mbar_wait(grad_done, (uint32_t)((b - 1) & 1), abort, p.status,
+                                        kWaitLimitNs)))
+            break;
+          tc_fence_after();
+          const uint32_t kq = k_s + kb * kRows * RB, vq = v_s + kb * kRows * RB;
+          const uint32_t qq = q_s + qt * kRows * RB, oq = o_s + qt * kRows * RB;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk)
+            umma_ss(tmem, wdesc_kmajor<HD>(kq, kk), wdesc_kmajor<HD>(qq, kk), id_s2, kk);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk)
+            umma_ss(tmem + kColDPT, wdesc_kmajor<HD>(vq, kk), wdesc_kmajor<HD>(oq, kk), id_s2, kk);
+          umma_commit(s2_full);
+          ok = mbar_wait(pds_full, (uint32_t)(b & 1), abort, p.status, kWaitLimitNs);
+          if (ok && b == 2) ok = mbar_wait(acc_free, (uint32_t)(k & 1), abort, p.status, kWaitLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk) {   // 16 queries per step
+            const uint32_t acc = (qt > 0 || kk > 0) ? 1u : 0u;
+            umma_ts(tmem + kColDV, tmem + 16 * kk, wdesc_mnmajor<HD>(oq, kk), id_g, acc);
+            umma_ts(tmem + kColDV, tmem + 16 * kk + 8, wdesc_mnmajor<HD>(oq, kk), id_g, 1);
+            umma_ts(tmem + kColDK, tmem + kColDPT + 16 * kk, wdesc_mnmajor<HD>(qq, kk), id_g, acc);
+            umma_ts(tmem + kColDK, tmem + kColDPT + 16 * kk + 8, wdesc_mnmajor<HD>(qq, kk), id_g, 1);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk) {   // 16 keys per step
+            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+            umma_ss(tmem + kColDQ + 64 * qt, desc_dsop(op_hi, kk), wdesc_mnmajor<HD>(kq, kk), id_q,
+                    acc);
+            umma_ss(tmem + kColDQ + 64 * qt, desc_dsop(op_lo, kk), wdesc_mnmajor<HD>(kq, kk), id_q,
+                    1);
+          }
+          umma_commit(grad_done);
+        }
+        if (ok) umma_commit(&empty[s]);
+      }
+      if (*abort) {
+        umma_commit(drain);
+        mbar_drain(drain, 0, kTestLimitNs * 100);
+      }
+    }
+  } else if (warp == kWideFoldWarp) {
+    // Each item's bins into the workspace's exact sums, in the window's unit.
+    for (long long k = 0, t = blockIdx.x; k < n_local; ++k, t += gridDim.x) {
+      const int par = (int)(k & 1);
+      if (!mbar_wait(&bins_full[par], (uint32_t)((k >> 1) & 1), abort, p.status, kWaitLimitNs))
+        break;
+      const int h = (int)(t - (t / g.heads) * g.heads);
+      int* bk = bins + par * bp;
+      const int E = wE[par];
+      const bool fin = wfin[par] != 0;
+      long long* acc = p.dt_acc + (size_t)h * bp * kLimbStride;
+      for (int i = lane; i < g.bins; i += 32) {
+        const int v = bk[i];
+        bk[i] = 0;
+        if (!fin) flag_nonfinite(acc + (size_t)i * kLimbStride);
+        else if (v != 0) add_fixed(acc + (size_t)i * kLimbStride, v, E);
+      }
+      __syncwarp();
+      mbar_arrive(&bins_empty[par]);
+    }
+  } else if (warp < 8) {
+    const int wg = warp >> 2;
+    const int r = threadIdx.x & (kWg - 1);
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tl = tmem + lane_base;
+    const float dscale = p.scale_log2 * (1.0f / kLog2e);   // head_dim^-1/2
+    const int C0 = (g.wh - 1) * (2 * g.ww - 1) + g.ww - 1;  // table offset of slot (0, 0)
+    const uint32_t op_base = smem_u32(smem + L.dsop);
+    for (long long k = 0; k < n_local; ++k) {
+      const long long t = blockIdx.x + k * (long long)gridDim.x;
+      const int s = (int)(k % NS), par = (int)(k & 1);
+      const long long win = t / g.heads;
+      const int h = (int)(t - win * g.heads);
+      const bool plain = WW > 0 && window_plain(g, win);
+      // this thread's slots r and 128 + r (query rows of phase 1 and the dQ
+      // epilogue, key rows of phase 2)
+      RowInfo ri[2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+        ri[x] = plain ? plain_row_info<(WW > 0 ? WW : 16)>(g, win, x * kRows + r)
+                      : row_info(g, win, x * kRows + r);
+      ci[wg * kRows + r] = key_word(ri[wg]);
+      if (named_sync_or(1, kSoft, *abort)) break;
+      if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
+      mbar_wait(&full[s], (uint32_t)((k / NS) & 1), abort, p.status, kWaitLimitNs);
+      const float* brow = bias + s * bp;
+      // ---- phase 1 ----
+      float bmax = 0.f;
+      for (int qt = 0; qt < kHalves; ++qt) {
+        const RowInfo& qi = ri[qt];
+        mbar_wait(s1_full, (uint32_t)qt, abort, p.status, kWaitLimitNs);
+        tc_fence_after();
+        float M, l, d, a;
+        const uint32_t sc = tl + wg * kRows, dc = tl + kColDP1 + wg * kRows;
+        if (WW > 0 && plain)
+          wide_row_stats<true, (WW > 0 ? WW : 16)>(sc, dc, wg * kRows, brow, ci, qi.bias_base,
+                                                   qi.label, p.scale_log2, M, l, d, a);
+        else
+          wide_row_stats<false, 16>(sc, dc, wg * kRows, brow, ci, qi.bias_base, qi.label,
+                                    p.scale_log2, M, l, d, a);
+        tc_fence_before();
+        mbar_arrive(t1_empty);
+        float* xq = xch + qt * 4 * kRows;
+        if (wg == 1) {
+          xq[r] = M;
+          xq[kRows + r] = l;
+          xq[2 * kRows + r] = d;
+          xq[3 * kRows + r] = a;
+        }
+        named_sync(1, kSoft);
+        if (wg == 0) {
+          const float M1 = xq[r], l1 = xq[kRows + r], d1 = xq[2 * kRows + r], a1 = xq[3 * kRows + r];
+          const float Mx = fmaxf(M, M1);
+          const float f0 = ex2(M - Mx), f1 = ex2(M1 - Mx);
+          const float lt = l * f0 + l1 * f1, dt = d * f0 + d1 * f1;
+          float2 st = make_float2(INFINITY, 0.f);   // not a real token: P = 0
+          if (qi.valid) {
+            const float inv = 1.f / lt;
+            st = make_float2(Mx + __log2f(lt), dt * inv);
+            // |dS_ij| <= max_j P_ij (max_j |dP_ij| + |D|), max_j P_ij = 1 / l;
+            // a NaN becomes +inf here, since fmaxf would drop it
+            float rb = inv * (fmaxf(a, a1) + fabsf(st.y));
+            if (!(rb <= 3.0e38f)) rb = INFINITY;
+            bmax = fmaxf(bmax, rb);
+          }
+          stats[qt * kRows + r] = st;
+        }
+      }
+      if (wg == 0) {
+        const float wb = warp_max(bmax);
+        if (lane == 0) wbnd[warp] = wb;
+      }
+      named_sync(1, kSoft);   // stats and bounds of the whole window are in
+      const float win_bound = fmaxf(fmaxf(wbnd[0], wbnd[1]), fmaxf(wbnd[2], wbnd[3]));
+      const bool finite = win_bound <= 3.0e38f;   // false for NaN and infinity
+      const int E = tile_exponent(finite ? win_bound : 0.f);
+      const float qs = exp2_int(E);
+      if (k >= 2)   // this parity's bins (and unit) were folded (item k - 2)
+        mbar_wait(&bins_empty[par], (uint32_t)(((k >> 1) - 1) & 1), abort, p.status, kWaitLimitNs);
+      if (threadIdx.x == 0) {
+        wE[par] = E;
+        wfin[par] = finite ? 1 : 0;
+      }
+      int* bins_k = bins + par * bp;
+      // ---- phase 2 ----
+      for (int b = 0; b < 4; ++b) {
+        const int kb = b >> 1, qt = b & 1;
+        const RowInfo& kj = ri[kb];
+        const float* bk = brow + C0 - kj.key_off;
+        int* bn = bins_k + C0 - kj.key_off;
+        const uint32_t keylab = kj.valid ? (uint32_t)kj.label : 14u;   // pad key: no query matches
+        const bool bins_on = finite && kj.valid;
+        mbar_wait(s2_full, (uint32_t)(b & 1), abort, p.status, kWaitLimitNs);
+        // the dQ operand is free once the previous block's products are done
+        if (b > 0) mbar_wait(grad_done, (uint32_t)((b - 1) & 1), abort, p.status, kWaitLimitNs);
+        tc_fence_after();
+        const int jr = r & 63;
+        const uint32_t op_row = op_base + ((r >> 6) * 2 + wg) * 8192 + jr * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          const int kk = wg * 4 + c;
+          const int i0 = qt * kRows + 16 * kk;
+          const uint32_t op_hi = op_row + (((2 * c) ^ (jr & 7)) << 4);
+          // (the second 16-byte chunk is at ((2c + 1) ^ (jr & 7)) << 4 = this ^ 16)
+          if (WW > 0 && plain)
+            wide_grad_chunk<true, (WW > 0 ? WW : 16)>(tl + 16 * kk, tl + kColDPT + 16 * kk, i0,
+                                                     stats, ci, bk, bn, keylab, bins_on,
+                                                     p.scale_log2, qs, dscale, op_hi,
+                                                     op_hi + 32768);
+          else
+            wide_grad_chunk<false, 16>(tl + 16 * kk, tl + kColDPT + 16 * kk, i0, stats, ci, bk,
+                                       bn, keylab, bins_on, p.scale_log2, qs, dscale, op_hi,
+                                       op_hi + 32768);
+        }
+        tmem_wait_st();
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(pds_full);
+        if (b == 1 || b == 3) {   // dV, dK of key half kb (and dQ after the last block)
+          mbar_wait(grad_done, (uint32_t)(b & 1), abort, p.status, kWaitLimitNs);
+          tc_fence_after();
+          const bool ok = !*abort;
+          if (b == 3) {
+            const RowInfo& qr = ri[wg];   // dQ rows: query slot 128 wg + r
+            store_acc_rows<HD>(tl + kColDQ + 64 * wg, qr, ok, (__nv_bfloat16*)p.out0, g.heads, h);
+          }
+          if (wg == 0)
+            store_acc_rows<HD>(tl + kColDV, kj, ok, (__nv_bfloat16*)p.out2, g.heads, h);
+          else
+            store_acc_rows<HD>(tl + kColDK, kj, ok, (__nv_bfloat16*)p.out1, g.heads, h);
+          tc_fence_before();
+          mbar_arrive(b == 1 ? acc_free : t_free);
+        }
+      }
+      mbar_arrive(&bins_full[par]);   // the fold warp adds them to the global sums
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int HD>
+size_t wide_bwd_smem(const Geo& g) {
+  return wide_bwd_layout<HD>(bins_padded(g.bins)).total + 1024;
+}
+
 template <int HD>
 size_t wide_fwd_smem(const Geo& g) {
   return wide_fwd_layout<HD>(bins_padded(g.bins)).total + 1024;
@@ -411,8 +925,9 @@ bool wide_supported(const Geo& g, int dtype) {
       if ((ylen[a] * xlen[c]) % 8) return false;
     }
   if (g.bins > 0xFFFF) return false;
-  const size_t sm = g.hd == 64 ? wide_fwd_smem<64>(g) : wide_fwd_smem<32>(g);
-  return sm <= kSmemLimit;
+  const size_t f = g.hd == 64 ? wide_fwd_smem<64>(g) : wide_fwd_smem<32>(g);
+  const size_t b = g.hd == 64 ? wide_bwd_smem<64>(g) : wide_bwd_smem<32>(g);
+  return f <= kSmemLimit && b <= kSmemLimit;
 }
 
 cudaError_t wide_forward(const Geo& g, const void* q, const void* k, const void* v,
@@ -436,6 +951,38 @@ cudaError_t wide_forward(const Geo& g, const void* q, const void* k, const void*
   const size_t smem = wide_fwd_smem<32>(g);
   return w16 ? wide_launch(wide_fwd_kernel<32, 16>, p, smem, kWideThreads, st)
              : wide_launch(wide_fwd_kernel<32, 0>, p, smem, kWideThreads, st);
+}
+
+cudaError_t wide_backward(const Geo& g, const void* q, const void* k, const void* v,
+                          const float* table, const void* dout, void* dq, void* dk, void* dv,
+                          float* dtable, void* ws, int flags, cudaStream_t st) {
+  float* bias_t = (float*)((char*)ws + kWsHeader);
+  long long* dt_acc = (long long*)((char*)ws + dbias_fixed_offset(g));
+  static thread_local FastParams p;
+  fill_wide(p, g, bias_t, (int*)ws, flags);
+  p.out0 = dq;
+  p.out1 = dk;
+  p.out2 = dv;
+  p.dt_acc = dt_acc;
+  if (!encode_maps(p, 0, q) || !encode_maps(p, 1, k) || !encode_maps(p, 2, v) ||
+      !encode_maps(p, 3, dout))
+    return cudaErrorInvalidValue;
+  cudaError_t e = prep_bias(g, table, bias_t, dt_acc, st);
+  if (e != cudaSuccess) return e;
+  const bool w16 = g.wh == 16 && g.ww == 16;
+  constexpr int thr = kWideBwdWarps * 32;
+  if (g.hd == 64) {
+    const size_t smem = wide_bwd_smem<64>(g);
+    e = w16 ? wide_launch(wide_bwd_kernel<64, 16>, p, smem, thr, st)
+            : wide_launch(wide_bwd_kernel<64, 0>, p, smem, thr, st);
+  } else {
+    const size_t smem = wide_bwd_smem<32>(g);
+    e = w16 ? wide_launch(wide_bwd_kernel<32, 16>, p, smem, thr, st)
+            : wide_launch(wide_bwd_kernel<32, 0>, p, smem, thr, st);
+  }
+  if (e != cudaSuccess) return e;
+  if (flags & SWIN_FLAG_DBIAS_SUMS) return cudaSuccess;   // the caller finishes the sums
+  return finish_dbias(g, dt_acc, dtable, st);
 }
 
 }  // namespace swin
