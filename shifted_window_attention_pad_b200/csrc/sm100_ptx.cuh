@@ -328,6 +328,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ void red_add_s32(void* p, int v) {
   asm volatile("red.shared.add.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
 }
+// The same without a compiler memory barrier, so loads of later terms can be
+// scheduled ahead of it; the caller orders the bins' readers with an mbarrier
+// arrive (which is one).
+__device__ __forceinline__ void red_add_s32_relaxed(const int* p, int v) {
+  asm volatile("red.shared.add.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v));
+}
 
 // Fire-and-forget 64-bit integer add to global memory (two's complement, so
 // signed values add correctly).

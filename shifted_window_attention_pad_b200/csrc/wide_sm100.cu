@@ -388,21 +388,31 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 //  Phase 2, gradients, key-major: for each block of 128 keys (kb) x 128
 //    queries (qt), S^T = K_kb Q_qt^T and dP^T = V_kb dO_qt^T (M = keys, so a
 //    thread holds one key and walks queries); P = 2^(x - L_i) and
-//    dS = P (dP - D_i) go back into their own columns as bf16 hi + lo pairs
-//    (the A operands, from TMEM, of dV_kb += P^T dO_qt and
-//    dK_kb += dS^T Q_qt), scale * dS also into shared memory as the MN-major
-//    A operand of dQ_qt += dS K_kb, and dS into the bias-gradient bins.
+//    dS = P (dP - D_i): P goes back into its S^T columns as bf16 hi + lo
+//    pairs (the A operand, from TMEM, of dV_kb += P^T dO_qt), dS as hi + lo
+//    into shared memory (the A operand of both dK_kb += dS^T Q_qt and
+//    dQ_qt += dS K_kb) and into the bias-gradient bins. The scale
+//    head_dim^-1/2 of dQ and dK is applied to their fp32 sums at the end.
 //    Warpgroup w takes queries 64 w .. 64 w + 63 of the block.
+//    The products overlap the row work: once a block's rows are done, dP^T of
+//    the next block goes into the dP^T columns (read already), dV of this
+//    block runs, then S^T of the next block replaces P, and dK and dQ of this
+//    block run while the next block's rows are worked on (its first write of
+//    dS waits for them).
 // TMEM: phase 1 S | dP at 0 | 256; phase 2 S^T | dP^T at 0 | 128, dV_kb at
-// 256, dK_kb at 320, dQ_0 at 384, dQ_1 at 448. dV and dK of a key half leave
-// after its two blocks, dQ after the last block.
+// 256, dK_kb at 320, dQ_0 at 384, dQ_1 at 448. dV and dK of key half 0 leave
+// after the third block's rows, the rest after the last block.
 template <int HD>
 struct WideBwdCfg {
   static constexpr uint32_t kRowBytes = HD * 2;
   static constexpr uint32_t kTileBytes = kKeys * kRowBytes;
-  static constexpr int kStages = HD > 32 ? 1 : 2;
+  static constexpr int kStages = 1;
   static constexpr uint32_t kOpBytes = 2 * 32768;   // scale * dS, hi and lo
 };
+// The bias row of the head in four copies, copy m shifted down by m floats,
+// so that any 16 consecutive entries are four aligned 16-byte loads from one
+// of them. Row stride in floats:
+__host__ __device__ inline int bias_copy_stride(int bins_pad) { return bins_pad + 4; }
 constexpr uint32_t kColDP1 = 256;                    // phase 1 dP (S at 0)
 constexpr uint32_t kColDPT = 128;                    // phase 2 dP^T (S^T at 0)
 constexpr uint32_t kColDV = 256, kColDK = 320, kColDQ = 384;
@@ -419,11 +429,12 @@ __host__ __device__ inline WideBwdLayout wide_bwd_layout(int bins_pad) {
   WideBwdLayout L;
   L.tiles = 0;
   L.dsop = L.tiles + C::kStages * 4 * C::kTileBytes;
+  L.xch = L.dsop;                            // [qt][4][128] partial statistics (phase 1
+                                             // only: the dQ operand is free then)
   L.bias = L.dsop + C::kOpBytes;
-  L.colinfo = L.bias + ((C::kStages * bins_pad * 4 + 15) & ~15);
+  L.colinfo = L.bias + C::kStages * 4 * bias_copy_stride(bins_pad) * 4;
   L.stats = L.colinfo + kKeys * 4;           // float2 {L, D} per query
-  L.xch = L.stats + kKeys * 8;               // [qt][4][128] partial statistics
-  L.bins = L.xch + 2 * 4 * kRows * 4;        // [2][bins_pad] int32 (item parity)
+  L.bins = L.stats + kKeys * 8;              // [2][bins_pad] int32 (item parity)
   L.wb = L.bins + 2 * bins_pad * 4;          // [4] warp bounds, [2] E, [2] finite
   L.bars = (L.wb + 64 + 7) & ~7u;
   L.misc = L.bars + 8 * 32;
@@ -431,27 +442,39 @@ __host__ __device__ inline WideBwdLayout wide_bwd_layout(int bins_pad) {
   return L;
 }
 
-// Scale * dS operand of dQ_qt += dS K_kb (M = 128 queries, K = 128 keys),
-// MN-major with 128-byte swizzle: 8 KB regions of 64 keys x 64 queries at
-// (key half * 2 + query half) * 8 KB, K step k16 = 16 keys.
-__device__ inline uint64_t desc_dsop(uint32_t base, int k16) {
-  return smem_desc(base + (k16 >> 2) * 16384 + (k16 & 3) * 2048, 8192, 1024, kSwizzle128);
+// dS of a block in shared memory, hi and lo: rows = keys, 128-byte rows of 64
+// queries, 128-byte swizzle, 8 KB regions of 64 keys x 64 queries at
+// (query half * 2 + key half) * 8 KB. The same bytes are two operands:
+// the MN-major A of dQ_qt += dS K_kb (M = queries, K = keys; K step k16 = 16
+// keys, the second 64-query atom 16 KB on) and the K-major A of
+// dK_kb += dS^T Q_qt (M = keys, K = queries; K step k16 = 16 queries, the 128
+// key rows evenly 1 KB per 8).
+__device__ inline uint64_t desc_ds_mn(uint32_t base, int k16) {
+  return smem_desc(base + (k16 >> 2) * 8192 + (k16 & 3) * 2048, 16384, 1024, kSwizzle128);
+}
+__device__ inline uint64_t desc_ds_k(uint32_t base, int k16) {
+  return smem_desc(base + (k16 >> 2) * 16384 + (k16 & 3) * 32, 16, 1024, kSwizzle128);
 }
 
-// hi / lo bf16 pairs of 16 values: hw[c] = (hi(v[2c]), hi(v[2c+1])), hi = v
-// with the low 16 bits cleared; lw[c] the bf16 of the remainders.
-__device__ inline void split_pairs16(const float* v, uint32_t* hw, uint32_t* lw) {
+// Logits of 16 keys k0.. of a plain WW x WW window (k0 a multiple of WW, or
+// of 16 inside a window row), as chunk_logits_plain.
+template <int WW>
+__device__ inline float chunk16_logits_plain(float* x, const float* bias_q, int k0, float c) {
+  bias_q -= (k0 / WW) * (2 * WW - 1) + k0 % WW;
+  float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const uint32_t a = __float_as_uint(v[2 * c]) & 0xFFFF0000u;
-    const uint32_t b = __float_as_uint(v[2 * c + 1]) & 0xFFFF0000u;
-    hw[c] = __byte_perm(a, b, 0x7632);
-    lw[c] = pack_bf16(v[2 * c] - __uint_as_float(a), v[2 * c + 1] - __uint_as_float(b));
+  for (int j = 0; j < 16; j += 2) {
+    x[j] = fmaf(x[j], c, bias_q[-plain_off<WW>(j)]);
+    x[j + 1] = fmaf(x[j + 1], c, bias_q[-plain_off<WW>(j + 1)]);
+    m0 = fmaxf(m0, x[j]);
+    m1 = fmaxf(m1, x[j + 1]);
   }
+  return fmaxf(m0, m1);
 }
 
 // Phase 1 over 128 keys of one row (columns s_col.. of S and dp_col.. of dP,
-// keys k0base..): online maximum M, l, d and max |dP|.
+// keys k0base..), 16 at a time with the next chunk's TMEM loads in flight:
+// online maximum M, l = sum 2^(x - M), d = sum 2^(x - M) dP, a = max |dP|.
 template <bool PLAIN, int WW>
 __device__ inline void wide_row_stats(uint32_t s_col, uint32_t dp_col, int k0base,
                                       const float* brow, const uint32_t* ci, int bias_base,
@@ -461,19 +484,13 @@ __device__ inline void wide_row_stats(uint32_t s_col, uint32_t dp_col, int k0bas
   l = 0.f;
   d = 0.f;
   a = 0.f;
-#pragma unroll 1
-  for (int kc = 0; kc < kRows; kc += 32) {
-    float x[32], dp[32];
-    __syncwarp();
-    tmem_ld32(s_col + kc, x);
-    tmem_ld32(dp_col + kc, dp);
-    tmem_wait_ld();
+  auto work = [&](float* x, int kc) {   // x: 16 of S, then 16 of dP
     const int k0 = k0base + kc;
     float cm;
     if constexpr (PLAIN)
-      cm = chunk_logits_plain<WW>(x, brow + bias_base, k0, c);
+      cm = chunk16_logits_plain<WW>(x, brow + bias_base, k0, c);
     else
-      cm = logits_general<32>(x, brow, ci + k0, bias_base, label, c);
+      cm = logits_general<16>(x, brow, ci + k0, bias_base, label, c);
     if (cm > M) {   // rescale the sums to the new maximum
       const float f = ex2(M - cm);
       l *= f;
@@ -483,77 +500,152 @@ __device__ inline void wide_row_stats(uint32_t s_col, uint32_t dp_col, int k0bas
     const float Mz = M == -INFINITY ? 0.f : M;   // a chunk of masked keys adds zeros
     float l0 = 0.f, l1 = 0.f, d0 = 0.f, d1 = 0.f, a0 = 0.f, a1 = 0.f;
 #pragma unroll
-    for (int j = 0; j < 32; j += 2) {
+    for (int j = 0; j < 16; j += 2) {
       const float e0 = ex2(x[j] - Mz), e1 = ex2(x[j + 1] - Mz);
       l0 += e0;
       l1 += e1;
-      d0 = fmaf(e0, dp[j], d0);
-      d1 = fmaf(e1, dp[j + 1], d1);
-      a0 = fmaxf(a0, fabsf(dp[j]));
-      a1 = fmaxf(a1, fabsf(dp[j + 1]));
+      d0 = fmaf(e0, x[16 + j], d0);
+      d1 = fmaf(e1, x[17 + j], d1);
+      a0 = fmaxf(a0, fabsf(x[16 + j]));
+      a1 = fmaxf(a1, fabsf(x[17 + j]));
     }
     l += l0 + l1;
     d += d0 + d1;
     a = fmaxf(a, fmaxf(a0, a1));
+  };
+  float xa[32], xb[32];
+  __syncwarp();
+  tmem_ld16(s_col, xa);
+  tmem_ld16(dp_col, xa + 16);
+#pragma unroll 1
+  for (int kc = 0; kc < kRows; kc += 32) {
+    tmem_wait_ld_regs(xa);
+    __syncwarp();
+    tmem_ld16(s_col + kc + 16, xb);
+    tmem_ld16(dp_col + kc + 16, xb + 16);
+    work(xa, kc);
+    tmem_wait_ld_regs(xb);
+    if (kc + 32 < kRows) {
+      __syncwarp();
+      tmem_ld16(s_col + kc + 32, xa);
+      tmem_ld16(dp_col + kc + 32, xa + 16);
+    }
+    work(xb, kc + 16);
   }
 }
 
-// Phase 2, one chunk of 16 queries (i0 .. i0 + 15) of this thread's key: P
-// and dS from S^T and dP^T, their hi / lo pairs back to TMEM, scale * dS to the
-// dQ operand in shared memory, dS to the bias-gradient bins.
-template <bool PLAIN, int WW>
-__device__ inline void wide_grad_chunk(uint32_t st_col, uint32_t dpt_col, int i0,
-                                       const float2* stats, const uint32_t* ci,
-                                       const float* bk, int* bn, uint32_t keylab, bool bins_on,
-                                       float c, float qs, float dscale, uint32_t op_hi,
-                                       uint32_t op_lo) {
-  float s[16], dp[16];
-  __syncwarp();
-  tmem_ld16(st_col, s);
-  tmem_ld16(dpt_col, dp);
-  tmem_wait_ld();
-  float pv[16], dv[16];
-  const int ib = PLAIN ? plain_off<WW>(i0) : 0;   // i0 starts a window row
-#pragma unroll
-  for (int ii = 0; ii < 16; ++ii) {
-    const float2 st = stats[i0 + ii];
-    float x;
-    int off;
+// Phase 2, this thread's key over the 64 queries of its warpgroup in one
+// block, in chunks of 16 (i0 = first query of the chunk): P and dS from S^T
+// and dP^T, P's hi / lo pairs back into its S^T columns, dS's into the
+// shared-memory operand (after `op_free`, when given), dS to the
+// bias-gradient bins. The TMEM load
+// of chunk c + 1 is in flight while chunk c is worked on. Bias and bins of
+// pair (i, j) sit at kbase + off(i), kbase = C0 - off(j). Plain 16 x 16
+// windows: a chunk is one window row of queries, so its 16 table entries are
+// consecutive and come as four 16-byte loads from the shifted bias copies.
+template <bool PLAIN>
+__device__ inline void wide_grad_block(uint32_t col0, int ib0, const float4* stats4,
+                                       const uint32_t* ci, const float* bias4, int bstride,
+                                       int kbase, int* bins, uint32_t keylab, bool bins_on,
+                                       float c, float qs, uint32_t op_row, int jr,
+                                       uint64_t* op_free, uint32_t op_phase, volatile int* abort,
+                                       int* status) {
+  float xa[32], xb[32];   // [0, 16) S^T, [16, 32) dP^T of one chunk
+  auto work = [&](float* x, int cc) {
+    const int i0 = ib0 + 16 * cc;
+    int base = 0, m = 0;
     if constexpr (PLAIN) {
-      off = ib + plain_off<WW>(ii);
-      x = fmaf(s[ii], c, bk[off]);
-    } else {
-      const uint32_t w = ci[i0 + ii];
-      off = (int)(w & 0xFFFF);
-      x = (w >> 16) == keylab ? fmaf(s[ii], c, bk[off]) : -INFINITY;
+      base = kbase + plain_off<16>(i0);
+      m = base & 3;
     }
-    const float P = ex2(x - st.x);
-    const float dS = P * (dp[ii] - st.y);
-    if (bins_on) red_add_s32(bn + off, round_to_int(dS * qs));
-    pv[ii] = P;
-    dv[ii] = dS * dscale;
-  }
-  uint32_t w[16];
-  split_pairs16(pv, w, w + 8);
+    const float4* bp = reinterpret_cast<const float4*>(bias4 + m * bstride + (base - m));
+    uint32_t pw[16], sw[16];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {   // 4 queries: one 16-byte bias load (plain windows)
+      float b4[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (PLAIN) {
+        const float4 v = bp[q4];
+        b4[0] = v.x;
+        b4[1] = v.y;
+        b4[2] = v.z;
+        b4[3] = v.w;
+      }
+#pragma unroll
+      for (int u2 = 0; u2 < 2; ++u2) {
+        const int u = 2 * q4 + u2;
+        const float4 st = stats4[(i0 >> 1) + u];   // (L, D) of queries i0 + 2u, i0 + 2u + 1
+        float P[2], dS[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int ii = 2 * u + e;
+          float x0;
+          int idx;
+          if constexpr (PLAIN) {
+            idx = base + ii;
+            x0 = fmaf(x[ii], c, b4[2 * u2 + e]);
+          } else {
+            const uint32_t w = ci[i0 + ii];
+            idx = kbase + (int)(w & 0xFFFF);
+            x0 = (w >> 16) == keylab ? fmaf(x[ii], c, bias4[idx]) : -INFINITY;
+          }
+          const float Li = e ? st.z : st.x, Di = e ? st.w : st.y;
+          P[e] = ex2(x0 - Li);
+          dS[e] = P[e] * (x[16 + ii] - Di);
+          if (bins_on) red_add_s32_relaxed(bins + idx, round_to_int(dS[e] * qs));
+        }
+        {
+          const uint32_t a = __float_as_uint(P[0]) & 0xFFFF0000u;
+          const uint32_t bb = __float_as_uint(P[1]) & 0xFFFF0000u;
+          pw[u] = __byte_perm(a, bb, 0x7632);
+          pw[8 + u] = pack_bf16(P[0] - __uint_as_float(a), P[1] - __uint_as_float(bb));
+        }
+        {
+          const uint32_t a = __float_as_uint(dS[0]) & 0xFFFF0000u;
+          const uint32_t bb = __float_as_uint(dS[1]) & 0xFFFF0000u;
+          sw[u] = __byte_perm(a, bb, 0x7632);
+          sw[8 + u] = pack_bf16(dS[0] - __uint_as_float(a), dS[1] - __uint_as_float(bb));
+        }
+      }
+    }
+    const uint32_t col = col0 + 16 * cc;
+    __syncwarp();
+    tmem_st16u(col, pw);
+    // the dS operand is free once the previous block's dK and dQ are done
+    if (cc == 0 && op_free) mbar_wait(op_free, op_phase, abort, status, kWaitLimitNs);
+    const uint32_t op_hi = op_row + (((2 * cc) ^ (jr & 7)) << 4);   // second chunk: ^ 16
+    st_shared_v4(op_hi, sw[0], sw[1], sw[2], sw[3]);
+    st_shared_v4(op_hi ^ 16u, sw[4], sw[5], sw[6], sw[7]);
+    st_shared_v4(op_hi + 32768, sw[8], sw[9], sw[10], sw[11]);
+    st_shared_v4((op_hi + 32768) ^ 16u, sw[12], sw[13], sw[14], sw[15]);
+  };
   __syncwarp();
-  tmem_st16u(st_col, w);
-  split_pairs16(dv, w, w + 8);
-  tmem_st16u(dpt_col, w);
-  st_shared_v4(op_hi, w[0], w[1], w[2], w[3]);
-  st_shared_v4(op_hi ^ 16u, w[4], w[5], w[6], w[7]);
-  st_shared_v4(op_lo, w[8], w[9], w[10], w[11]);
-  st_shared_v4(op_lo ^ 16u, w[12], w[13], w[14], w[15]);
+  tmem_ld16(col0, xa);
+  tmem_ld16(col0 + kColDPT, xa + 16);
+#pragma unroll
+  for (int cc = 0; cc < 4; cc += 2) {
+    tmem_wait_ld_regs(xa);
+    __syncwarp();
+    tmem_ld16(col0 + 16 * (cc + 1), xb);
+    tmem_ld16(col0 + kColDPT + 16 * (cc + 1), xb + 16);
+    work(xa, cc);
+    tmem_wait_ld_regs(xb);
+    if (cc + 2 < 4) {
+      __syncwarp();
+      tmem_ld16(col0 + 16 * (cc + 2), xa);
+      tmem_ld16(col0 + kColDPT + 16 * (cc + 2), xa + 16);
+    }
+    work(xb, cc + 1);
+  }
 }
 
 // Rows of one accumulator (HD columns) to the grid tokens of `ri` (lane = row).
 template <int HD>
-__device__ inline void store_acc_rows(uint32_t taddr, const RowInfo& ri, bool ok,
-                                      __nv_bfloat16* out, int heads, int h) {
+__device__ inline void store_acc_rows(uint32_t taddr, bool stored, long long token,
+                                      __nv_bfloat16* out, int heads, int h, float mul) {
   float o[HD];
   tmem_load_cols<HD>(taddr, o);
   tmem_wait_ld();
-  store_rows_bf16<HD>(o, 1.f, ri.stored && ok ? (const void*)(out + (ri.token * heads + h) * HD)
-                                               : nullptr);
+  store_rows_bf16<HD>(o, mul, stored ? (const void*)(out + (token * heads + h) * HD) : nullptr);
 }
 
 template <int HD, int WW>
@@ -585,7 +677,8 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
   uint64_t* s2_full = t1_empty + 1;
   uint64_t* pds_full = s2_full + 1;
   uint64_t* grad_done = pds_full + 1;
-  uint64_t* acc_free = grad_done + 1;
+  uint64_t* gv_done = grad_done + 1;
+  uint64_t* acc_free = gv_done + 1;
   uint64_t* t_free = acc_free + 1;
   uint64_t* bins_full = t_free + 1;    // [2]
   uint64_t* bins_empty = bins_full + 2;
@@ -603,6 +696,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
     mbar_init(s2_full, 1);
     mbar_init(pds_full, kSoft);
     mbar_init(grad_done, 1);
+    mbar_init(gv_done, 1);
     mbar_init(acc_free, kSoft);
     mbar_init(t_free, kSoft);
     for (int i = 0; i < 2; ++i) { mbar_init(&bins_full[i], kSoft); mbar_init(&bins_empty[i], 32); }
@@ -632,7 +726,8 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
         const uint32_t ph = (uint32_t)((k / NS) & 1);
         if (!mbar_wait(&empty[s], ph ^ 1, abort, p.status, kWaitLimitNs)) break;
         mbar_arrive_expect_tx(&full[s], 4 * tile_bytes + bp * 4);
-        issue_item_loads<HD, 4>(p, t, tiles + s * 4 * tile_bytes, bias + s * bp, &full[s]);
+        issue_item_loads<HD, 4>(p, t, tiles + s * 4 * tile_bytes,
+                                bias + s * 4 * bias_copy_stride(bp), &full[s]);
       }
       if (*abort) {
         const long long first = k > NS ? k - NS : 0;
@@ -673,39 +768,59 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
         }
         if (!ok || !mbar_wait(t1_empty, 1, abort, p.status, kWaitLimitNs)) break;
         // phase 2: blocks (kb, qt) = (0,0), (0,1), (1,0), (1,1)
-        for (int b = 0; b < 4 && ok; ++b) {
-          const int kb = b >> 1, qt = b & 1;
-          if (b > 0 && !(ok = mbar_wait(grad_done, (uint32_t)((b - 1) & 1), abort, p.status,
-                                        kWaitLimitNs)))
-            break;
-          tc_fence_after();
-          const uint32_t kq = k_s + kb * kRows * RB, vq = v_s + kb * kRows * RB;
-          const uint32_t qq = q_s + qt * kRows * RB, oq = o_s + qt * kRows * RB;
+        auto issue_st = [&](int b) {   // S^T of block b into columns 0-127
+          const uint32_t kq = k_s + (b >> 1) * kRows * RB, qq = q_s + (b & 1) * kRows * RB;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk)
             umma_ss(tmem, wdesc_kmajor<HD>(kq, kk), wdesc_kmajor<HD>(qq, kk), id_s2, kk);
+        };
+        auto issue_dpt = [&](int b) {   // dP^T of block b into columns 128-255
+          const uint32_t vq = v_s + (b >> 1) * kRows * RB, oq = o_s + (b & 1) * kRows * RB;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk)
             umma_ss(tmem + kColDPT, wdesc_kmajor<HD>(vq, kk), wdesc_kmajor<HD>(oq, kk), id_s2, kk);
-          umma_commit(s2_full);
-          ok = mbar_wait(pds_full, (uint32_t)(b & 1), abort, p.status, kWaitLimitNs);
-          if (ok && b == 2) ok = mbar_wait(acc_free, (uint32_t)(k & 1), abort, p.status, kWaitLimitNs);
-          if (!ok) break;
+        };
+        tc_fence_after();
+        issue_st(0);
+        issue_dpt(0);
+        umma_commit(s2_full);
+        for (int b = 0; b < 4 && ok; ++b) {
+          const int kb = b >> 1, qt = b & 1;
+          const uint32_t kq = k_s + kb * kRows * RB;
+          const uint32_t qq = q_s + qt * kRows * RB, oq = o_s + qt * kRows * RB;
+          if (!(ok = mbar_wait(pds_full, (uint32_t)(b & 1), abort, p.status, kWaitLimitNs))) break;
+          tc_fence_after();
+          if (b < 3) issue_dpt(b + 1);   // its columns were read by the rows of block b
+          // dV_1 and dK_1 start over the columns of dV_0 and dK_0: wait for their rows
+          if (b == 2 && !(ok = mbar_wait(acc_free, (uint32_t)(k & 1), abort, p.status,
+                                         kWaitLimitNs)))
+            break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk) {   // 16 queries per step
+          for (int kk = 0; kk < kRows / 16; ++kk) {   // dV += P^T dO, 16 queries per step
             const uint32_t acc = (qt > 0 || kk > 0) ? 1u : 0u;
             umma_ts(tmem + kColDV, tmem + 16 * kk, wdesc_mnmajor<HD>(oq, kk), id_g, acc);
             umma_ts(tmem + kColDV, tmem + 16 * kk + 8, wdesc_mnmajor<HD>(oq, kk), id_g, 1);
-            umma_ts(tmem + kColDK, tmem + kColDPT + 16 * kk, wdesc_mnmajor<HD>(qq, kk), id_g, acc);
-            umma_ts(tmem + kColDK, tmem + kColDPT + 16 * kk + 8, wdesc_mnmajor<HD>(qq, kk), id_g, 1);
+          }
+          umma_commit(gv_done);
+          if (b < 3) {   // S^T of the next block over P, once dV has read it
+            if (!(ok = mbar_wait(gv_done, (uint32_t)(b & 1), abort, p.status, kWaitLimitNs))) break;
+            tc_fence_after();
+            issue_st(b + 1);
+            umma_commit(s2_full);
           }
 #pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk) {   // 16 keys per step
+          for (int kk = 0; kk < kRows / 16; ++kk) {   // dK += dS^T Q, 16 queries per step
+            const uint32_t acc = (qt > 0 || kk > 0) ? 1u : 0u;
+            umma_ss(tmem + kColDK, desc_ds_k(op_hi, kk), wdesc_mnmajor<HD>(qq, kk), id_g, acc);
+            umma_ss(tmem + kColDK, desc_ds_k(op_lo, kk), wdesc_mnmajor<HD>(qq, kk), id_g, 1);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk) {   // dQ += dS K, 16 keys per step
             const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-            umma_ss(tmem + kColDQ + 64 * qt, desc_dsop(op_hi, kk), wdesc_mnmajor<HD>(kq, kk), id_q,
+            umma_ss(tmem + kColDQ + 64 * qt, desc_ds_mn(op_hi, kk), wdesc_mnmajor<HD>(kq, kk), id_q,
                     acc);
-            umma_ss(tmem + kColDQ + 64 * qt, desc_dsop(op_lo, kk), wdesc_mnmajor<HD>(kq, kk), id_q,
+            umma_ss(tmem + kColDQ + 64 * qt, desc_ds_mn(op_lo, kk), wdesc_mnmajor<HD>(kq, kk), id_q,
                     1);
           }
           umma_commit(grad_done);
@@ -753,30 +868,52 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
       const bool plain = WW > 0 && window_plain(g, win);
       // this thread's slots r and 128 + r (query rows of phase 1 and the dQ
       // epilogue, key rows of phase 2)
-      RowInfo ri[2];
+      // This thread's slots r and 128 + r (query rows of phase 1 and of the dQ
+      // epilogue, key rows of phase 2), packed: key offset (bits 0-15), label
+      // (16-19), valid (20), stored (21). Grid tokens are recomputed for the
+      // epilogues only.
+      uint32_t slotw[2];
 #pragma unroll
-      for (int x = 0; x < 2; ++x)
-        ri[x] = plain ? plain_row_info<(WW > 0 ? WW : 16)>(g, win, x * kRows + r)
-                      : row_info(g, win, x * kRows + r);
-      ci[wg * kRows + r] = key_word(ri[wg]);
+      for (int x = 0; x < 2; ++x) {
+        const RowInfo ri = plain ? plain_row_info<(WW > 0 ? WW : 16)>(g, win, x * kRows + r)
+                                 : row_info(g, win, x * kRows + r);
+        slotw[x] = (uint32_t)ri.key_off | ((uint32_t)ri.label << 16) | ((uint32_t)ri.valid << 20) |
+                   ((uint32_t)ri.stored << 21);
+        if (x == wg) ci[wg * kRows + r] = key_word(ri);
+      }
+      auto slot_token = [&](int x) {
+        return (plain ? plain_row_info<(WW > 0 ? WW : 16)>(g, win, x * kRows + r)
+                      : row_info(g, win, x * kRows + r)).token;
+      };
       if (named_sync_or(1, kSoft, *abort)) break;
       if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
       mbar_wait(&full[s], (uint32_t)((k / NS) & 1), abort, p.status, kWaitLimitNs);
-      const float* brow = bias + s * bp;
+      const int bstride = bias_copy_stride(bp);
+      float* brow = bias + s * 4 * bstride;   // copy 0 (the loaded row), then copies 1-3
+      for (int i = wg * kWg + r; i < g.bins; i += kSoft) {
+        const float v = brow[i];
+        if (i >= 1) brow[bstride + i - 1] = v;
+        if (i >= 2) brow[2 * bstride + i - 2] = v;
+        if (i >= 3) brow[3 * bstride + i - 3] = v;
+      }
+      named_sync(1, kSoft);
       // ---- phase 1 ----
       float bmax = 0.f;
       for (int qt = 0; qt < kHalves; ++qt) {
-        const RowInfo& qi = ri[qt];
+        const uint32_t qw = qt ? slotw[1] : slotw[0];
+        const int q_base = C0 + (int)(qw & 0xFFFF);
+        const int q_label = (int)((qw >> 16) & 15);
+        const bool q_valid = (qw >> 20) & 1;
         mbar_wait(s1_full, (uint32_t)qt, abort, p.status, kWaitLimitNs);
         tc_fence_after();
         float M, l, d, a;
         const uint32_t sc = tl + wg * kRows, dc = tl + kColDP1 + wg * kRows;
         if (WW > 0 && plain)
-          wide_row_stats<true, (WW > 0 ? WW : 16)>(sc, dc, wg * kRows, brow, ci, qi.bias_base,
-                                                   qi.label, p.scale_log2, M, l, d, a);
+          wide_row_stats<true, (WW > 0 ? WW : 16)>(sc, dc, wg * kRows, brow, ci, q_base, q_label,
+                                                   p.scale_log2, M, l, d, a);
         else
-          wide_row_stats<false, 16>(sc, dc, wg * kRows, brow, ci, qi.bias_base, qi.label,
-                                    p.scale_log2, M, l, d, a);
+          wide_row_stats<false, 16>(sc, dc, wg * kRows, brow, ci, q_base, q_label, p.scale_log2,
+                                    M, l, d, a);
         tc_fence_before();
         mbar_arrive(t1_empty);
         float* xq = xch + qt * 4 * kRows;
@@ -793,7 +930,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
           const float f0 = ex2(M - Mx), f1 = ex2(M1 - Mx);
           const float lt = l * f0 + l1 * f1, dt = d * f0 + d1 * f1;
           float2 st = make_float2(INFINITY, 0.f);   // not a real token: P = 0
-          if (qi.valid) {
+          if (q_valid) {
             const float inv = 1.f / lt;
             st = make_float2(Mx + __log2f(lt), dt * inv);
             // |dS_ij| <= max_j P_ij (max_j |dP_ij| + |D|), max_j P_ij = 1 / l;
@@ -822,53 +959,52 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
       }
       int* bins_k = bins + par * bp;
       // ---- phase 2 ----
+      const float4* stats4 = reinterpret_cast<const float4*>(stats);
+      const int jr = r & 63;
+      const uint32_t op_row = op_base + (wg * 2 + (r >> 6)) * 8192 + jr * 128;
       for (int b = 0; b < 4; ++b) {
         const int kb = b >> 1, qt = b & 1;
-        const RowInfo& kj = ri[kb];
-        const float* bk = brow + C0 - kj.key_off;
-        int* bn = bins_k + C0 - kj.key_off;
-        const uint32_t keylab = kj.valid ? (uint32_t)kj.label : 14u;   // pad key: no query matches
-        const bool bins_on = finite && kj.valid;
+        const uint32_t kw = kb ? slotw[1] : slotw[0];
+        const int key_off = (int)(kw & 0xFFFF);
+        const bool k_valid = (kw >> 20) & 1;
+        const uint32_t keylab = k_valid ? (kw >> 16) & 15 : 14u;   // pad key: no query matches
         mbar_wait(s2_full, (uint32_t)(b & 1), abort, p.status, kWaitLimitNs);
-        // the dQ operand is free once the previous block's products are done
-        if (b > 0) mbar_wait(grad_done, (uint32_t)((b - 1) & 1), abort, p.status, kWaitLimitNs);
         tc_fence_after();
-        const int jr = r & 63;
-        const uint32_t op_row = op_base + ((r >> 6) * 2 + wg) * 8192 + jr * 128;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          const int kk = wg * 4 + c;
-          const int i0 = qt * kRows + 16 * kk;
-          const uint32_t op_hi = op_row + (((2 * c) ^ (jr & 7)) << 4);
-          // (the second 16-byte chunk is at ((2c + 1) ^ (jr & 7)) << 4 = this ^ 16)
-          if (WW > 0 && plain)
-            wide_grad_chunk<true, (WW > 0 ? WW : 16)>(tl + 16 * kk, tl + kColDPT + 16 * kk, i0,
-                                                     stats, ci, bk, bn, keylab, bins_on,
-                                                     p.scale_log2, qs, dscale, op_hi,
-                                                     op_hi + 32768);
-          else
-            wide_grad_chunk<false, 16>(tl + 16 * kk, tl + kColDPT + 16 * kk, i0, stats, ci, bk,
-                                       bn, keylab, bins_on, p.scale_log2, qs, dscale, op_hi,
-                                       op_hi + 32768);
-        }
+        const int ib0 = qt * kRows + 64 * wg;
+        const bool bins_on = finite && k_valid;
+        uint64_t* opf = b > 0 ? grad_done : nullptr;   // block b - 1's dK and dQ
+        const uint32_t opph = (uint32_t)((b - 1) & 1);
+        if (WW == 16 && plain)
+          wide_grad_block<true>(tl + 64 * wg, ib0, stats4, ci, brow, bstride, C0 - key_off,
+                                bins_k, keylab, bins_on, p.scale_log2, qs, op_row, jr, opf, opph,
+                                abort, p.status);
+        else
+          wide_grad_block<false>(tl + 64 * wg, ib0, stats4, ci, brow, bstride, C0 - key_off,
+                                 bins_k, keylab, bins_on, p.scale_log2, qs, op_row, jr, opf, opph,
+                                 abort, p.status);
         tmem_wait_st();
         fence_proxy_async();
         tc_fence_before();
         mbar_arrive(pds_full);
-        if (b == 1 || b == 3) {   // dV, dK of key half kb (and dQ after the last block)
-          mbar_wait(grad_done, (uint32_t)(b & 1), abort, p.status, kWaitLimitNs);
+        if (b == 2 || b == 3) {
+          // b = 2: dV and dK of key half 0 (their last products, block 1's, are
+          // done); b = 3: dV and dK of key half 1 and dQ, after the last block
+          const int eb = b == 2 ? 1 : 3, ek = b == 2 ? 0 : 1;
+          mbar_wait(grad_done, (uint32_t)(eb & 1), abort, p.status, kWaitLimitNs);
           tc_fence_after();
           const bool ok = !*abort;
-          if (b == 3) {
-            const RowInfo& qr = ri[wg];   // dQ rows: query slot 128 wg + r
-            store_acc_rows<HD>(tl + kColDQ + 64 * wg, qr, ok, (__nv_bfloat16*)p.out0, g.heads, h);
-          }
+          if (b == 3)   // dQ rows: query slot 128 wg + r
+            store_acc_rows<HD>(tl + kColDQ + 64 * wg, ok && (((wg ? slotw[1] : slotw[0]) >> 21) & 1),
+                               slot_token(wg), (__nv_bfloat16*)p.out0, g.heads, h, dscale);
+          const uint32_t ew = ek ? slotw[1] : slotw[0];
+          const bool k_st = ok && ((ew >> 21) & 1);
+          const long long k_tok = slot_token(ek);
           if (wg == 0)
-            store_acc_rows<HD>(tl + kColDV, kj, ok, (__nv_bfloat16*)p.out2, g.heads, h);
+            store_acc_rows<HD>(tl + kColDV, k_st, k_tok, (__nv_bfloat16*)p.out2, g.heads, h, 1.f);
           else
-            store_acc_rows<HD>(tl + kColDK, kj, ok, (__nv_bfloat16*)p.out1, g.heads, h);
+            store_acc_rows<HD>(tl + kColDK, k_st, k_tok, (__nv_bfloat16*)p.out1, g.heads, h, dscale);
           tc_fence_before();
-          mbar_arrive(b == 1 ? acc_free : t_free);
+          mbar_arrive(b == 2 ? acc_free : t_free);
         }
       }
       mbar_arrive(&bins_full[par]);   // the fold warp adds them to the global sums
