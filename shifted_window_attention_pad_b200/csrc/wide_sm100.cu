@@ -456,61 +456,67 @@ __device__ inline uint64_t desc_ds_k(uint32_t base, int k16) {
   return smem_desc(base + (k16 >> 2) * 16384 + (k16 & 3) * 32, 16, 1024, kSwizzle128);
 }
 
-// Logits of 16 keys k0.. of a plain WW x WW window (k0 a multiple of WW, or
-// of 16 inside a window row), as chunk_logits_plain.
-template <int WW>
-__device__ inline float chunk16_logits_plain(float* x, const float* bias_q, int k0, float c) {
-  bias_q -= (k0 / WW) * (2 * WW - 1) + k0 % WW;
-  float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < 16; j += 2) {
-    x[j] = fmaf(x[j], c, bias_q[-plain_off<WW>(j)]);
-    x[j + 1] = fmaf(x[j + 1], c, bias_q[-plain_off<WW>(j + 1)]);
-    m0 = fmaxf(m0, x[j]);
-    m1 = fmaxf(m1, x[j + 1]);
-  }
-  return fmaxf(m0, m1);
-}
-
 // Phase 1 over 128 keys of one row (columns s_col.. of S and dp_col.. of dP,
 // keys k0base..), 16 at a time with the next chunk's TMEM loads in flight:
 // online maximum M, l = sum 2^(x - M), d = sum 2^(x - M) dP, a = max |dP|.
-template <bool PLAIN, int WW>
+// Plain 16 x 16 windows: the 16 keys of a chunk are one window row, whose
+// table entries (bias_base - plain offset of the key) are a run of 16
+// consecutive floats read as four 16-byte loads from the shifted copies.
+template <bool PLAIN>
 __device__ inline void wide_row_stats(uint32_t s_col, uint32_t dp_col, int k0base,
-                                      const float* brow, const uint32_t* ci, int bias_base,
-                                      int label, float c, float& M, float& l, float& d,
-                                      float& a) {
+                                      const float* bias4, int bstride, const uint32_t* ci,
+                                      int bias_base, int label, float c, float& M, float& l,
+                                      float& d, float& a) {
   M = -INFINITY;
-  l = 0.f;
-  d = 0.f;
+  float2 l2 = make_float2(0.f, 0.f), d2 = make_float2(0.f, 0.f);
   a = 0.f;
   auto work = [&](float* x, int kc) {   // x: 16 of S, then 16 of dP
     const int k0 = k0base + kc;
     float cm;
-    if constexpr (PLAIN)
-      cm = chunk16_logits_plain<WW>(x, brow + bias_base, k0, c);
-    else
-      cm = logits_general<16>(x, brow, ci + k0, bias_base, label, c);
+    if constexpr (PLAIN) {
+      const int lo = bias_base - plain_off<16>(k0) - 15;   // entry of key k0 + 15
+      const int m = lo & 3;
+      const float4* bp = reinterpret_cast<const float4*>(bias4 + m * bstride + (lo - m));
+      float b[16];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 v = bp[u];   // entries of keys k0 + 15 - 4u .. k0 + 12 - 4u
+        b[15 - 4 * u] = v.x;
+        b[14 - 4 * u] = v.y;
+        b[13 - 4 * u] = v.z;
+        b[12 - 4 * u] = v.w;
+      }
+      float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 16; j += 2) {
+        const float2 v = __ffma2_rn(make_float2(x[j], x[j + 1]), make_float2(c, c),
+                                    make_float2(b[j], b[j + 1]));
+        x[j] = v.x;
+        x[j + 1] = v.y;
+        m0 = fmaxf(m0, v.x);
+        m1 = fmaxf(m1, v.y);
+      }
+      cm = fmaxf(m0, m1);
+    } else {
+      cm = logits_general<16>(x, bias4, ci + k0, bias_base, label, c);
+    }
     if (cm > M) {   // rescale the sums to the new maximum
       const float f = ex2(M - cm);
-      l *= f;
-      d *= f;
+      l2 = __fmul2_rn(l2, make_float2(f, f));
+      d2 = __fmul2_rn(d2, make_float2(f, f));
       M = cm;
     }
-    const float Mz = M == -INFINITY ? 0.f : M;   // a chunk of masked keys adds zeros
-    float l0 = 0.f, l1 = 0.f, d0 = 0.f, d1 = 0.f, a0 = 0.f, a1 = 0.f;
+    const float nM = M == -INFINITY ? 0.f : -M;   // a chunk of masked keys adds zeros
+    float a0 = 0.f, a1 = 0.f;
 #pragma unroll
     for (int j = 0; j < 16; j += 2) {
-      const float e0 = ex2(x[j] - Mz), e1 = ex2(x[j + 1] - Mz);
-      l0 += e0;
-      l1 += e1;
-      d0 = fmaf(e0, x[16 + j], d0);
-      d1 = fmaf(e1, x[17 + j], d1);
+      const float2 t = __fadd2_rn(make_float2(x[j], x[j + 1]), make_float2(nM, nM));
+      const float2 e = make_float2(ex2(t.x), ex2(t.y));
+      l2 = __fadd2_rn(l2, e);
+      d2 = __ffma2_rn(e, make_float2(x[16 + j], x[17 + j]), d2);
       a0 = fmaxf(a0, fabsf(x[16 + j]));
       a1 = fmaxf(a1, fabsf(x[17 + j]));
     }
-    l += l0 + l1;
-    d += d0 + d1;
     a = fmaxf(a, fmaxf(a0, a1));
   };
   float xa[32], xb[32];
@@ -532,6 +538,8 @@ __device__ inline void wide_row_stats(uint32_t s_col, uint32_t dp_col, int k0bas
     }
     work(xb, kc + 16);
   }
+  l = l2.x + l2.y;
+  d = d2.x + d2.y;
 }
 
 // Phase 2, this thread's key over the 64 queries of its warpgroup in one
@@ -573,37 +581,46 @@ __device__ inline void wide_grad_block(uint32_t col0, int ib0, const float4* sta
 #pragma unroll
       for (int u2 = 0; u2 < 2; ++u2) {
         const int u = 2 * q4 + u2;
-        const float4 st = stats4[(i0 >> 1) + u];   // (L, D) of queries i0 + 2u, i0 + 2u + 1
-        float P[2], dS[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int ii = 2 * u + e;
-          float x0;
-          int idx;
-          if constexpr (PLAIN) {
-            idx = base + ii;
-            x0 = fmaf(x[ii], c, b4[2 * u2 + e]);
-          } else {
-            const uint32_t w = ci[i0 + ii];
-            idx = kbase + (int)(w & 0xFFFF);
-            x0 = (w >> 16) == keylab ? fmaf(x[ii], c, bias4[idx]) : -INFINITY;
-          }
-          const float Li = e ? st.z : st.x, Di = e ? st.w : st.y;
-          P[e] = ex2(x0 - Li);
-          dS[e] = P[e] * (x[16 + ii] - Di);
-          if (bins_on) red_add_s32_relaxed(bins + idx, round_to_int(dS[e] * qs));
+        const float4 st = stats4[(i0 >> 1) + u];   // -L, -D of queries i0 + 2u, i0 + 2u + 1
+        const float2 s2 = make_float2(x[2 * u], x[2 * u + 1]);
+        float2 lg;
+        int idx0, idx1;
+        if constexpr (PLAIN) {
+          idx0 = base + 2 * u;
+          idx1 = idx0 + 1;
+          lg = __ffma2_rn(s2, make_float2(c, c), make_float2(b4[2 * u2], b4[2 * u2 + 1]));
+        } else {
+          const uint32_t w0 = ci[i0 + 2 * u], w1 = ci[i0 + 2 * u + 1];
+          idx0 = kbase + (int)(w0 & 0xFFFF);
+          idx1 = kbase + (int)(w1 & 0xFFFF);
+          lg.x = (w0 >> 16) == keylab ? fmaf(s2.x, c, bias4[idx0]) : -INFINITY;
+          lg.y = (w1 >> 16) == keylab ? fmaf(s2.y, c, bias4[idx1]) : -INFINITY;
         }
+        const float2 t = __fadd2_rn(lg, make_float2(st.x, st.y));
+        const float2 P = make_float2(ex2(t.x), ex2(t.y));
+        const float2 dS =
+            __fmul2_rn(P, __fadd2_rn(make_float2(x[16 + 2 * u], x[17 + 2 * u]), make_float2(st.z, st.w)));
+        if (bins_on) {   // dS in units of 2^-E, rounded to integers (q = 2^E: the product is exact)
+          const float2 q = __ffma2_rn(dS, make_float2(qs, qs), make_float2(12582912.0f, 12582912.0f));
+          red_add_s32_relaxed(bins + idx0, __float_as_int(q.x) - 0x4B400000);
+          red_add_s32_relaxed(bins + idx1, __float_as_int(q.y) - 0x4B400000);
+        }
+        // hi = the top 16 bits of each value (bf16 truncation), lo = bf16 of the rest
         {
-          const uint32_t a = __float_as_uint(P[0]) & 0xFFFF0000u;
-          const uint32_t bb = __float_as_uint(P[1]) & 0xFFFF0000u;
+          const uint32_t a = __float_as_uint(P.x), bb = __float_as_uint(P.y);
           pw[u] = __byte_perm(a, bb, 0x7632);
-          pw[8 + u] = pack_bf16(P[0] - __uint_as_float(a), P[1] - __uint_as_float(bb));
+          const float2 r2 = __ffma2_rn(
+              make_float2(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(bb & 0xFFFF0000u)),
+              make_float2(-1.f, -1.f), P);
+          pw[8 + u] = pack_bf16(r2.x, r2.y);
         }
         {
-          const uint32_t a = __float_as_uint(dS[0]) & 0xFFFF0000u;
-          const uint32_t bb = __float_as_uint(dS[1]) & 0xFFFF0000u;
+          const uint32_t a = __float_as_uint(dS.x), bb = __float_as_uint(dS.y);
           sw[u] = __byte_perm(a, bb, 0x7632);
-          sw[8 + u] = pack_bf16(dS[0] - __uint_as_float(a), dS[1] - __uint_as_float(bb));
+          const float2 r2 = __ffma2_rn(
+              make_float2(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(bb & 0xFFFF0000u)),
+              make_float2(-1.f, -1.f), dS);
+          sw[8 + u] = pack_bf16(r2.x, r2.y);
         }
       }
     }
@@ -908,12 +925,12 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
         tc_fence_after();
         float M, l, d, a;
         const uint32_t sc = tl + wg * kRows, dc = tl + kColDP1 + wg * kRows;
-        if (WW > 0 && plain)
-          wide_row_stats<true, (WW > 0 ? WW : 16)>(sc, dc, wg * kRows, brow, ci, q_base, q_label,
-                                                   p.scale_log2, M, l, d, a);
+        if (WW == 16 && plain)
+          wide_row_stats<true>(sc, dc, wg * kRows, brow, bstride, ci, q_base, q_label,
+                               p.scale_log2, M, l, d, a);
         else
-          wide_row_stats<false, 16>(sc, dc, wg * kRows, brow, ci, q_base, q_label, p.scale_log2,
-                                    M, l, d, a);
+          wide_row_stats<false>(sc, dc, wg * kRows, brow, bstride, ci, q_base, q_label,
+                                p.scale_log2, M, l, d, a);
         tc_fence_before();
         mbar_arrive(t1_empty);
         float* xq = xch + qt * 4 * kRows;
@@ -939,7 +956,12 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
             if (!(rb <= 3.0e38f)) rb = INFINITY;
             bmax = fmaxf(bmax, rb);
           }
-          stats[qt * kRows + r] = st;
+          // per query pair: (-L0, -L1, -D0, -D1), so one 16-byte load gives
+          // both queries' values as operand pairs of the packed arithmetic
+          const int qi = qt * kRows + r;
+          float* sp = reinterpret_cast<float*>(stats) + (qi >> 1) * 4 + (qi & 1);
+          sp[0] = -st.x;
+          sp[2] = -st.y;
         }
       }
       if (wg == 0) {
