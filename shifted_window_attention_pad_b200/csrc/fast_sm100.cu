@@ -366,11 +366,13 @@ __device__ inline void store_split_cols_part(uint32_t blk_hi, uint32_t blk_lo, i
     uint32_t hw[4], lw[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const uint32_t a = __float_as_uint(v[cc * 8 + 2 * e]) & 0xFFFF0000u;
-      const uint32_t b = __float_as_uint(v[cc * 8 + 2 * e + 1]) & 0xFFFF0000u;
-      hw[e] = __byte_perm(a, b, 0x7632);
-      lw[e] = pack_bf16(v[cc * 8 + 2 * e] - __uint_as_float(a),
-                        v[cc * 8 + 2 * e + 1] - __uint_as_float(b));
+      const float2 x = make_float2(v[cc * 8 + 2 * e], v[cc * 8 + 2 * e + 1]);
+      const uint32_t a = __float_as_uint(x.x), b = __float_as_uint(x.y);
+      hw[e] = __byte_perm(a, b, 0x7632);   // the top 16 bits of each
+      const float2 r = __ffma2_rn(make_float2(__uint_as_float(a & 0xFFFF0000u),
+                                              __uint_as_float(b & 0xFFFF0000u)),
+                                  make_float2(-1.f, -1.f), x);   // exact remainders
+      lw[e] = pack_bf16(r.x, r.y);
     }
     const uint32_t off = lr * 128 + ((c ^ (lr & 7)) << 4);
     st_shared_v4(blk_hi + off, hw[0], hw[1], hw[2], hw[3]);
@@ -623,26 +625,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       if (me.valid) {
         inv = 1.f / exp_sum<N>(x, m);
 #pragma unroll
-        for (int j = 0; j < N; ++j) x[j] *= inv;
+        for (int j = 0; j < N; j += 2) {
+          const float2 pj = __fmul2_rn(make_float2(x[j], x[j + 1]), make_float2(inv, inv));
+          x[j] = pj.x;
+          x[j + 1] = pj.y;
+        }
       } else {
 #pragma unroll
         for (int j = 0; j < N; ++j) x[j] = 0.f;
       }
       // TMEM loads are warp-collective: every lane runs them, valid row or not
       // (x = 0 on invalid rows, so D = 0 and dS = 0 there).
-      float dd[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 dda = make_float2(0.f, 0.f), ddb = make_float2(0.f, 0.f);   // keys j mod 4
       float mdp = 0.f;
       {
         float dp[N];
         tmem_load_cols<N>(dp_col, dp);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < N; ++j) {
-          dd[j & 3] = fmaf(x[j], dp[j], dd[j & 3]);
-          mdp = fmaxf(mdp, fabsf(dp[j]));
+        for (int j = 0; j < N; j += 4) {
+          dda = __ffma2_rn(make_float2(x[j], x[j + 1]), make_float2(dp[j], dp[j + 1]), dda);
+          ddb = __ffma2_rn(make_float2(x[j + 2], x[j + 3]), make_float2(dp[j + 2], dp[j + 3]), ddb);
+          mdp = fmaxf(mdp, fmaxf(fmaxf(fabsf(dp[j]), fabsf(dp[j + 1])),
+                                 fmaxf(fabsf(dp[j + 2]), fabsf(dp[j + 3]))));
         }
       }
-      const float D = (dd[0] + dd[1]) + (dd[2] + dd[3]);
+      const float D = (dda.x + dda.y) + (ddb.x + ddb.y);
       __syncwarp();
 #pragma unroll
       for (int c = 0; c < N / 32; ++c) tmem_st32(s_col + 32 * c, x + 32 * c);
@@ -676,20 +684,35 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         tmem_ld32(s_col + 32 * c, pc);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ds[j] = pc[j] * (ds[j] - D);   // dS (0 off the row)
+        for (int j = 0; j < 32; j += 2) {   // dS (0 off the row)
+          const float2 v = __fmul2_rn(make_float2(pc[j], pc[j + 1]),
+                                      __fadd2_rn(make_float2(ds[j], ds[j + 1]), make_float2(-D, -D)));
+          ds[j] = v.x;
+          ds[j + 1] = v.y;
+        }
         if (me.valid && finite) {
           // bias-gradient bins: integers in units of 2^-E; integer adds
           // commute, so the sums do not depend on the order the lanes land in
           // (unrolled: a runtime index would put ds in local memory)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(32 * c + j)
-                                  : (int)(lds_u32(cw + 32 * c + j) & 0xFFFF);
-            red_add_s32(bq - off, round_to_int(ds[j] * qs));
+          for (int j = 0; j < 32; j += 2) {
+            // ds * 2^E is exact, so one fused multiply-add rounds it to an integer
+            const float2 q = __ffma2_rn(make_float2(ds[j], ds[j + 1]), make_float2(qs, qs),
+                                        make_float2(12582912.0f, 12582912.0f));
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int off = plain ? plain_off<(WW > 0 ? WW : 8)>(32 * c + j + e)
+                                    : (int)(lds_u32(cw + 32 * c + j + e) & 0xFFFF);
+              red_add_s32(bq - off, __float_as_int(e ? q.y : q.x) - 0x4B400000);
+            }
           }
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ds[j] *= dscale;
+        for (int j = 0; j < 32; j += 2) {
+          const float2 v = __fmul2_rn(make_float2(ds[j], ds[j + 1]), make_float2(dscale, dscale));
+          ds[j] = v.x;
+          ds[j + 1] = v.y;
+        }
         __syncwarp();
         tmem_st32(dp_col + 32 * c, ds);
       }

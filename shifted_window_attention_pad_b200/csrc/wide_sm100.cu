@@ -109,10 +109,12 @@ __device__ inline float chunk_logits_plain(float* x, const float* bias_q, int k0
   float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
-    x[j] = fmaf(x[j], c, bias_q[-plain_off<WW>(j)]);
-    x[j + 1] = fmaf(x[j + 1], c, bias_q[-plain_off<WW>(j + 1)]);
-    m0 = fmaxf(m0, x[j]);
-    m1 = fmaxf(m1, x[j + 1]);
+    const float2 v = __ffma2_rn(make_float2(x[j], x[j + 1]), make_float2(c, c),
+                                make_float2(bias_q[-plain_off<WW>(j)], bias_q[-plain_off<WW>(j + 1)]));
+    x[j] = v.x;
+    x[j + 1] = v.y;
+    m0 = fmaxf(m0, v.x);
+    m1 = fmaxf(m1, v.y);
   }
   return fmaxf(m0, m1);
 }
@@ -165,16 +167,16 @@ __device__ inline float wide_pass2(uint32_t slot, float mo) {
   float l = 0.f;
   for_row_chunks(slot, [&](float* x, int k0) {
     uint32_t w[16];
-    float la = 0.f, lb = 0.f;
+    float2 l2 = make_float2(0.f, 0.f);
+    const float2 nm = make_float2(-mo, -mo);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const float a = ex2(x[2 * j] - mo);
-      const float b = ex2(x[2 * j + 1] - mo);
-      la += a;
-      lb += b;
-      w[j] = pack_bf16(a, b);
+      const float2 t = __fadd2_rn(make_float2(x[2 * j], x[2 * j + 1]), nm);
+      const float2 e = make_float2(ex2(t.x), ex2(t.y));
+      l2 = __fadd2_rn(l2, e);
+      w[j] = pack_bf16(e.x, e.y);
     }
-    l += la + lb;
+    l += l2.x + l2.y;
     __syncwarp();
     tmem_st16u(slot + k0 / 2, w);
   });

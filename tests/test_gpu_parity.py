@@ -306,11 +306,12 @@ def test_tiled_path_forced_on_window64_workloads(name):
             assert e <= BF16_TOL, (h, n, e)
 
 
-def test_tiled_backward_is_deterministic():
+@pytest.mark.parametrize("path", [3, 2])
+def test_backward_of_256_token_windows_is_deterministic(path):
     wl = WORKLOADS["downsampled-128x272-w16"]
     inp = make_inputs(wl)
-    d = sb.desc_for(wl)
-    assert sb.swin_wattn_path(d) == 2
+    d = sb.desc_for(wl, flags=sb.SWIN_FLAG_FORCE_TILED if path == 2 else 0)
+    assert sb.swin_wattn_path(d) == path
     a = run_gpu(d, inp, want_lse=False)
     b = run_gpu(d, inp, want_lse=False)
     for n in ("o", "dq", "dk", "dv", "dT"):
