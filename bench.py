@@ -45,8 +45,8 @@ def dominant_kernel(kpath, wl):
         return ("bwd_kernel<%d,%d> (tcgen05/TMA fused backward: S, dP, dV, dQ, dK, dT)" %
                 (wl.head_dim, 8 if wl.win == 8 else 0))
     if kpath == 3:
-        return ("tiled_bwd_kernel<%d,256,32> (warp-MMA backward, one CTA per window and head)" %
-                wl.head_dim)
+        return ("wide_bwd_kernel<%d,%d> (tcgen05/TMA backward of 256-token windows: row "
+                "statistics, S^T, dP^T, dV, dK, dQ, dT)" % (wl.head_dim, 16 if wl.win == 16 else 0))
     if kpath == 2:
         return ("tiled_bwd_kernel<%d,%d,32> (warp-MMA backward, one CTA per window and head)" %
                 (wl.head_dim, 64 if wl.win ** 2 <= 64 else (128 if wl.win ** 2 <= 128 else 256)))
@@ -57,7 +57,8 @@ KERNEL_SOURCES = {
     1: ("shifted_window_attention_pad_b200/csrc/fast_sm100.cu",
         "shifted_window_attention_pad_b200/csrc/fast_common.cuh",
         "shifted_window_attention_pad_b200/csrc/sm100_ptx.cuh"),
-    3: ("shifted_window_attention_pad_b200/csrc/tiled_mma.cu",
+    3: ("shifted_window_attention_pad_b200/csrc/wide_sm100.cu",
+        "shifted_window_attention_pad_b200/csrc/fast_common.cuh",
         "shifted_window_attention_pad_b200/csrc/sm100_ptx.cuh"),
     2: ("shifted_window_attention_pad_b200/csrc/tiled_mma.cu",
         "shifted_window_attention_pad_b200/csrc/sm100_ptx.cuh"),
