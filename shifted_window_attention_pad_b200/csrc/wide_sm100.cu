@@ -381,9 +381,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 // Per (window, head) item, with Q, K, V, dO of the window in shared memory:
 //  Phase 1, row statistics, query-major: for each 128-query half qt,
 //    S = Q_qt K^T and dP = dO_qt V^T over all 256 keys fill the 512 TMEM
-//    columns; warpgroup w reads keys 128 w .. 128 w + 127 of every row and
-//    keeps an online maximum M, l = sum 2^(x - M), d = sum 2^(x - M) dP and
-//    max |dP|; the two halves of a row are merged through shared memory into
+//    columns; warpgroup w (of three) reads the 16-key chunks w, w + 3, ... of
+//    every row and keeps an online maximum M, l = sum 2^(x - M),
+//    d = sum 2^(x - M) dP and max |dP|; the partials of a row are merged
+//    through shared memory into
 //    L = M + log2 l (log2 units) and D = d / l = sum_j P_ij dP_ij, and a bound
 //    (max_j |dP_ij| + |D|) / l >= |dS_ij| of the row. The largest bound of the
 //    window sets the unit 2^-E of its exact bias-gradient sums.
@@ -395,7 +396,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 //    into shared memory (the A operand of both dK_kb += dS^T Q_qt and
 //    dQ_qt += dS K_kb) and into the bias-gradient bins. The scale
 //    head_dim^-1/2 of dQ and dK is applied to their fp32 sums at the end.
-//    Warpgroup w takes queries 64 w .. 64 w + 63 of the block.
+//    Warpgroup w takes the 16-query chunks w, w + 3, w + 6 of the block.
 //    The products overlap the row work: once a block's rows are done, dP^T of
 //    the next block goes into the dP^T columns (read already), dV of this
 //    block runs, then S^T of the next block replaces P, and dK and dQ of this
@@ -418,8 +419,11 @@ __host__ __device__ inline int bias_copy_stride(int bins_pad) { return bins_pad 
 constexpr uint32_t kColDP1 = 256;                    // phase 1 dP (S at 0)
 constexpr uint32_t kColDPT = 128;                    // phase 2 dP^T (S^T at 0)
 constexpr uint32_t kColDV = 256, kColDK = 320, kColDQ = 384;
-constexpr int kWideBwdWarps = 11;                    // 8 softmax, producer, MMA, bin fold
-constexpr int kWideFoldWarp = 10;
+// Backward warps: three softmax warpgroups (0-11), the TMA producer, the MMA
+// issuer and the bin fold. Fifteen warps leave 128 registers a thread.
+constexpr int kWideBwdWarps = 15;
+constexpr int kWideSoftWg = 3;
+constexpr int kWideProducerWarp = 12, kWideMmaWarp = 13, kWideFoldWarp = 14;
 
 struct WideBwdLayout {
   uint32_t tiles, dsop, bias, colinfo, stats, xch, bins, wb, bars, misc, total;
@@ -431,8 +435,9 @@ __host__ __device__ inline WideBwdLayout wide_bwd_layout(int bins_pad) {
   WideBwdLayout L;
   L.tiles = 0;
   L.dsop = L.tiles + C::kStages * 4 * C::kTileBytes;
-  L.xch = L.dsop;                            // [qt][4][128] partial statistics (phase 1
-                                             // only: the dQ operand is free then)
+  L.xch = L.dsop;                            // [qt][2][4][128] partial statistics of
+                                             // warpgroups 1 and 2 (phase 1 only: the
+                                             // dQ operand is free then)
   L.bias = L.dsop + C::kOpBytes;
   L.colinfo = L.bias + C::kStages * 4 * bias_copy_stride(bins_pad) * 4;
   L.stats = L.colinfo + kKeys * 4;           // float2 {L, D} per query
@@ -458,22 +463,44 @@ __device__ inline uint64_t desc_ds_k(uint32_t base, int k16) {
   return smem_desc(base + (k16 >> 2) * 16384 + (k16 & 3) * 32, 16, 1024, kSwizzle128);
 }
 
-// Phase 1 over 128 keys of one row (columns s_col.. of S and dp_col.. of dP,
-// keys k0base..), 16 at a time with the next chunk's TMEM loads in flight:
-// online maximum M, l = sum 2^(x - M), d = sum 2^(x - M) dP, a = max |dP|.
-// Plain 16 x 16 windows: the 16 keys of a chunk are one window row, whose
-// table entries (bias_base - plain offset of the key) are a run of 16
-// consecutive floats read as four 16-byte loads from the shifted copies.
+// Runs work(x, i) over the n chunks i = 0 .. n-1 of a thread's list (n is
+// the same for the whole warp): load(x, i) issues the TMEM loads of chunk i.
+// One register buffer: with three softmax warpgroups the other warps of the
+// scheduler cover the load latency.
+template <typename LD, typename WK>
+__device__ inline void pipelined_chunks(int n, LD&& load, WK&& work) {
+#pragma unroll 1
+  for (int i = 0; i < n; ++i) {
+    float x[32];
+    load(x, i);
+    tmem_wait_ld_regs(x);
+    work(x, i);
+  }
+}
+
+// Phase 1 over the 16-key chunks w, w + 3, w + 6, ... of one row (S at
+// columns s_col + 16 c, dP at dp_col + 16 c for chunk c): online maximum M,
+// l = sum 2^(x - M), d = sum 2^(x - M) dP, a = max |dP|. Plain 16 x 16
+// windows: the 16 keys of a chunk are one window row, whose table entries
+// (bias_base - plain offset of the key) are a run of 16 consecutive floats
+// read as four 16-byte loads from the shifted copies.
 template <bool PLAIN>
-__device__ inline void wide_row_stats(uint32_t s_col, uint32_t dp_col, int k0base,
+__device__ inline void wide_row_stats(uint32_t s_col, uint32_t dp_col, int w,
                                       const float* bias4, int bstride, const uint32_t* ci,
                                       int bias_base, int label, float c, float& M, float& l,
                                       float& d, float& a) {
   M = -INFINITY;
   float2 l2 = make_float2(0.f, 0.f), d2 = make_float2(0.f, 0.f);
   a = 0.f;
-  auto work = [&](float* x, int kc) {   // x: 16 of S, then 16 of dP
-    const int k0 = k0base + kc;
+  const int n = (kKeys / 16 - w + kWideSoftWg - 1) / kWideSoftWg;
+  auto load = [&](float* x, int i) {
+    const int k0 = 16 * (w + kWideSoftWg * i);
+    __syncwarp();
+    tmem_ld16(s_col + k0, x);
+    tmem_ld16(dp_col + k0, x + 16);
+  };
+  auto work = [&](float* x, int i) {   // x: 16 of S, then 16 of dP
+    const int k0 = 16 * (w + kWideSoftWg * i);
     float cm;
     if constexpr (PLAIN) {
       const int lo = bias_base - plain_off<16>(k0) - 15;   // entry of key k0 + 15
@@ -521,48 +548,36 @@ __device__ inline void wide_row_stats(uint32_t s_col, uint32_t dp_col, int k0bas
     }
     a = fmaxf(a, fmaxf(a0, a1));
   };
-  float xa[32], xb[32];
-  __syncwarp();
-  tmem_ld16(s_col, xa);
-  tmem_ld16(dp_col, xa + 16);
-#pragma unroll 1
-  for (int kc = 0; kc < kRows; kc += 32) {
-    tmem_wait_ld_regs(xa);
-    __syncwarp();
-    tmem_ld16(s_col + kc + 16, xb);
-    tmem_ld16(dp_col + kc + 16, xb + 16);
-    work(xa, kc);
-    tmem_wait_ld_regs(xb);
-    if (kc + 32 < kRows) {
-      __syncwarp();
-      tmem_ld16(s_col + kc + 32, xa);
-      tmem_ld16(dp_col + kc + 32, xa + 16);
-    }
-    work(xb, kc + 16);
-  }
+  pipelined_chunks(n, load, work);
   l = l2.x + l2.y;
   d = d2.x + d2.y;
 }
 
-// Phase 2, this thread's key over the 64 queries of its warpgroup in one
-// block, in chunks of 16 (i0 = first query of the chunk): P and dS from S^T
-// and dP^T, P's hi / lo pairs back into its S^T columns, dS's into the
-// shared-memory operand (after `op_free`, when given), dS to the
-// bias-gradient bins. The TMEM load
-// of chunk c + 1 is in flight while chunk c is worked on. Bias and bins of
-// pair (i, j) sit at kbase + off(i), kbase = C0 - off(j). Plain 16 x 16
-// windows: a chunk is one window row of queries, so its 16 table entries are
-// consecutive and come as four 16-byte loads from the shifted bias copies.
+// Phase 2, this thread's key over the 16-query chunks kk = w, w + 3, w + 6
+// (kk < 8) of one block (i0 = ib0 + 16 kk, the chunk's first query): P and dS
+// from S^T and dP^T, P's hi / lo pairs back into its S^T columns, dS's into
+// the shared-memory operand (after `op_free`, when given), dS to the
+// bias-gradient bins. Bias and bins of pair (i, j) sit at kbase + off(i),
+// kbase = C0 - off(j). Plain 16 x 16 windows: a chunk is one window row of
+// queries, so its 16 table entries are consecutive and come as four 16-byte
+// loads from the shifted bias copies.
 template <bool PLAIN>
-__device__ inline void wide_grad_block(uint32_t col0, int ib0, const float4* stats4,
+__device__ inline void wide_grad_block(uint32_t tl, int w, int ib0, const float4* stats4,
                                        const uint32_t* ci, const float* bias4, int bstride,
                                        int kbase, int* bins, uint32_t keylab, bool bins_on,
-                                       float c, float qs, uint32_t op_row, int jr,
+                                       float c, float qs, uint32_t op_key, int jr,
                                        uint64_t* op_free, uint32_t op_phase, volatile int* abort,
                                        int* status) {
-  float xa[32], xb[32];   // [0, 16) S^T, [16, 32) dP^T of one chunk
-  auto work = [&](float* x, int cc) {
-    const int i0 = ib0 + 16 * cc;
+  const int n = (kRows / 16 - w + kWideSoftWg - 1) / kWideSoftWg;
+  auto load = [&](float* x, int i) {   // [0, 16) S^T, [16, 32) dP^T of chunk w + 3 i
+    const int kk = w + kWideSoftWg * i;
+    __syncwarp();
+    tmem_ld16(tl + 16 * kk, x);
+    tmem_ld16(tl + kColDPT + 16 * kk, x + 16);
+  };
+  auto work = [&](float* x, int i) {
+    const int kk = w + kWideSoftWg * i;
+    const int i0 = ib0 + 16 * kk;
     int base = 0, m = 0;
     if constexpr (PLAIN) {
       base = kbase + plain_off<16>(i0);
@@ -626,35 +641,18 @@ __device__ inline void wide_grad_block(uint32_t col0, int ib0, const float4* sta
         }
       }
     }
-    const uint32_t col = col0 + 16 * cc;
     __syncwarp();
-    tmem_st16u(col, pw);
+    tmem_st16u(tl + 16 * kk, pw);
     // the dS operand is free once the previous block's dK and dQ are done
-    if (cc == 0 && op_free) mbar_wait(op_free, op_phase, abort, status, kWaitLimitNs);
-    const uint32_t op_hi = op_row + (((2 * cc) ^ (jr & 7)) << 4);   // second chunk: ^ 16
+    if (i == 0 && op_free) mbar_wait(op_free, op_phase, abort, status, kWaitLimitNs);
+    // query half kk / 4, 16-byte chunks 2 (kk % 4) and 2 (kk % 4) + 1 of the key's row
+    const uint32_t op_hi = op_key + (kk >> 2) * 16384 + (((2 * (kk & 3)) ^ (jr & 7)) << 4);
     st_shared_v4(op_hi, sw[0], sw[1], sw[2], sw[3]);
     st_shared_v4(op_hi ^ 16u, sw[4], sw[5], sw[6], sw[7]);
     st_shared_v4(op_hi + 32768, sw[8], sw[9], sw[10], sw[11]);
     st_shared_v4((op_hi + 32768) ^ 16u, sw[12], sw[13], sw[14], sw[15]);
   };
-  __syncwarp();
-  tmem_ld16(col0, xa);
-  tmem_ld16(col0 + kColDPT, xa + 16);
-#pragma unroll
-  for (int cc = 0; cc < 4; cc += 2) {
-    tmem_wait_ld_regs(xa);
-    __syncwarp();
-    tmem_ld16(col0 + 16 * (cc + 1), xb);
-    tmem_ld16(col0 + kColDPT + 16 * (cc + 1), xb + 16);
-    work(xa, cc);
-    tmem_wait_ld_regs(xb);
-    if (cc + 2 < 4) {
-      __syncwarp();
-      tmem_ld16(col0 + 16 * (cc + 2), xa);
-      tmem_ld16(col0 + kColDPT + 16 * (cc + 2), xa + 16);
-    }
-    work(xb, cc + 1);
-  }
+  pipelined_chunks(n, load, work);
 }
 
 // Rows of one accumulator (HD columns) to the grid tokens of `ri` (lane = row).
@@ -675,7 +673,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
   using C = WideBwdCfg<HD>;
   constexpr int NS = C::kStages;
   constexpr uint32_t tile_bytes = C::kTileBytes, RB = C::kRowBytes;
-  constexpr int kSoft = 2 * kWg;   // threads of the two softmax warpgroups
+  constexpr int kSoft = kWideSoftWg * kWg;   // threads of the softmax warpgroups
   const Geo& g = p.g;
   const int bp = p.bins_pad;
   const WideBwdLayout L = wide_bwd_layout<HD>(bp);
@@ -724,11 +722,11 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == kProducerWarp && lane == 0)
+  if (warp == kWideProducerWarp && lane == 0)
     for (int tt = 0; tt < 4; ++tt)
       for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
   for (int i = threadIdx.x; i < 2 * bp; i += kWideBwdWarps * 32) bins[i] = 0;
-  if (warp == kMmaWarp) {
+  if (warp == kWideMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -737,7 +735,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kProducerWarp) {
+  if (warp == kWideProducerWarp) {
     if (lane == 0) {
       long long k = 0;
       for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
@@ -754,7 +752,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
           mbar_drain(&full[j % NS], (uint32_t)((j / NS) & 1), kTestLimitNs * 100);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kWideMmaWarp) {
     if (lane == 0) {   // every product, in dependency order
       constexpr uint32_t id_s1 = idesc_bf16(kRows, kKeys, 0, 0);
       constexpr uint32_t id_s2 = idesc_bf16(kRows, kRows, 0, 0);
@@ -871,7 +869,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
       __syncwarp();
       mbar_arrive(&bins_empty[par]);
     }
-  } else if (warp < 8) {
+  } else if (warp < kWideSoftWg * 4) {
     const int wg = warp >> 2;
     const int r = threadIdx.x & (kWg - 1);
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -898,7 +896,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
                                  : row_info(g, win, x * kRows + r);
         slotw[x] = (uint32_t)ri.key_off | ((uint32_t)ri.label << 16) | ((uint32_t)ri.valid << 20) |
                    ((uint32_t)ri.stored << 21);
-        if (x == wg) ci[wg * kRows + r] = key_word(ri);
+        if (x == wg) ci[wg * kRows + r] = key_word(ri);   // (warpgroups 0 and 1)
       }
       auto slot_token = [&](int x) {
         return (plain ? plain_row_info<(WW > 0 ? WW : 16)>(g, win, x * kRows + r)
@@ -926,28 +924,30 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
         mbar_wait(s1_full, (uint32_t)qt, abort, p.status, kWaitLimitNs);
         tc_fence_after();
         float M, l, d, a;
-        const uint32_t sc = tl + wg * kRows, dc = tl + kColDP1 + wg * kRows;
         if (WW == 16 && plain)
-          wide_row_stats<true>(sc, dc, wg * kRows, brow, bstride, ci, q_base, q_label,
+          wide_row_stats<true>(tl, tl + kColDP1, wg, brow, bstride, ci, q_base, q_label,
                                p.scale_log2, M, l, d, a);
         else
-          wide_row_stats<false>(sc, dc, wg * kRows, brow, bstride, ci, q_base, q_label,
+          wide_row_stats<false>(tl, tl + kColDP1, wg, brow, bstride, ci, q_base, q_label,
                                 p.scale_log2, M, l, d, a);
         tc_fence_before();
         mbar_arrive(t1_empty);
-        float* xq = xch + qt * 4 * kRows;
-        if (wg == 1) {
-          xq[r] = M;
-          xq[kRows + r] = l;
-          xq[2 * kRows + r] = d;
-          xq[3 * kRows + r] = a;
+        float* xq = xch + qt * 2 * 4 * kRows;   // [warpgroup - 1][M, l, d, a][row]
+        if (wg > 0) {
+          float* xw = xq + (wg - 1) * 4 * kRows;
+          xw[r] = M;
+          xw[kRows + r] = l;
+          xw[2 * kRows + r] = d;
+          xw[3 * kRows + r] = a;
         }
         named_sync(1, kSoft);
         if (wg == 0) {
-          const float M1 = xq[r], l1 = xq[kRows + r], d1 = xq[2 * kRows + r], a1 = xq[3 * kRows + r];
-          const float Mx = fmaxf(M, M1);
-          const float f0 = ex2(M - Mx), f1 = ex2(M1 - Mx);
-          const float lt = l * f0 + l1 * f1, dt = d * f0 + d1 * f1;
+          const float M1 = xq[r], l1 = xq[kRows + r], d1 = xq[2 * kRows + r];
+          const float M2 = xq[4 * kRows + r], l2 = xq[5 * kRows + r], d2 = xq[6 * kRows + r];
+          const float a1 = fmaxf(xq[3 * kRows + r], xq[7 * kRows + r]);
+          const float Mx = fmaxf(M, fmaxf(M1, M2));
+          const float f0 = ex2(M - Mx), f1 = ex2(M1 - Mx), f2 = ex2(M2 - Mx);
+          const float lt = l * f0 + l1 * f1 + l2 * f2, dt = d * f0 + d1 * f1 + d2 * f2;
           float2 st = make_float2(INFINITY, 0.f);   // not a real token: P = 0
           if (q_valid) {
             const float inv = 1.f / lt;
@@ -985,7 +985,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
       // ---- phase 2 ----
       const float4* stats4 = reinterpret_cast<const float4*>(stats);
       const int jr = r & 63;
-      const uint32_t op_row = op_base + (wg * 2 + (r >> 6)) * 8192 + jr * 128;
+      const uint32_t op_key = op_base + (r >> 6) * 8192 + jr * 128;   // this key's row, query half 0
       for (int b = 0; b < 4; ++b) {
         const int kb = b >> 1, qt = b & 1;
         const uint32_t kw = kb ? slotw[1] : slotw[0];
@@ -994,18 +994,18 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
         const uint32_t keylab = k_valid ? (kw >> 16) & 15 : 14u;   // pad key: no query matches
         mbar_wait(s2_full, (uint32_t)(b & 1), abort, p.status, kWaitLimitNs);
         tc_fence_after();
-        const int ib0 = qt * kRows + 64 * wg;
+        const int ib0 = qt * kRows;
         const bool bins_on = finite && k_valid;
         uint64_t* opf = b > 0 ? grad_done : nullptr;   // block b - 1's dK and dQ
         const uint32_t opph = (uint32_t)((b - 1) & 1);
         if (WW == 16 && plain)
-          wide_grad_block<true>(tl + 64 * wg, ib0, stats4, ci, brow, bstride, C0 - key_off,
-                                bins_k, keylab, bins_on, p.scale_log2, qs, op_row, jr, opf, opph,
-                                abort, p.status);
+          wide_grad_block<true>(tl, wg, ib0, stats4, ci, brow, bstride, C0 - key_off, bins_k,
+                                keylab, bins_on, p.scale_log2, qs, op_key, jr, opf, opph, abort,
+                                p.status);
         else
-          wide_grad_block<false>(tl + 64 * wg, ib0, stats4, ci, brow, bstride, C0 - key_off,
-                                 bins_k, keylab, bins_on, p.scale_log2, qs, op_row, jr, opf, opph,
-                                 abort, p.status);
+          wide_grad_block<false>(tl, wg, ib0, stats4, ci, brow, bstride, C0 - key_off, bins_k,
+                                 keylab, bins_on, p.scale_log2, qs, op_key, jr, opf, opph, abort,
+                                 p.status);
         tmem_wait_st();
         fence_proxy_async();
         tc_fence_before();
@@ -1017,16 +1017,24 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
           mbar_wait(grad_done, (uint32_t)(eb & 1), abort, p.status, kWaitLimitNs);
           tc_fence_after();
           const bool ok = !*abort;
-          if (b == 3)   // dQ rows: query slot 128 wg + r
-            store_acc_rows<HD>(tl + kColDQ + 64 * wg, ok && (((wg ? slotw[1] : slotw[0]) >> 21) & 1),
-                               slot_token(wg), (__nv_bfloat16*)p.out0, g.heads, h, dscale);
-          const uint32_t ew = ek ? slotw[1] : slotw[0];
-          const bool k_st = ok && ((ew >> 21) & 1);
-          const long long k_tok = slot_token(ek);
-          if (wg == 0)
-            store_acc_rows<HD>(tl + kColDV, k_st, k_tok, (__nv_bfloat16*)p.out2, g.heads, h, 1.f);
-          else
-            store_acc_rows<HD>(tl + kColDK, k_st, k_tok, (__nv_bfloat16*)p.out1, g.heads, h, dscale);
+          // warpgroup 0: dV rows, 1: dK rows (key slots), 2: dQ rows of both
+          // query halves (query slots r and 128 + r) after the last block
+          if (wg == 2) {
+            if (b == 3)
+              for (int x = 0; x < 2; ++x)
+                store_acc_rows<HD>(tl + kColDQ + 64 * x,
+                                   ok && (((x ? slotw[1] : slotw[0]) >> 21) & 1), slot_token(x),
+                                   (__nv_bfloat16*)p.out0, g.heads, h, dscale);
+          } else {
+            const uint32_t ew = ek ? slotw[1] : slotw[0];
+            const bool k_st = ok && ((ew >> 21) & 1);
+            const long long k_tok = slot_token(ek);
+            if (wg == 0)
+              store_acc_rows<HD>(tl + kColDV, k_st, k_tok, (__nv_bfloat16*)p.out2, g.heads, h, 1.f);
+            else
+              store_acc_rows<HD>(tl + kColDK, k_st, k_tok, (__nv_bfloat16*)p.out1, g.heads, h,
+                                 dscale);
+          }
           tc_fence_before();
           mbar_arrive(b == 2 ? acc_free : t_free);
         }
@@ -1036,7 +1044,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kWideMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
