@@ -419,11 +419,13 @@ __host__ __device__ inline int bias_copy_stride(int bins_pad) { return bins_pad 
 constexpr uint32_t kColDP1 = 256;                    // phase 1 dP (S at 0)
 constexpr uint32_t kColDPT = 128;                    // phase 2 dP^T (S^T at 0)
 constexpr uint32_t kColDV = 256, kColDK = 320, kColDQ = 384;
-// Backward warps: three softmax warpgroups (0-11), the TMA producer, the MMA
-// issuer and the bin fold. Fifteen warps leave 128 registers a thread.
-constexpr int kWideBwdWarps = 15;
-constexpr int kWideSoftWg = 3;
-constexpr int kWideProducerWarp = 12, kWideMmaWarp = 13, kWideFoldWarp = 14;
+// Backward warps: four softmax warpgroups (0-15), the TMA producer, the MMA
+// issuer and the bin fold. Nineteen warps leave 96 registers a thread, which
+// the one-buffer chunk loops fit.
+constexpr int kWideSoftWg = 4;
+constexpr int kWideBwdWarps = kWideSoftWg * 4 + 3;
+constexpr int kWideProducerWarp = kWideSoftWg * 4, kWideMmaWarp = kWideProducerWarp + 1,
+              kWideFoldWarp = kWideProducerWarp + 2;
 
 struct WideBwdLayout {
   uint32_t tiles, dsop, bias, colinfo, stats, xch, bins, wb, bars, misc, total;
@@ -435,9 +437,9 @@ __host__ __device__ inline WideBwdLayout wide_bwd_layout(int bins_pad) {
   WideBwdLayout L;
   L.tiles = 0;
   L.dsop = L.tiles + C::kStages * 4 * C::kTileBytes;
-  L.xch = L.dsop;                            // [qt][2][4][128] partial statistics of
-                                             // warpgroups 1 and 2 (phase 1 only: the
-                                             // dQ operand is free then)
+  L.xch = L.dsop;                            // [qt][warpgroup - 1][4][128] partial
+                                             // statistics (phase 1 only: the dQ
+                                             // operand is free then)
   L.bias = L.dsop + C::kOpBytes;
   L.colinfo = L.bias + C::kStages * 4 * bias_copy_stride(bins_pad) * 4;
   L.stats = L.colinfo + kKeys * 4;           // float2 {L, D} per query
@@ -932,7 +934,7 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
                                 p.scale_log2, M, l, d, a);
         tc_fence_before();
         mbar_arrive(t1_empty);
-        float* xq = xch + qt * 2 * 4 * kRows;   // [warpgroup - 1][M, l, d, a][row]
+        float* xq = xch + qt * (kWideSoftWg - 1) * 4 * kRows;   // [wg - 1][M, l, d, a][row]
         if (wg > 0) {
           float* xw = xq + (wg - 1) * 4 * kRows;
           xw[r] = M;
@@ -942,12 +944,21 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
         }
         named_sync(1, kSoft);
         if (wg == 0) {
-          const float M1 = xq[r], l1 = xq[kRows + r], d1 = xq[2 * kRows + r];
-          const float M2 = xq[4 * kRows + r], l2 = xq[5 * kRows + r], d2 = xq[6 * kRows + r];
-          const float a1 = fmaxf(xq[3 * kRows + r], xq[7 * kRows + r]);
-          const float Mx = fmaxf(M, fmaxf(M1, M2));
-          const float f0 = ex2(M - Mx), f1 = ex2(M1 - Mx), f2 = ex2(M2 - Mx);
-          const float lt = l * f0 + l1 * f1 + l2 * f2, dt = d * f0 + d1 * f1 + d2 * f2;
+          float Mx = M, a1 = 0.f;
+#pragma unroll
+          for (int w = 1; w < kWideSoftWg; ++w) {
+            Mx = fmaxf(Mx, xq[(w - 1) * 4 * kRows + r]);
+            a1 = fmaxf(a1, xq[(w - 1) * 4 * kRows + 3 * kRows + r]);
+          }
+          const float f0 = ex2(M - Mx);
+          float lt = l * f0, dt = d * f0;
+#pragma unroll
+          for (int w = 1; w < kWideSoftWg; ++w) {
+            const float* xw = xq + (w - 1) * 4 * kRows;
+            const float f = ex2(xw[r] - Mx);
+            lt = fmaf(xw[kRows + r], f, lt);
+            dt = fmaf(xw[2 * kRows + r], f, dt);
+          }
           float2 st = make_float2(INFINITY, 0.f);   // not a real token: P = 0
           if (q_valid) {
             const float inv = 1.f / lt;
@@ -1017,14 +1028,15 @@ __global__ void __launch_bounds__(kWideBwdWarps * 32, 1)
           mbar_wait(grad_done, (uint32_t)(eb & 1), abort, p.status, kWaitLimitNs);
           tc_fence_after();
           const bool ok = !*abort;
-          // warpgroup 0: dV rows, 1: dK rows (key slots), 2: dQ rows of both
-          // query halves (query slots r and 128 + r) after the last block
-          if (wg == 2) {
-            if (b == 3)
-              for (int x = 0; x < 2; ++x)
-                store_acc_rows<HD>(tl + kColDQ + 64 * x,
-                                   ok && (((x ? slotw[1] : slotw[0]) >> 21) & 1), slot_token(x),
-                                   (__nv_bfloat16*)p.out0, g.heads, h, dscale);
+          // warpgroup 0: dV rows, 1: dK rows (key slots); after the last block
+          // warpgroups 2 and 3 the dQ rows of query halves 0 and 1 (query slots
+          // r and 128 + r)
+          if (wg >= 2) {
+            if (b == 3) {
+              const int x = wg - 2;
+              store_acc_rows<HD>(tl + kColDQ + 64 * x, ok && (((x ? slotw[1] : slotw[0]) >> 21) & 1),
+                                 slot_token(x), (__nv_bfloat16*)p.out0, g.heads, h, dscale);
+            }
           } else {
             const uint32_t ew = ek ? slotw[1] : slotw[0];
             const bool k_st = ok && ((ew >> 21) & 1);
