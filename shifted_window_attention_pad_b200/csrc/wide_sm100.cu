@@ -33,7 +33,13 @@ using namespace ptx;
 
 constexpr int kKeys = 256;                 // tokens of a window = keys of every row
 constexpr int kHalves = kKeys / kRows;     // query halves per window
-constexpr int kWideThreads = 352;          // 11 warps
+// Forward warps: four softmax warpgroups (query half hf, key half kh =
+// warpgroup >> 1, & 1), the TMA producer, the S issuer, the O issuer: 19
+// warps, 96 registers a thread.
+constexpr int kWideFwdWg = 4;
+constexpr int kWideThreads = (kWideFwdWg * 4 + 3) * 32;
+constexpr int kWideFwdProducer = kWideFwdWg * 4, kWideFwdMma = kWideFwdProducer + 1,
+              kWideFwdMma2 = kWideFwdProducer + 2;
 constexpr uint32_t kSlotColsW = 256;       // TMEM columns of one half
 
 template <int HD>
@@ -41,15 +47,17 @@ struct WideFwdCfg {
   static constexpr uint32_t kRowBytes = HD * 2;
   static constexpr uint32_t kTileBytes = kKeys * kRowBytes;   // one tensor of one item
   static constexpr int kStages = HD > 32 ? 2 : 4;
-  static constexpr uint32_t kOCol = 128;                       // O inside a half's slot
+  static constexpr uint32_t kOCol = 64;                        // O inside a half's slot
 };
 
 struct WideLayout {
-  uint32_t tiles, bias, colinfo, bars, misc, total;
+  uint32_t tiles, bias, colinfo, xch, bars, misc, total;
 };
 
 // NS stages of three [256][HD] tiles (Q, K, V), the stages' bias rows, per
-// warpgroup two buffers of 256 key words, mbarriers, two words.
+// query half two buffers of 256 key words, the row maxima and sums the two
+// key-half warpgroups of a row exchange ([max, sum][half][key half][row]),
+// mbarriers, two words.
 template <int HD>
 __host__ __device__ inline WideLayout wide_fwd_layout(int bins_pad) {
   using C = WideFwdCfg<HD>;
@@ -57,7 +65,8 @@ __host__ __device__ inline WideLayout wide_fwd_layout(int bins_pad) {
   L.tiles = 0;
   L.bias = L.tiles + C::kStages * 3 * C::kTileBytes;
   L.colinfo = L.bias + ((C::kStages * bins_pad * 4 + 15) & ~15);
-  L.bars = (L.colinfo + kHalves * 2 * kKeys * 4 + 7) & ~7u;
+  L.xch = L.colinfo + kHalves * 2 * kKeys * 4;
+  L.bars = (L.xch + 2 * kHalves * 2 * kRows * 4 + 7) & ~7u;
   L.misc = L.bars + 8 * 32;
   L.total = L.misc + 16;
   return L;
@@ -119,35 +128,19 @@ __device__ inline float chunk_logits_plain(float* x, const float* bias_q, int k0
   return fmaxf(m0, m1);
 }
 
-// The row's 256 columns in chunks of 32, two register buffers: the TMEM load
-// of chunk c + 1 is in flight while chunk c is worked on.
-template <typename F>
-__device__ inline void for_row_chunks(uint32_t slot, F&& work) {
-  float xa[32], xb[32];
-  __syncwarp();
-  tmem_ld32(slot, xa);
-#pragma unroll 1
-  for (int k0 = 0; k0 < kKeys; k0 += 64) {
-    tmem_wait_ld_regs(xa);
-    __syncwarp();
-    tmem_ld32(slot + k0 + 32, xb);
-    work(xa, k0);
-    tmem_wait_ld_regs(xb);
-    if (k0 + 64 < kKeys) {
-      __syncwarp();
-      tmem_ld32(slot + k0 + 64, xa);
-    }
-    work(xb, k0 + 32);
-  }
-}
-
-// Pass 1 over a row of 256 keys: logits (scale, bias, mask) written back over
-// S in TMEM; returns the row maximum.
+// Pass 1 over the 128 keys k0base .. k0base + 127 of a row (32 at a time):
+// logits (scale, bias, mask) written back over S in TMEM; returns their
+// maximum.
 template <bool PLAIN, int WW>
-__device__ inline float wide_pass1(uint32_t slot, const float* brow, const uint32_t* ci,
-                                   const RowInfo& me, float c) {
+__device__ inline float wide_pass1(uint32_t slot, int k0base, const float* brow,
+                                   const uint32_t* ci, const RowInfo& me, float c) {
   float m = -INFINITY;
-  for_row_chunks(slot, [&](float* x, int k0) {
+#pragma unroll 1
+  for (int k0 = k0base; k0 < k0base + kRows; k0 += 32) {
+    float x[32];
+    __syncwarp();
+    tmem_ld32(slot + k0, x);
+    tmem_wait_ld_regs(x);
     float cm;
     if constexpr (PLAIN)
       cm = chunk_logits_plain<WW>(x, brow + me.bias_base, k0, c);
@@ -156,16 +149,22 @@ __device__ inline float wide_pass1(uint32_t slot, const float* brow, const uint3
     m = fmaxf(m, cm);
     __syncwarp();
     tmem_st32(slot + k0, x);
-  });
+  }
   return m;
 }
 
-// Pass 2: P = 2^(x - mo) as bf16 pairs over columns 0-127 (pair columns
-// k0/2 .. k0/2 + 15 come from keys k0 .. k0 + 31, whose logits columns were
-// read before they are overwritten); returns the row sum.
-__device__ inline float wide_pass2(uint32_t slot, float mo) {
+// Pass 2 over the same keys: P = 2^(x - mo) as bf16 pairs, the pair of keys
+// k0base + 2c, + 1 in column k0base + c (keys 32 i .. 32 i + 31 of the half
+// give columns 16 i .. 16 i + 15, whose logits were read before they are
+// overwritten); returns the sum.
+__device__ inline float wide_pass2(uint32_t slot, int k0base, float mo) {
   float l = 0.f;
-  for_row_chunks(slot, [&](float* x, int k0) {
+#pragma unroll 1
+  for (int i = 0; i < kRows / 32; ++i) {
+    float x[32];
+    __syncwarp();
+    tmem_ld32(slot + k0base + 32 * i, x);
+    tmem_wait_ld_regs(x);
     uint32_t w[16];
     float2 l2 = make_float2(0.f, 0.f);
     const float2 nm = make_float2(-mo, -mo);
@@ -178,8 +177,8 @@ __device__ inline float wide_pass2(uint32_t slot, float mo) {
     }
     l += l2.x + l2.y;
     __syncwarp();
-    tmem_st16u(slot + k0 / 2, w);
-  });
+    tmem_st16u(slot + k0base + 16 * i, w);
+  }
   return l;
 }
 
@@ -196,6 +195,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   uint8_t* tiles = smem + L.tiles;
   float* bias = (float*)(smem + L.bias);
   uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
+  float* xch = (float*)(smem + L.xch);
   uint64_t* bars = (uint64_t*)(smem + L.bars);
   uint64_t* full = bars;
   uint64_t* empty = full + NS;
@@ -213,8 +213,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < kHalves; ++i) {
-      mbar_init(&s_full[i], 1); mbar_init(&p_full[i], kWg);
-      mbar_init(&o_full[i], 1); mbar_init(&t_empty[i], kWg);
+      mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 2 * kWg);
+      mbar_init(&o_full[i], 1); mbar_init(&t_empty[i], 2 * kWg);
     }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
@@ -222,10 +222,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == kProducerWarp && lane == 0)
+  if (warp == kWideFwdProducer && lane == 0)
     for (int tt = 0; tt < 3; ++tt)
       for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
-  if (warp == kMmaWarp) {
+  if (warp == kWideFwdMma) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kProducerWarp) {
+  if (warp == kWideFwdProducer) {
     if (lane == 0) {
       long long k = 0;
       for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           mbar_drain(&full[j % NS], (uint32_t)((j / NS) & 1), kTestLimitNs * 100);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kWideFwdMma) {
     if (lane == 0) {   // S = Q_half K^T of both halves of every item
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kKeys, 0, 0);
       bool ok = true;
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         mbar_drain(&drain[0], 0, kTestLimitNs * 100);
       }
     }
-  } else if (warp == kMma2Warp) {
+  } else if (warp == kWideFwdMma2) {
     if (lane == 0) {   // O = P V of both halves, as soon as each P is written
       constexpr uint32_t idesc_o = idesc_bf16(kRows, HD, 0, 1);
       bool ok = true;
@@ -294,10 +294,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           }
           tc_fence_after();
           const uint32_t slot = tmem + hf * kSlotColsW;
-          // A = P from TMEM: 16 keys per step are 8 columns of bf16 pairs
+          // A = P from TMEM: 16 keys per step are 8 columns of bf16 pairs, key
+          // half 0 in columns 0-63, key half 1 in 128-191
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk)
-            umma_ts(slot + C::kOCol, slot + kk * 8, wdesc_mnmajor<HD>(v_s, kk), idesc_o, kk);
+            umma_ts(slot + C::kOCol, slot + (kk >> 3) * kRows + (kk & 7) * 8,
+                    wdesc_mnmajor<HD>(v_s, kk), idesc_o, kk);
           umma_commit(&o_full[hf]);
         }
         if (ok) umma_commit(&empty[s]);
@@ -307,15 +309,20 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         mbar_drain(&drain[1], 0, kTestLimitNs * 100);
       }
     }
-  } else if (warp < kHalves * 4) {
-    // Softmax / epilogue: warpgroup hf holds query rows 128 hf .. 128 hf + 127
-    // of every item; thread = row = TMEM lane.
-    const int hf = warp >> 2;
+  } else if (warp < kWideFwdWg * 4) {
+    // Softmax / epilogue: warpgroup wg holds query rows 128 hf .. 128 hf + 127
+    // (hf = wg >> 1) of every item and their keys 128 kh .. 128 kh + 127
+    // (kh = wg & 1); thread = row = TMEM lane. The two key halves of a row
+    // exchange their maxima and sums through shared memory.
+    const int wg = warp >> 2, hf = wg >> 1, kh = wg & 1;
     const int row = threadIdx.x & (kWg - 1);
     const int lr = hf * kRows + row;               // query slot in the window
     const int lo = (1 - hf) * kRows + row;         // the other half's slot
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t slot = tmem + lane_base + hf * kSlotColsW;
+    float* xm = xch + (hf * 2 + kh) * kRows;                  // this thread's maximum, sum
+    float* xm_o = xch + (hf * 2 + (1 - kh)) * kRows;          // the other key half's
+    constexpr int kSumOff = kHalves * 2 * kRows;
     for (long long k = 0; k < n_local; ++k) {
       const long long t = blockIdx.x + k * (long long)gridDim.x;
       const int s = (int)(k % NS);
@@ -326,50 +333,60 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       const RowInfo me = plain ? plain_row_info<(WW > 0 ? WW : 16)>(g, win, lr)
                                : row_info(g, win, lr);
       uint32_t* ci = colinfo + (hf * 2 + (int)(k & 1)) * kKeys;
-      if (!plain) {
-        ci[lr] = key_word(me);
-        ci[lo] = key_word(row_info(g, win, lo));
+      if (!plain) {   // key words of the half's two slots per row: one each
+        if (kh == 0) ci[lr] = key_word(me);
+        else ci[lo] = key_word(row_info(g, win, lo));
       }
-      if (named_sync_or(1 + hf, kWg, *abort)) break;
+      if (named_sync_or(1 + hf, 2 * kWg, *abort)) break;
       if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
       mbar_wait(&s_full[hf], pht, abort, p.status, kWaitLimitNs);
       mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
       tc_fence_after();
       const float* brow = bias + s * p.bins_pad;
-      // pass 1: logits written back over S, row maximum (the window kind
-      // decides the code path once per item, not per chunk)
+      // pass 1: logits written back over S, maximum of this key half (the
+      // window kind decides the code path once per item, not per chunk)
       float m;
       if (WW > 0 && plain)
-        m = wide_pass1<true, (WW > 0 ? WW : 16)>(slot, brow, ci, me, p.scale_log2);
+        m = wide_pass1<true, (WW > 0 ? WW : 16)>(slot, kh * kRows, brow, ci, me, p.scale_log2);
       else
-        m = wide_pass1<false, 16>(slot, brow, ci, me, p.scale_log2);
+        m = wide_pass1<false, 16>(slot, kh * kRows, brow, ci, me, p.scale_log2);
+      xm[row] = m;
       tmem_wait_st();
-      // pass 2: P over columns 0-127; a row that is not a real token
-      // subtracts +inf instead of its maximum, so its P is zero without a select
-      const float l = wide_pass2(slot, me.valid ? m : INFINITY);
+      named_sync(1 + hf, 2 * kWg);
+      m = fmaxf(m, xm_o[row]);
+      // pass 2: P of this key half; a row that is not a real token subtracts
+      // +inf instead of its maximum, so its P is zero without a select
+      float l = wide_pass2(slot, kh * kRows, me.valid ? m : INFINITY);
+      xm[kSumOff + row] = l;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[hf]);
-      // epilogue: O row from TMEM, normalised, straight to its grid token
+      named_sync(1 + hf, 2 * kWg);
+      l += xm_o[kSumOff + row];
+      // epilogue: this key half's warpgroup stores columns (HD / 2) kh .. of
+      // the O row, normalised, straight to its grid token
       mbar_wait(&o_full[hf], pht, abort, p.status, kWaitLimitNs);
       tc_fence_after();
       {
+        constexpr int OC = HD / 2;
         const float inv = me.valid ? 1.f / l : 0.f;
-        __nv_bfloat16* dst = (__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD;
-        float o[HD];
-        tmem_load_cols<HD>(slot + C::kOCol, o);
+        __nv_bfloat16* dst = (__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD + OC * kh;
+        float o[OC];
+        __syncwarp();
+        if constexpr (OC == 16) tmem_ld16(slot + C::kOCol + OC * kh, o);
+        else tmem_ld32(slot + C::kOCol + OC * kh, o);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&t_empty[hf]);
-        if (me.stored && !*abort) store_row_bf16<HD>(dst, o, inv);
+        if (me.stored && !*abort) store_row_bf16<OC>(dst, o, inv);
       }
-      if (me.stored && !*abort && p.lse)
+      if (kh == 0 && me.stored && !*abort && p.lse)
         p.lse[me.token * g.heads + h] = me.valid ? (m + __log2f(l)) * 0.69314718055994531f : 0.f;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kWideFwdMma) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
