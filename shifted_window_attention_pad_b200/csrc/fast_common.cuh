@@ -74,10 +74,11 @@ struct Layout {
 };
 
 // NS stages of NTEN input tiles, then PBYTES of P / dS operand blocks, the
-// bias rows of the stages, per warpgroup two buffers of key words, int32
-// bias-gradient bins per warp (two warps hold a window's rows) and four
-// per-warp bounds, mbarriers and two words (TMEM base, abort flag).
-template <int HD, int NS, int NTEN, uint32_t PBYTES>
+// bias rows of the stages, NCOLBUF buffers of key words, int32 bias-gradient
+// bins per warp of NBINWG warpgroups (two warps hold a window's rows) and four
+// per-warp bounds each, mbarriers and two words (TMEM base, abort flag).
+template <int HD, int NS, int NTEN, uint32_t PBYTES, int NCOLBUF = 2 * kNumWg,
+          int NBINWG = kNumWg>
 __host__ __device__ inline Layout make_layout(int bins_pad) {
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   Layout L;
@@ -85,15 +86,19 @@ __host__ __device__ inline Layout make_layout(int bins_pad) {
   L.ptile = L.tiles + NS * NTEN * tile_bytes;
   L.bias = L.ptile + PBYTES;
   L.colinfo = L.bias + ((NS * bins_pad * 4 + 15) & ~15);
-  L.bins_w = L.colinfo + kNumWg * 2 * kRows * 4;
-  L.bars = (L.bins_w + kNumWg * (4 * bins_pad + 4) * 4 + 7) & ~7u;
+  L.bins_w = L.colinfo + NCOLBUF * kRows * 4;
+  L.bars = (L.bins_w + NBINWG * (4 * bins_pad + 4) * 4 + 7) & ~7u;
   L.misc = L.bars + 8 * 32;
   L.total = L.misc + 16;
   return L;
 }
 
 // Rows of the 128-row tile are windows g = row / N; inside a window the rows
-// follow the sub-boxes in order (y segment, x segment), each row-major.
+// follow the sub-boxes column segment first (x segment, then y segment), each
+// row-major -- so within a column segment the window's rows come in their
+// natural order whether or not the window wraps at the row seam. A row band
+// changes only the wrapping of rows, so a window keeps its slot order (and a
+// row's sums add its keys in the same order) in a band and in the whole grid.
 struct SubBox {
   int y, x, rows, cols, map_id, row_off;
 };
@@ -125,8 +130,8 @@ __device__ inline int plan_window(const Geo& g, int wy, int wx, SubBox* sb) {
     xs[0] = 0; xl[0] = g.ww; xk[0] = 0;
   }
   int n = 0, off = 0;
-  for (int a = 0; a < ny; ++a)
-    for (int c = 0; c < nx; ++c) {
+  for (int c = 0; c < nx; ++c)
+    for (int a = 0; a < ny; ++a) {
       sb[n].y = (wy * g.wh + ys[a] + g.sh) % g.Hp;
       sb[n].x = (wx * g.ww + xs[c] + g.sw) % g.Wp;
       sb[n].rows = yl[a];
@@ -139,22 +144,16 @@ __device__ inline int plan_window(const Geo& g, int wy, int wx, SubBox* sb) {
   return n;
 }
 
-// Slot coordinates (iy, ix) of row r (0..N-1) of window (wy, wx) in sub-box order.
+// Slot coordinates (iy, ix) of row r (0..N-1) of window (wy, wx) in sub-box
+// order: column segments of w0 and ww - w0 columns, each all wh rows in order.
 __device__ inline void row_slot(const Geo& g, int wy, int wx, int r, int& iy, int& ix) {
-  const bool wrap_y = g.sh > 0 && wy == g.nWy - 1;
   const bool wrap_x = g.sw > 0 && wx == g.nWx - 1;
-  const int h0 = wrap_y ? g.wh - g.sh : g.wh;
   const int w0 = wrap_x ? g.ww - g.sw : g.ww;
-  const int top = h0 * g.ww;
-  const int yseg = r >= top;
-  const int rr = yseg ? r - top : r;
-  const int yh = yseg ? g.wh - h0 : h0;
-  const int xseg = rr >= yh * w0;
-  const int r2 = xseg ? rr - yh * w0 : rr;
+  const int xseg = r >= g.wh * w0;
+  const int rr = xseg ? r - g.wh * w0 : r;
   const int wseg = xseg ? g.ww - w0 : w0;
-  const int ly = r2 / wseg;
-  iy = (yseg ? h0 : 0) + ly;
-  ix = (xseg ? w0 : 0) + (r2 - ly * wseg);
+  iy = rr / wseg;
+  ix = (xseg ? w0 : 0) + (rr - iy * wseg);
 }
 
 // Everything the softmax warpgroup needs to know about its own row.
@@ -563,11 +562,12 @@ void fill_common(FastParams& p, const Geo& g, const float* bias_t, int* status, 
 }
 
 template <typename K>
-cudaError_t launch(K kernel, const FastParams& p, size_t smem, cudaStream_t st) {
+cudaError_t launch(K kernel, const FastParams& p, size_t smem, cudaStream_t st,
+                   int threads = kThreads) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
-  kernel<<<(unsigned)(grid > 0 ? grid : 1), kThreads, smem, st>>>(p);
+  kernel<<<(unsigned)(grid > 0 ? grid : 1), threads, smem, st>>>(p);
   note_launch();
   return cudaGetLastError();
 }

@@ -332,12 +332,22 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 // three 128-column gradients need
 // 384 columns, so one slot (dV | dQ | dK at 0 / 128 / 256 over S | dP) and
 // one softmax warpgroup.
+// HD <= 64 also splits every row's 64 keys between two warpgroups (32 each):
+// four softmax warpgroups, two per tile in flight, 20 warps at 96 registers a
+// thread. The two halves of a row exchange their maxima, sums, D and max |dP|
+// through TMEM columns of the other window's S, which that row never reads.
 template <int HD>
 struct BwdCfg {
   static constexpr bool kWide = HD > 64;
   static constexpr int kStages = kWide ? 1 : 2;
   static constexpr int kSlots = kWide ? 1 : 2;
-  static constexpr int kWarpgroups = kWide ? 1 : kNumWg;
+  static constexpr int kWarpgroups = kWide ? 1 : kNumWg;    // tiles in flight
+  static constexpr int kKeySplit = kWide ? 1 : 2;           // warpgroups per tile
+  static constexpr int kSoftWg = kWarpgroups * kKeySplit;
+  static constexpr int kProducer = kSoftWg > 2 ? kSoftWg * 4 : kProducerWarp;
+  static constexpr int kMma = kProducer + 1, kMma2 = kProducer + 2, kFold = kProducer + 3;
+  static constexpr int kThreads = (kProducer + 4) * 32;
+  static constexpr int kColBufs = kKeySplit > 1 ? kWarpgroups : 2 * kWarpgroups;
   static constexpr uint32_t kGradCols = kWide ? 128 : 64;   // dV, dQ, dK spacing
 };
 constexpr uint32_t kBlk = 8192;
@@ -381,23 +391,26 @@ __device__ inline void store_split_cols_part(uint32_t blk_hi, uint32_t blk_lo, i
 }
 
 template <int HD, int WW>
-__global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ FastParams p) {
+__global__ void __launch_bounds__(BwdCfg<HD>::kThreads, 1)
+    bwd_kernel(const __grid_constant__ FastParams p) {
   constexpr int N = 64, G = kRows / N;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   using C = BwdCfg<HD>;
   constexpr int NS = C::kStages, NT = C::kSlots, NWG = C::kWarpgroups;
+  constexpr int KS = C::kKeySplit, SW = C::kSoftWg;
+  constexpr int KN = 64 / KS;   // keys of a row each thread takes
   constexpr uint32_t GC = C::kGradCols;
   constexpr uint32_t tile_bytes = kRows * HD * 2;
   const Geo& g = p.g;
   const int bp = p.bins_pad;
-  const Layout L = make_layout<HD, NS, 4, kNumBlk * kBlk>(bp);
+  const Layout L = make_layout<HD, NS, 4, kNumBlk * kBlk, C::kColBufs, SW>(bp);
   uint8_t* tiles = smem + L.tiles;
   uint8_t* blocks = smem + L.ptile;
   float* bias = (float*)(smem + L.bias);
   uint32_t* colinfo = (uint32_t*)(smem + L.colinfo);
   int* bins = (int*)(smem + L.bins_w);               // [wg][warp][bins_pad] bins
-  float* tbound = (float*)(bins + kNumWg * 4 * bp);  // [wg][4] per-warp |dS| bounds
+  float* tbound = (float*)(bins + SW * 4 * bp);      // [wg][4] per-warp |dS| bounds
   uint64_t* bars = (uint64_t*)(smem + L.bars);
   uint64_t* full = bars;
   uint64_t* empty = full + NS;
@@ -409,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint64_t* never = drain + 2;
   uint64_t* gradv_full = never + 1;          // [NT] dV products done
   uint64_t* bins_full = gradv_full + NT;     // [wg] a tile's bins are complete
-  uint64_t* bins_empty = bins_full + kNumWg; // [wg] ... and folded into global sums
+  uint64_t* bins_empty = bins_full + NWG;    // [pair] ... and folded into global sums
   uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
   volatile int* abort = (volatile int*)(smem + L.misc + 4);
 
@@ -418,27 +431,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < NT; ++i) {
-      mbar_init(&sdp_full[i], 1); mbar_init(&pds_full[i], kWg);
-      mbar_init(&grad_full[i], 1); mbar_init(&t_empty[i], kWg);
+      mbar_init(&sdp_full[i], 1); mbar_init(&pds_full[i], KS * kWg);
+      mbar_init(&grad_full[i], 1); mbar_init(&t_empty[i], KS * kWg);
       mbar_init(&gradv_full[i], 1);
     }
-    for (int i = 0; i < kNumWg; ++i) { mbar_init(&bins_full[i], kWg); mbar_init(&bins_empty[i], 32); }
+    for (int i = 0; i < NWG; ++i) { mbar_init(&bins_full[i], KS * kWg); mbar_init(&bins_empty[i], 32); }
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     mbar_init(never, 1);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == kProducerWarp && lane == 0)
+  if (warp == C::kProducer && lane == 0)
     for (int tt = 0; tt < 4; ++tt)
       for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
-  for (uint32_t i = threadIdx.x; i < kBlk / 16; i += kThreads) {
+  for (uint32_t i = threadIdx.x; i < kBlk / 16; i += C::kThreads) {
     reinterpret_cast<uint4*>(blocks + kZ1 * kBlk)[i] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(blocks + kZ2 * kBlk)[i] = make_uint4(0, 0, 0, 0);
   }
-  for (int i = threadIdx.x; i < kNumWg * 4 * bp; i += kThreads) bins[i] = 0;
+  for (int i = threadIdx.x; i < SW * 4 * bp; i += C::kThreads) bins[i] = 0;
   fence_proxy_async();
-  if (warp == kMmaWarp) {
+  if (warp == C::kMma) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -447,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kProducerWarp) {
+  if (warp == C::kProducer) {
     if (lane == 0) {
       long long k = 0;
       for (long long t = blockIdx.x; t < p.n_tiles; t += gridDim.x, ++k) {
@@ -463,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           mbar_drain(&full[j % NS], (uint32_t)((j / NS) & 1), kTestLimitNs * 100);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == C::kMma) {
     if (lane == 0) {   // S = Q K^T and dP = dO V^T of every tile
       constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);
       for (long long k = 0; k < n_local; ++k) {
@@ -492,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         mbar_drain(&drain[0], 0, kTestLimitNs * 100);
       }
     }
-  } else if (warp == kMma2Warp) {
+  } else if (warp == C::kMma2) {
     if (lane == 0) {   // dV, dQ, dK of every tile, once its operand blocks are written
       constexpr uint32_t idesc_t = idesc_bf16(kRows, HD, 1, 1);         // dV, dK: A = X^T
       constexpr uint32_t idesc_q = idesc_bf16(kRows, HD, 0, 1);         // dQ
@@ -548,34 +561,41 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         mbar_drain(&drain[1], 0, kTestLimitNs * 100);
       }
     }
-  } else if (warp == kFoldWarp) {
-    // Each tile's bins, per warp, into the workspace's exact sums: the two
-    // warps of a window add up (exact integers), in the window's own unit.
+  } else if (warp == C::kFold) {
+    // Each tile's bins, per warp, into the workspace's exact sums: the warps
+    // of a window (two per warpgroup of the tile) add up (exact integers), in
+    // the window's own unit.
     for (long long k = 0, t = blockIdx.x; k < n_local; ++k, t += gridDim.x) {
       const int wgk = (int)(k % NWG);
       if (!mbar_wait(&bins_full[wgk], (uint32_t)((k / NWG) & 1), abort, p.status, kWaitLimitNs))
         break;
       const int h = (int)(t - (t / g.heads) * g.heads);
-      int* tbk = bins + wgk * 4 * bp;
-      const float* bk = tbound + wgk * 4;
+      int* tbk = bins + wgk * KS * 4 * bp;
+      const float* bk = tbound + wgk * KS * 4;   // (the key parts' bounds are equal)
       long long* acc = p.dt_acc + (size_t)h * bp * kLimbStride;
       for (int i = lane; i < 2 * g.bins; i += 32) {
         const int w2 = i >= g.bins;
         const int b = i - (w2 ? g.bins : 0);
         const float wbd = fmaxf(bk[2 * w2], bk[2 * w2 + 1]);
         const bool fin = wbd <= 3.0e38f;
-        int* b0 = tbk + (2 * w2) * bp + b;
-        int* b1 = b0 + bp;
-        const int v = *b0 + *b1;
-        *b0 = 0;
-        *b1 = 0;
+        int v = 0;
+#pragma unroll
+        for (int kh = 0; kh < KS; ++kh) {
+          int* b0 = tbk + (kh * 4 + 2 * w2) * bp + b;
+          v += b0[0] + b0[bp];
+          b0[0] = 0;
+          b0[bp] = 0;
+        }
         if (!fin) flag_nonfinite(acc + (size_t)b * kLimbStride);
         else if (v != 0) add_fixed(acc + (size_t)b * kLimbStride, v, tile_exponent(wbd));
       }
       mbar_arrive(&bins_empty[wgk]);
     }
-  } else if (warp < NWG * 4) {
-    const int wg = warp >> 2;
+  } else if (warp < SW * 4) {
+    const int wgi = warp >> 2;       // softmax warpgroup
+    const int wg = wgi / KS;         // tile pair: takes tiles wg, wg + NWG, ...
+    const int kh = wgi - wg * KS;    // keys kh * KN .. kh * KN + KN - 1 of every row
+    const int k0 = kh * KN;
     const int row = threadIdx.x & (kWg - 1);
     const int gw = row / N, lr = row - gw * N;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -583,8 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const uint32_t bb = smem_u32(blocks);
     const uint32_t blk_ph = bb + (gw ? kP1h : kP0h) * kBlk, blk_pl = bb + (gw ? kP1l : kP0l) * kBlk;
     const uint32_t blk_sh = bb + (gw ? kS1h : kS0h) * kBlk, blk_sl = bb + (gw ? kS1l : kS0l) * kBlk;
-    int* tb = bins + (wg * 4 + (warp & 3)) * bp;   // this warp's bins
-    float* bnd = tbound + wg * 4;
+    int* tb = bins + (wgi * 4 + (warp & 3)) * bp;   // this warp's bins
+    float* bnd = tbound + wgi * 4;
     __nv_bfloat16* const outs[3] = {(__nv_bfloat16*)p.out2, (__nv_bfloat16*)p.out0,
                                     (__nv_bfloat16*)p.out1};   // TMEM order: dV, dQ, dK
     __nv_bfloat16* const outs_h[3] = {(__nv_bfloat16*)p.out2h, (__nv_bfloat16*)p.out0h,
@@ -599,9 +619,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const long long win = group * G + gw;
       const bool plain = WW > 0 && window_plain(g, win);
       const RowInfo me = plain ? plain_row_info<WW>(g, win, lr) : row_info(g, win, lr);
-      uint32_t* ci = colinfo + (wg * 2 + ((k / NWG) & 1)) * kRows;
-      ci[row] = key_word(me);
-      if (named_sync_or(1 + wg, kWg, *abort)) break;
+      // key words: one buffer per tile pair when the keys are split (the
+      // exchange barrier below keeps a fast warp's next words behind every
+      // read of these), two otherwise
+      uint32_t* ci = colinfo + (KS > 1 ? wg : (wg * 2 + (int)((k / NWG) & 1))) * kRows;
+      if (kh == 0) ci[row] = key_word(me);
+      if (named_sync_or(1 + wg, KS * kWg, *abort)) break;
       if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
       mbar_wait(&sdp_full[sl], pht, abort, p.status, kWaitLimitNs);
       mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
@@ -609,65 +632,96 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       // S row -> P (registers) -> D from dP; P back into its S columns; dS and
       // the bias-gradient bins from P and dP chunks; scale * dS into the dP
       // columns. All of this runs before the shared operand blocks are free.
-      float x[N];
-      const uint32_t s_col = tmem + lane_base + sl * 256 + gw * N;
+      float x[KN];
+      const uint32_t s_col = tmem + lane_base + sl * 256 + gw * N + k0;
       const uint32_t dp_col = s_col + 128;
-      tmem_load_cols<N>(s_col, x);
+      // (exchange columns: the other window's S in this row's lane)
+      const uint32_t x_col = tmem + lane_base + sl * 256 + (1 - gw) * N;
+      tmem_load_cols<KN>(s_col, x);
       tmem_wait_ld();
       const float* brow = bias + s * bp;
-      const uint32_t* cw = ci + gw * N;
+      const uint32_t* cw = ci + gw * N + k0;
       float m;
       if (plain)
-        m = logits_plain<N, (WW > 0 ? WW : 8)>(x, brow + me.bias_base, p.scale_log2);
+        m = logits_plain<KN, (WW > 0 ? WW : 8)>(x, brow + me.bias_base - plain_off<(WW > 0 ? WW : 8)>(k0),
+                                                p.scale_log2);
       else
-        m = logits_general<N>(x, brow, cw, me.bias_base, me.label, p.scale_log2);
-      float inv = 0.f;   // max_j P_ij (= 1 / row sum); 0 on pad rows
+        m = logits_general<KN>(x, brow, cw, me.bias_base, me.label, p.scale_log2);
+      if constexpr (KS > 1) {   // the row's maximum over both key parts
+        tmem_st4(x_col + 4 * kh, m, 0.f, 0.f, 0.f);
+        tmem_wait_st();
+        tc_fence_before();
+        named_sync(1 + wg, KS * kWg);
+        tc_fence_after();
+        float o4[4];
+        tmem_ld4(x_col + 4 * (1 - kh), o4);
+        tmem_wait_ld();
+        m = fmaxf(m, o4[0]);
+      }
+      // 2^(x - m) (unnormalised), then D = (sum 2^(x - m) dP) / l, max |dP|
+      float l = 0.f;
       if (me.valid) {
-        inv = 1.f / exp_sum<N>(x, m);
-#pragma unroll
-        for (int j = 0; j < N; j += 2) {
-          const float2 pj = __fmul2_rn(make_float2(x[j], x[j + 1]), make_float2(inv, inv));
-          x[j] = pj.x;
-          x[j + 1] = pj.y;
-        }
+        l = exp_sum<KN>(x, m);
       } else {
 #pragma unroll
-        for (int j = 0; j < N; ++j) x[j] = 0.f;
+        for (int j = 0; j < KN; ++j) x[j] = 0.f;
       }
       // TMEM loads are warp-collective: every lane runs them, valid row or not
       // (x = 0 on invalid rows, so D = 0 and dS = 0 there).
       float2 dda = make_float2(0.f, 0.f), ddb = make_float2(0.f, 0.f);   // keys j mod 4
       float mdp = 0.f;
       {
-        float dp[N];
-        tmem_load_cols<N>(dp_col, dp);
+        float dp[KN];
+        tmem_load_cols<KN>(dp_col, dp);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < N; j += 4) {
+        for (int j = 0; j < KN; j += 4) {
           dda = __ffma2_rn(make_float2(x[j], x[j + 1]), make_float2(dp[j], dp[j + 1]), dda);
           ddb = __ffma2_rn(make_float2(x[j + 2], x[j + 3]), make_float2(dp[j + 2], dp[j + 3]), ddb);
           mdp = fmaxf(mdp, fmaxf(fmaxf(fabsf(dp[j]), fabsf(dp[j + 1])),
                                  fmaxf(fabsf(dp[j + 2]), fabsf(dp[j + 3]))));
         }
       }
-      const float D = (dda.x + dda.y) + (ddb.x + ddb.y);
+      float d = (dda.x + dda.y) + (ddb.x + ddb.y);
+      if constexpr (KS > 1) {   // sums and max |dP| over both key parts
+        tmem_st4(x_col + 8 + 4 * kh, l, d, mdp, 0.f);
+        tmem_wait_st();
+        tc_fence_before();
+        named_sync(1 + wg, KS * kWg);
+        tc_fence_after();
+        float o4[4];
+        tmem_ld4(x_col + 8 + 4 * (1 - kh), o4);
+        tmem_wait_ld();
+        l += o4[0];
+        d += o4[1];
+        mdp = fmaxf(mdp, o4[2]);
+      }
+      const float inv = me.valid ? 1.f / l : 0.f;   // max_j P_ij (= 1 / row sum); 0 on pad rows
+      const float D = d * inv;
+#pragma unroll
+      for (int j = 0; j < KN; j += 2) {
+        const float2 pj = __fmul2_rn(make_float2(x[j], x[j + 1]), make_float2(inv, inv));
+        x[j] = pj.x;
+        x[j + 1] = pj.y;
+      }
       __syncwarp();
 #pragma unroll
-      for (int c = 0; c < N / 32; ++c) tmem_st32(s_col + 32 * c, x + 32 * c);
+      for (int c = 0; c < KN / 32; ++c) tmem_st32(s_col + 32 * c, x + 32 * c);
       // The bins and bounds are free once the fold warp has taken this
-      // warpgroup's previous tile.
+      // tile pair's previous tile.
       if (k >= NWG)
         mbar_wait(&bins_empty[wg], (uint32_t)(((k / NWG) - 1) & 1), abort, p.status,
                   kWaitLimitNs);
       // |dS_ij| = P_ij |dP_ij - D| <= max_j P_ij * (max_j |dP_ij| + |D|); a NaN
-      // becomes +inf here, since fmaxf would drop it
+      // becomes +inf here, since fmaxf would drop it (both key parts of a row
+      // compute the same bound)
       {
         float rb = inv * (mdp + fabsf(D));
         if (!(rb <= 3.0e38f)) rb = INFINITY;
         const float wb = warp_max(rb);
         if (lane == 0) bnd[warp & 3] = wb;
       }
-      named_sync(3 + wg, kWg);
+      named_sync(3 + wgi, kWg);
       // Each window has its own unit (warps 2gw and 2gw+1 hold its rows), so
       // its integer sums do not depend on which window shares its tile.
       const float win_bound = fmaxf(bnd[2 * gw], bnd[2 * gw + 1]);
@@ -675,9 +729,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const int E = tile_exponent(finite ? win_bound : 0.f);
       const float qs = exp2_int(E);
       tmem_wait_st();
-      int* bq = tb + me.bias_base;
+      int* bq = tb + me.bias_base - (plain ? plain_off<(WW > 0 ? WW : 8)>(k0) : 0);
 #pragma unroll 1
-      for (int c = 0; c < N / 32; ++c) {
+      for (int c = 0; c < KN / 32; ++c) {
         float ds[32], pc[32];
         __syncwarp();
         tmem_ld32(dp_col + 32 * c, ds);
@@ -726,57 +780,58 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         mbar_wait(&grad_full[(k - 1) % NT], (uint32_t)(((k - 1) / NT) & 1), abort, p.status,
                   kWaitLimitNs);
 #pragma unroll 1
-      for (int c = 0; c < N / 32; ++c) {
+      for (int c = 0; c < KN / 32; ++c) {
         float pc[32], ds[32];
         __syncwarp();
         tmem_ld32(s_col + 32 * c, pc);
         tmem_ld32(dp_col + 32 * c, ds);
         tmem_wait_ld();
-        store_split_cols_part<32>(blk_ph, blk_pl, lr, 32 * c, pc);
-        store_split_cols_part<32>(blk_sh, blk_sl, lr, 32 * c, ds);
+        store_split_cols_part<32>(blk_ph, blk_pl, lr, k0 + 32 * c, pc);
+        store_split_cols_part<32>(blk_sh, blk_sl, lr, k0 + 32 * c, ds);
       }
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(&pds_full[sl]);
       // epilogue: dV (as soon as its products are done), then dQ and dK,
       // from TMEM to their grid tokens in whole-row stores (zero rows beyond
-      // the valid extent)
-      constexpr int OC = HD > 64 ? 64 : HD;   // columns per TMEM read
+      // the valid extent); each key part stores its own HD / KS columns
+      constexpr int HC = HD / KS;               // columns of each output this thread stores
+      constexpr int OC = HC > 64 ? 64 : HC;     // columns per TMEM read
+      const int c_lo = kh * HC;
       const bool st_row = me.stored && !*abort;
       const long long roff = (me.token * g.heads + h) * HD;
+      auto store_part = [&](int part, int c0) {
+        float o[OC];
+        if constexpr (OC == 16) {
+          __syncwarp();
+          tmem_ld16(tmem + lane_base + sl * 256 + part * GC + c0, o);
+        } else {
+          tmem_load_cols<OC>(tmem + lane_base + sl * 256 + part * GC + c0, o);
+        }
+        tmem_wait_ld();
+        if (part == 2 && c0 + OC == c_lo + HC) {
+          tc_fence_before();
+          mbar_arrive(&t_empty[sl]);
+        }
+        store_rows_bf16<OC>(o, 1.f, st_row ? (const void*)((me.halo ? outs_h[part] : outs[part]) +
+                                                            roff + c0)
+                                           : nullptr);
+      };
       mbar_wait(&gradv_full[sl], pht, abort, p.status, kWaitLimitNs);
       tc_fence_after();
 #pragma unroll
-      for (int c0 = 0; c0 < HD; c0 += OC) {
-        float o[OC];
-        tmem_load_cols<OC>(tmem + lane_base + sl * 256 + c0, o);
-        tmem_wait_ld();
-        store_rows_bf16<OC>(o, 1.f, st_row ? (const void*)((me.halo ? outs_h[0] : outs[0]) + roff + c0)
-                                           : nullptr);
-      }
+      for (int c0 = 0; c0 < HC; c0 += OC) store_part(0, c_lo + c0);
       mbar_wait(&grad_full[sl], pht, abort, p.status, kWaitLimitNs);
       tc_fence_after();
 #pragma unroll
-      for (int part = 1; part < 3; ++part) {
+      for (int part = 1; part < 3; ++part)
 #pragma unroll
-        for (int c0 = 0; c0 < HD; c0 += OC) {
-          float o[OC];
-          tmem_load_cols<OC>(tmem + lane_base + sl * 256 + part * GC + c0, o);
-          tmem_wait_ld();
-          if (part == 2 && c0 + OC == HD) {
-            tc_fence_before();
-            mbar_arrive(&t_empty[sl]);
-          }
-          store_rows_bf16<OC>(o, 1.f, st_row ? (const void*)((me.halo ? outs_h[part] : outs[part]) +
-                                                              roff + c0)
-                                             : nullptr);
-        }
-      }
+        for (int c0 = 0; c0 < HC; c0 += OC) store_part(part, c_lo + c0);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == C::kMma) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -866,7 +921,9 @@ size_t fwd_smem(const Geo& g) {
 }
 template <int HD>
 size_t bwd_smem(const Geo& g) {
-  return make_layout<HD, BwdCfg<HD>::kStages, 4, kNumBlk * kBlk>(bins_padded(g.bins)).total +
+  using C = BwdCfg<HD>;
+  return make_layout<HD, C::kStages, 4, kNumBlk * kBlk, C::kColBufs, C::kSoftWg>(
+             bins_padded(g.bins)).total +
          1024;
 }
 size_t fwd_smem_any(const Geo& g) {
@@ -960,11 +1017,14 @@ cudaError_t fast_backward(const Geo& g, const void* q, const void* k, const void
   const size_t smem = bwd_smem_any(g);
   const bool w8 = g.wh == 8 && g.ww == 8;
   if (g.hd == 128)
-    e = w8 ? launch(bwd_kernel<128, 8>, p, smem, st) : launch(bwd_kernel<128, 0>, p, smem, st);
+    e = w8 ? launch(bwd_kernel<128, 8>, p, smem, st, BwdCfg<128>::kThreads)
+           : launch(bwd_kernel<128, 0>, p, smem, st, BwdCfg<128>::kThreads);
   else if (g.hd == 64)
-    e = w8 ? launch(bwd_kernel<64, 8>, p, smem, st) : launch(bwd_kernel<64, 0>, p, smem, st);
+    e = w8 ? launch(bwd_kernel<64, 8>, p, smem, st, BwdCfg<64>::kThreads)
+           : launch(bwd_kernel<64, 0>, p, smem, st, BwdCfg<64>::kThreads);
   else
-    e = w8 ? launch(bwd_kernel<32, 8>, p, smem, st) : launch(bwd_kernel<32, 0>, p, smem, st);
+    e = w8 ? launch(bwd_kernel<32, 8>, p, smem, st, BwdCfg<32>::kThreads)
+           : launch(bwd_kernel<32, 0>, p, smem, st, BwdCfg<32>::kThreads);
   if (e != cudaSuccess) return e;
   if (flags & SWIN_FLAG_DBIAS_SUMS) return cudaSuccess;   // the caller finishes the sums
   return finish_dbias(g, dt_acc, dtable, st);
