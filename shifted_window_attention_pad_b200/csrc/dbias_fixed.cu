@@ -17,6 +17,9 @@ constexpr float kLog2eP = 1.4426950408889634f;
 __global__ void bias_prep_kernel(const float* __restrict__ table, int bins, int heads,
                                  int bins_pad, float* __restrict__ out,
                                  long long* __restrict__ acc) {
+  // Launched as a programmatic dependent of the kernel before it (which may
+  // still read this workspace): nothing is touched before that one completes.
+  ptx::grid_dep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= heads * bins_pad) return;
   const int h = i / bins_pad, b = i - h * bins_pad;
@@ -31,6 +34,7 @@ __global__ void bias_prep_kernel(const float* __restrict__ table, int bins, int 
 // fp32; NaN where a non-finite value reached the sum.
 __global__ void dbias_finish_kernel(const long long* __restrict__ acc, int bins, int heads,
                                     int bins_pad, float* __restrict__ dtable) {
+  ptx::grid_dep_wait();   // the gradient sums are complete once the kernel before has completed
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= bins * heads) return;
   const int b = i / heads, h = i - b * heads;
@@ -65,21 +69,37 @@ size_t dbias_fixed_offset(const Geo& g) {
   return kWsHeader + align256((size_t)g.heads * bins_padded(g.bins) * 4);
 }
 
+namespace {
+// Launch as a programmatic dependent of the previous kernel on the stream, so
+// that the launch overlaps that kernel's last blocks (the kernel itself waits
+// for it to complete before touching memory). The tensor-core kernels are
+// launched plainly: as dependents of these small kernels they measured slower.
+template <typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Args...), int n, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((n + 255) / 256 > 0 ? (n + 255) / 256 : 1));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  note_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t prep_bias(const Geo& g, const float* table, float* bias_t, long long* acc,
                       cudaStream_t st) {
-  const int n = g.heads * bins_padded(g.bins);
-  bias_prep_kernel<<<(n + 255) / 256, 256, 0, st>>>(table, g.bins, g.heads, bins_padded(g.bins),
-                                                    bias_t, acc);
-  note_launch();
-  return cudaGetLastError();
+  return launch_dependent(bias_prep_kernel, g.heads * bins_padded(g.bins), st, table, g.bins,
+                          g.heads, bins_padded(g.bins), bias_t, acc);
 }
 
 cudaError_t finish_dbias(const Geo& g, const long long* acc, float* dtable, cudaStream_t st) {
-  const int n = g.bins * g.heads;
-  dbias_finish_kernel<<<(n + 255) / 256, 256, 0, st>>>(acc, g.bins, g.heads, bins_padded(g.bins),
-                                                       dtable);
-  note_launch();
-  return cudaGetLastError();
+  return launch_dependent(dbias_finish_kernel, g.bins * g.heads, st, acc, g.bins, g.heads,
+                          bins_padded(g.bins), dtable);
 }
 
 }  // namespace swin

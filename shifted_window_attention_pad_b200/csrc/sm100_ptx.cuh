@@ -138,6 +138,15 @@ __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- programmatic dependent launch -----------------------------------------------
+// A kernel launched as a programmatic dependent of the one before it on the
+// stream may be scheduled as that one's blocks exit, before its writes are
+// flushed; grid_dep_wait blocks until that kernel has completed and its writes
+// are visible.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---- named barriers ---------------------------------------------------------------
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
