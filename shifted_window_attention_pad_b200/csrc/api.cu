@@ -41,12 +41,14 @@ static int check_desc(const swin_wattn_desc* d) {
 }
 
 // 1 = tcgen05/TMA kernels (64-token windows), 3 = tcgen05/TMA kernels
-// (256-token windows), 2 = warp-level tensor-core kernels, 0 = portable.
+// (256-token windows), 4 = tcgen05/TMA kernels (1024-token windows),
+// 2 = warp-level tensor-core kernels, 0 = portable.
 static int choose_path(const swin_wattn_desc* d, const Geo& g) {
   if (d->flags & SWIN_FLAG_FORCE_GENERIC) return 0;
   if (!(d->flags & SWIN_FLAG_FORCE_TILED)) {
     if (fast_supported(g, d->dtype)) return 1;
     if (wide_supported(g, d->dtype)) return 3;
+    if (large_supported(g, d->dtype)) return 4;
   }
   if (tiled_supported(g, d->dtype)) return 2;
   return 0;
@@ -57,6 +59,7 @@ static int cuda_status(cudaError_t e) { return e == cudaSuccess ? SWIN_OK : SWIN
 static size_t need_workspace(const swin_wattn_desc* d, const Geo& g) {
   switch (choose_path(d, g)) {
     case 1: case 3: return fast_workspace(g);
+    case 4: return large_workspace(g);
     case 2: return tiled_workspace(g);
     default: return generic_workspace(g);
   }
@@ -120,6 +123,8 @@ int swin_wattn_fwd(const swin_wattn_desc* desc, const void* q, const void* k, co
     return cuda_status(fast_forward(g, q, k, v, bias_table, out, lse, workspace, desc->flags, st));
   if (path == 3)
     return cuda_status(wide_forward(g, q, k, v, bias_table, out, lse, workspace, desc->flags, st));
+  if (path == 4)
+    return cuda_status(large_forward(g, q, k, v, bias_table, out, lse, workspace, desc->flags, st));
   if (path == 2)
     return cuda_status(tiled_forward(g, q, k, v, bias_table, out, lse, workspace, st));
   return cuda_status(
@@ -143,6 +148,9 @@ int swin_wattn_bwd(const swin_wattn_desc* desc, const void* q, const void* k, co
   if (path == 3)
     return cuda_status(wide_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
                                      workspace, desc->flags, st));
+  if (path == 4)
+    return cuda_status(large_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
+                                      workspace, desc->flags, st));
   if (path == 2)
     return cuda_status(tiled_backward(g, q, k, v, bias_table, dout, dq, dk, dv, dbias_table,
                                       workspace, desc->flags, st));

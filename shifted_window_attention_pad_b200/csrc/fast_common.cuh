@@ -167,19 +167,10 @@ struct RowInfo {
   long long token;  // (b H + y) W + x
 };
 
-__device__ inline RowInfo row_info(const Geo& g, long long win, int r) {
+// Row of slot (iy, ix) of window (wy, wx) of image b.
+__device__ inline RowInfo row_info_at(const Geo& g, int b, int wy, int wx, int iy, int ix) {
   RowInfo ri;
-  ri.valid = false;
-  ri.stored = false;
   ri.halo = false;
-  ri.label = 15;
-  ri.bias_base = 0;
-  ri.key_off = 0;
-  ri.token = 0;
-  if (win >= g.n_win) return ri;
-  int b, wy, wx, iy, ix;
-  window_coords(g, win, b, wy, wx);
-  row_slot(g, wy, wx, r, iy, ix);
   const int yr = wy * g.wh + iy, xr = wx * g.ww + ix;
   const int y = (yr + g.sh) % g.Hp, x = (xr + g.sw) % g.Wp;
   ri.stored = y < g.H && x < g.W;
@@ -195,6 +186,85 @@ __device__ inline RowInfo row_info(const Geo& g, long long win, int r) {
     ri.token = ((long long)b * g.sh + y) * g.W + x;
   }
   return ri;
+}
+
+__device__ inline RowInfo no_row() {
+  RowInfo ri;
+  ri.valid = false;
+  ri.stored = false;
+  ri.halo = false;
+  ri.label = 15;
+  ri.bias_base = 0;
+  ri.key_off = 0;
+  ri.token = 0;
+  return ri;
+}
+
+__device__ inline RowInfo row_info(const Geo& g, long long win, int r) {
+  if (win >= g.n_win) return no_row();
+  int b, wy, wx, iy, ix;
+  window_coords(g, win, b, wy, wx);
+  row_slot(g, wy, wx, r, iy, ix);
+  return row_info_at(g, b, wy, wx, iy, ix);
+}
+
+// ---- windows of more than 256 tokens: 128-token blocks --------------------------
+// A window of ww = 32 columns is taken in blocks of 128 slots, 128 / ww whole
+// window rows each. Inside a block the slots follow its sub-boxes column
+// segment first, as for a whole window, so a block of a window on the column
+// seam is two (or, where the block also straddles the row seam, four)
+// sub-boxes. Block-row boxes have 128 / ww rows, or the two parts
+// (wh - sh) mod (128 / ww) and the rest where a block straddles the row seam.
+__device__ inline int plan_block(const Geo& g, int wy, int wx, int blk, SubBox* sb) {
+  const int bh = kRows / g.ww;
+  const int y0 = blk * bh;
+  const int ysplit = g.wh - g.sh;   // first window row whose source row wraps
+  const bool split_y = g.sh > 0 && wy == g.nWy - 1 && ysplit > y0 && ysplit < y0 + bh;
+  const bool wrap_x = g.sw > 0 && wx == g.nWx - 1;
+  int ys[2], yl[2], yk[2], xs[2], xl[2], xk[2];
+  const int ny = split_y ? 2 : 1, nx = wrap_x ? 2 : 1;
+  if (split_y) {
+    ys[0] = y0; yl[0] = ysplit - y0; yk[0] = 1;
+    ys[1] = ysplit; yl[1] = y0 + bh - ysplit; yk[1] = 2;
+  } else {
+    ys[0] = y0; yl[0] = bh; yk[0] = 0;
+  }
+  if (wrap_x) {
+    xs[0] = 0; xl[0] = g.ww - g.sw; xk[0] = 1;
+    xs[1] = g.ww - g.sw; xl[1] = g.sw; xk[1] = 2;
+  } else {
+    xs[0] = 0; xl[0] = g.ww; xk[0] = 0;
+  }
+  int n = 0, off = 0;
+  for (int c = 0; c < nx; ++c)
+    for (int a = 0; a < ny; ++a) {
+      sb[n].y = (wy * g.wh + ys[a] + g.sh) % g.Hp;
+      sb[n].x = (wx * g.ww + xs[c] + g.sw) % g.Wp;
+      sb[n].rows = yl[a];
+      sb[n].cols = xl[c];
+      sb[n].map_id = yk[a] * 3 + xk[c];
+      sb[n].row_off = off;
+      off += yl[a] * xl[c];
+      ++n;
+    }
+  return n;
+}
+
+// Row of window slot r (block r / 128, slot r % 128 of the block).
+__device__ inline RowInfo block_row_info(const Geo& g, long long win, int r) {
+  if (win >= g.n_win) return no_row();
+  int b, wy, wx;
+  window_coords(g, win, b, wy, wx);
+  const int bh = kRows / g.ww;
+  const int blk = r / kRows, rb = r - blk * kRows;
+  const bool wrap_x = g.sw > 0 && wx == g.nWx - 1;
+  const int w0 = wrap_x ? g.ww - g.sw : g.ww;
+  const int xseg = rb >= bh * w0;
+  const int rr = xseg ? rb - bh * w0 : rb;
+  const int wseg = xseg ? g.ww - w0 : w0;
+  const int iy = blk * bh + rr / wseg;
+  const int ix = (xseg ? w0 : 0) + (rr - (rr / wseg) * wseg);
+  return row_info_at(g, b, wy, wx, iy, ix);
 }
 
 // Packed per-key info: low 16 bits key offset into the bias table, bits 16-19

@@ -76,6 +76,17 @@ cudaError_t wide_backward(const Geo& g, const void* q, const void* k, const void
                           const float* table, const void* dout, void* dq, void* dk, void* dv,
                           float* dtable, void* ws, int flags, cudaStream_t st);
 
+// ---- tcgen05 / TMA kernels for 1024-token windows (32 x 32, bf16, head_dim
+// 64 or 128) --------------------------------------------------------------------
+bool large_supported(const Geo& g, int dtype);
+size_t large_workspace(const Geo& g);
+cudaError_t large_forward(const Geo& g, const void* q, const void* k, const void* v,
+                          const float* table, void* out, float* lse, void* ws, int flags,
+                          cudaStream_t st);
+cudaError_t large_backward(const Geo& g, const void* q, const void* k, const void* v,
+                           const float* table, const void* dout, void* dq, void* dk, void* dv,
+                           float* dtable, void* ws, int flags, cudaStream_t st);
+
 // ---- warp-level tensor-core kernels: one CTA per (window, head), windows of
 // up to 256 tokens (bf16, head_dim 32 or 64) ----------------------------------
 bool tiled_supported(const Geo& g, int dtype);

@@ -61,11 +61,21 @@ def test_path_selection_on_the_workloads(L):
 
 @pytest.mark.parametrize("win,hd,want", [((7, 7), 64, 2), ((8, 12), 32, 2), ((16, 16), 64, 3),
                                          ((16, 16), 32, 3), ((8, 32), 64, 3), ((16, 8), 64, 2),
-                                         ((12, 12), 32, 2), ((16, 17), 64, 0), ((32, 32), 64, 0),
+                                         ((12, 12), 32, 2), ((16, 17), 64, 0), ((32, 32), 64, 4),
+                                         ((32, 32), 128, 4), ((32, 32), 32, 0),
                                          ((16, 16), 128, 0), ((8, 8), 64, 1), ((8, 8), 128, 1),
                                          ((4, 16), 128, 1), ((7, 7), 128, 0)])
-def test_tensor_core_paths_cover_windows_up_to_256_tokens(L, win, hd, want):
+def test_tensor_core_paths_cover_windows_up_to_1024_tokens(L, win, hd, want):
     d = sb.make_desc(1, 40, 52, win, (win[0] // 2, win[1] // 2), 2, hd, "bf16")
+    assert sb.swin_wattn_path(d) == want
+
+
+@pytest.mark.parametrize("shift,want", [((16, 16), 4), ((14, 16), 4), ((0, 0), 4), ((2, 12), 4),
+                                        ((15, 16), 4), ((16, 6), 4), ((16, 3), 0), ((13, 5), 0)])
+def test_1024_token_windows_need_sub_boxes_of_whole_swizzle_atoms(L, shift, want):
+    """A 128-token block's sub-boxes (rows of 4, or the two parts at the row
+    seam, times the column segments) must each hold a multiple of 8 rows."""
+    d = sb.make_desc(1, 64, 96, (32, 32), shift, 2, 128, "bf16")
     assert sb.swin_wattn_path(d) == want
 
 

@@ -32,9 +32,9 @@ def _table(win, heads, seed):
         (nb, heads)).astype(np.float32) * 0.02)
 
 
-# (name, description, inputs, path): the ragged workload on the tcgen05 kernels
-# and a padded 16 x 16-window grid on the 256-token tcgen05 kernels and on the
-# warp-MMA kernels
+# (name, description, inputs, path): the ragged workload on the tcgen05 kernels,
+# a padded 16 x 16-window grid on the 256-token tcgen05 kernels and on the
+# warp-MMA kernels, and 32 x 32 windows on the 1024-token tcgen05 kernels
 def _cases():
     wl = WORKLOADS["ragged-90x180-w8"]
     yield "tcgen05-ragged", sb.desc_for(wl), make_inputs(wl), 1
@@ -43,6 +43,8 @@ def _cases():
     yield "tcgen05-40x52-w16", sb.make_desc(1, 40, 52, 16, 8, 2, 64, "bf16"), inp, 3
     yield ("warp-mma-40x52-w16",
            sb.make_desc(1, 40, 52, 16, 8, 2, 64, "bf16", flags=sb.SWIN_FLAG_FORCE_TILED), inp, 2)
+    w32 = Workload("w32", 1, 64, 96, 32, 16, 2, 128, "bf16", 42)
+    yield "tcgen05-64x96-w32", sb.make_desc(1, 64, 96, 32, 16, 2, 128, "bf16"), make_inputs(w32), 4
 
 
 CASES = list(_cases())

@@ -282,6 +282,40 @@ def test_wide_path_parity(case):
         assert e <= BF16_TOL, (case, n, e)
 
 
+# ---------------------------------------------------------------------------
+# tcgen05 kernels for 1024-token windows (path 4)
+# ---------------------------------------------------------------------------
+# (B, H, W, window, shift, heads, head_dim, seed): both seams at head_dim 128
+# and 64, a padded grid, no shift, batch 2, a row shift whose seam splits a
+# 128-token block (window row 18 of 32), the largest model's window at the
+# 1/12-degree grid's width
+LARGE = [
+    (1, 64, 96, (32, 32), (16, 16), 2, 128, 91),
+    (1, 40, 72, (32, 32), (16, 16), 1, 64, 92),
+    (1, 32, 64, (32, 32), (0, 0), 2, 128, 93),
+    (2, 64, 64, (32, 32), (16, 16), 1, 128, 94),
+    (1, 64, 96, (32, 32), (14, 16), 1, 64, 95),
+    (1, 32, 544, (32, 32), (16, 16), 1, 128, 96),
+]
+
+
+@pytest.mark.parametrize("case", LARGE, ids=lambda c: "%dx%dx%d-w%dx%d-s%dx%d-hd%d" % (
+    c[0], c[1], c[2], *c[3], *c[4], c[6]))
+def test_large_path_parity(case):
+    B, H, W, win, shift, heads, hd, seed = case
+    d = sb.make_desc(B, H, W, win, shift, heads, hd, "bf16")
+    assert sb.swin_wattn_path(d) == 4
+    wl = Workload("large", B, H, W, win[0], shift[0], heads, hd, "bf16", seed)
+    inp = make_inputs(wl, shape_override=(B, H, W, heads, hd))
+    nb = (2 * win[0] - 1) * (2 * win[1] - 1)
+    inp["table"] = torch.from_numpy(np.random.Generator(np.random.PCG64(seed)).standard_normal(
+        (nb, heads)).astype(np.float32) * 0.02)
+    errs = compare(run_gpu(d, inp), run_oracle(d, inp), "bf16")
+    print(case, errs)
+    for n, e in errs.items():
+        assert e <= BF16_TOL, (case, n, e)
+
+
 @pytest.mark.parametrize("name", ["ragged-90x180-w8", "small-patch-2x512x1088-w8"])
 def test_tiled_path_forced_on_window64_workloads(name):
     """The warp-MMA kernels on the 8 x 8-window workloads the tcgen05 kernels
@@ -376,12 +410,15 @@ def test_bias_gradient_sums_to_zero_and_backward_is_deterministic():
     assert np.all(np.abs(dT.sum(axis=0)) <= 1e-3 * np.abs(dT).sum(axis=0) + 1e-6)
 
 
-def test_bounded_wait_reports_timeout_and_context_survives():
+@pytest.mark.parametrize("path", [1, 4])
+def test_bounded_wait_reports_timeout_and_context_survives(path):
     """A wait on a barrier that nothing arrives on runs out after ~1 ms: the call
     reports SWIN_ERR_TIMEOUT through the workspace status word, and the next
-    call on the same context works."""
-    wl = WORKLOADS["ragged-90x180-w8"]
+    call on the same context works (64-token and 1024-token kernels)."""
+    wl = (WORKLOADS["ragged-90x180-w8"] if path == 1 else
+          Workload("w32", 1, 40, 72, 32, 16, 2, 64, "bf16", 43))
     inp = make_inputs(wl)
+    assert sb.swin_wattn_path(sb.desc_for(wl)) == path
     dev = "cuda"
     q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "dout"))
     T = inp["table"].to(dev)
