@@ -1,4 +1,4 @@
-"""The five synthetic workloads: shapes and dtypes only, no arithmetic.
+"""The synthetic workloads: shapes and dtypes only, no arithmetic.
 
 Shapes follow the TERRA page ("TERRA: A Hierarchical Parallel Training and
 Memory Orchestration Framework for High-Resolution AI-based Earth Modeling"):
@@ -67,6 +67,12 @@ class Workload:
         """q, k, v, dO read and dq, dk, dv written once each."""
         return 7 * self.tokens * self.heads * self.head_dim * self.elem_bytes()
 
+    def flops_bwd(self):
+        """Dense window FLOPs of the backward alone: 8*N*hd per padded token per
+        head (dV, dP, dQ, dK; the recompute of S not counted)."""
+        N = self.win * self.win
+        return 8 * N * self.head_dim * self.B * self.Hp * self.Wp * self.heads
+
 
 WORKLOADS = {
     w.name: w for w in (
@@ -88,6 +94,9 @@ WORKLOADS = {
         Workload("table5-256x544-8x128-w8", 1, 256, 544, 8, 4, 8, 128, "bf16", 5,
                  "the 1/12-degree token grid with the 128-channel heads of Table V: "
                  "d=1024 = 8 heads x 128, 8x8 windows, shift 4"),
+        Workload("table5-large-256x544-8x128-w32", 1, 256, 544, 32, 16, 8, 128, "bf16", 7,
+                 "the 1/12-degree token grid with the window of Table V's largest model: "
+                 "32x32 windows (1024 tokens), shift 16, d=1024 = 8 heads x 128"),
     )
 }
 
