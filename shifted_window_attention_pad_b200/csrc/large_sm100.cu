@@ -450,8 +450,11 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
 // ================================================================================
 // Two kernels, because dQ sums over the key blocks and dK, dV over the query
 // blocks, and neither fits in one CTA's TMEM for a whole window:
+// Both take the keys (queries) of a block in two 64-wide sub-blocks, one per
+// softmax warpgroup and TMEM buffer, so that one warpgroup's products run
+// while the other works on its rows.
 //  * query kernel, item = (window, head, query block qb): pass 1 runs
-//    S = Q K_kb^T and dP = dO V_kb^T over the eight key blocks and keeps, per
+//    S = Q K_u^T and dP = dO V_u^T over the sixteen sub-blocks and keeps, per
 //    row and key half, an online maximum M, l = sum 2^(x - M),
 //    d = sum 2^(x - M) dP and max |dP|; the halves merge into L = M + log2 l
 //    and D = d / l = sum_j P_ij dP_ij, written to the workspace for the key
@@ -475,7 +478,10 @@ __host__ __device__ inline int kband0(int kb) { return (28 - 4 * kb) * 63; }
 constexpr int kBwdWarps = 12;   // two softmax warpgroups, producer, two MMA issuers, fold
 constexpr int kBwdThreads = kBwdWarps * 32;
 constexpr int kBwdProducer = 8, kBwdMma = 9, kBwdMma2 = 10, kBwdFold = 11;
-constexpr uint32_t kColDP = 128, kColGrad = 256;   // S at 0, dP at 128, gradients from 256
+// TMEM: two buffers of 128 columns, one per softmax warpgroup, each a 64-key
+// (query kernel) or 64-query (key kernel) sub-block's S and dP (S^T, dP^T) at
+// 128 b and 128 b + 64; the gradient accumulators from column 256.
+constexpr uint32_t kColGrad = 256;
 
 template <int HD>
 struct LargeBwdCfg {
@@ -570,11 +576,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* qd_empty = qd_full + 1;
   uint64_t* kv_full = qd_empty + 1;
   uint64_t* kv_empty = kv_full + NS;
-  uint64_t* sd_full = kv_empty + NS;
-  uint64_t* st_free = sd_full + 1;   // pass 1: the softmax has read S and dP
-  uint64_t* ds_full = st_free + 1;
-  uint64_t* dq_done = ds_full + 1;
-  uint64_t* t_empty = dq_done + 1;
+  uint64_t* sd_full = kv_empty + NS;   // [2] per TMEM buffer (= softmax warpgroup)
+  uint64_t* st_free = sd_full + 2;     // [2] pass 1: the warpgroup has read S and dP
+  uint64_t* ds_full = st_free + 2;     // [2]
+  uint64_t* dq_done = ds_full + 2;     // [2]
+  uint64_t* t_empty = dq_done + 2;
   uint64_t* bins_full = t_empty + 1;
   uint64_t* bins_empty = bins_full + 1;
   uint64_t* drain = bins_empty + 1;   // [2]
@@ -588,10 +594,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(qd_full, 1);
     mbar_init(qd_empty, 1 + 8);   // the last S / dP products and every softmax warp
     for (int i = 0; i < NS; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
-    mbar_init(sd_full, 1);
-    mbar_init(st_free, 2 * kWg);
-    mbar_init(ds_full, 2 * kWg);
-    mbar_init(dq_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sd_full[i], 1);
+      mbar_init(&st_free[i], kWg);
+      mbar_init(&ds_full[i], kWg);
+      mbar_init(&dq_done[i], 1);
+    }
     mbar_init(t_empty, 2 * kWg);
     mbar_init(bins_full, 2 * kWg);
     mbar_init(bins_empty, 32);
@@ -647,48 +655,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   } else if (warp == kBwdMma) {
-    if (lane == 0) {   // S = Q K_kb^T and dP = dO V_kb^T, sixteen steps an item
-      constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);
+    if (lane == 0) {   // S = Q K_u^T and dP = dO V_u^T of 64-key sub-blocks u, both passes
+      constexpr uint32_t idesc_s = idesc_bf16(kRows, 64, 0, 0);
       long long e = 0;
       bool ok = true;
       for (long long k = 0; k < n_local && ok; ++k) {
         if (!mbar_wait(qd_full, (uint32_t)(k & 1), abort, p.status, kWaitLimitNs)) break;
         const uint32_t q_s = smem_u32(qd), do_s = smem_u32(qd + TB);
-        for (int st = 0; st < 2 * kLargeBlocks; ++st, ++e) {
-          const int s = (int)(e % NS), kb = st & (kLargeBlocks - 1);
-          if (!mbar_wait(&kv_full[s], (uint32_t)((e / NS) & 1), abort, p.status,
-                         kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          // S and dP columns are free once the previous step is done with them:
-          // pass 1 steps once the softmax has read them, pass 2 steps once the
-          // dQ products have read the dS written over them
-          bool w = true;
-          if (st == 0) {
-            if (k > 0) w = mbar_wait(dq_done, 1u, abort, p.status, kWaitLimitNs);
-          } else if (st < kLargeBlocks || kb == 0) {
-            w = mbar_wait(st_free, (uint32_t)((st - 1) & 1), abort, p.status, kWaitLimitNs);
-          } else {
-            w = mbar_wait(dq_done, (uint32_t)((kb - 1) & 1), abort, p.status, kWaitLimitNs);
-          }
-          if (!w) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t k_s = smem_u32(ring + (s * 2 + 0) * TB);
-          const uint32_t v_s = smem_u32(ring + (s * 2 + 1) * TB);
+        for (int pass = 0; pass < 2 && ok; ++pass)
+          for (int u = 0; u < 2 * kLargeBlocks; ++u) {
+            const int b = u & 1, j = u >> 1;   // buffer (= warpgroup), key block
+            const int s = (int)(e % NS);
+            if (b == 0 && !mbar_wait(&kv_full[s], (uint32_t)((e / NS) & 1), abort, p.status,
+                                     kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            // buffer b is free once its previous sub-block is done with it: in
+            // pass 1 once the warpgroup has read S and dP, in pass 2 once the dQ
+            // products have read the dS written over dP
+            bool w = true;
+            if (pass == 0 && j == 0) {
+              if (k > 0) w = mbar_wait(&dq_done[b], 1u, abort, p.status, kWaitLimitNs);
+            } else if (pass == 0 || j == 0) {
+              w = mbar_wait(&st_free[b], (uint32_t)((j - 1) & 1), abort, p.status, kWaitLimitNs);
+            } else {
+              w = mbar_wait(&dq_done[b], (uint32_t)((j - 1) & 1), abort, p.status, kWaitLimitNs);
+            }
+            if (!w) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t k_s = smem_u32(ring + (s * 2 + 0) * TB) + b * 64 * TileGeom<HD>::kRowBytes;
+            const uint32_t v_s = smem_u32(ring + (s * 2 + 1) * TB) + b * 64 * TileGeom<HD>::kRowBytes;
+            const uint32_t d = tmem + 128 * b;
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk)
-            umma_ss(tmem, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk), idesc_s, kk);
+            for (int kk = 0; kk < HD / 16; ++kk)
+              umma_ss(d, desc_kmajor_tile<HD>(q_s, kk), desc_kmajor_tile<HD>(k_s, kk), idesc_s, kk);
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk)
-            umma_ss(tmem + kColDP, desc_kmajor_tile<HD>(do_s, kk), desc_kmajor_tile<HD>(v_s, kk),
-                    idesc_s, kk);
-          umma_commit(sd_full);
-          if (st < kLargeBlocks) umma_commit(&kv_empty[s]);   // pass 1: K, V read
-        }
+            for (int kk = 0; kk < HD / 16; ++kk)
+              umma_ss(d + 64, desc_kmajor_tile<HD>(do_s, kk), desc_kmajor_tile<HD>(v_s, kk),
+                      idesc_s, kk);
+            umma_commit(&sd_full[b]);
+            if (b == 1) {
+              if (pass == 0) umma_commit(&kv_empty[s]);   // pass 1: K, V of the block read
+              ++e;
+            }
+          }
         if (ok) umma_commit(qd_empty);
       }
       if (*abort) {
@@ -697,34 +711,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   } else if (warp == kBwdMma2) {
-    if (lane == 0) {   // dQ += scale dS K_kb (hi, then lo), pass 2
+    if (lane == 0) {   // dQ += scale dS_u K_u (hi, then lo), pass 2, sub-block by sub-block
       constexpr uint32_t idesc_q = idesc_bf16(kRows, HD, 0, 1);
       long long e = 0;
       bool ok = true;
       for (long long k = 0; k < n_local && ok; ++k) {
         e += kLargeBlocks;   // pass 1 entries of the ring
-        for (int kb = 0; kb < kLargeBlocks; ++kb, ++e) {
+        for (int u = 0; u < 2 * kLargeBlocks; ++u) {
+          const int b = u & 1, j = u >> 1;
           const int s = (int)(e % NS);
-          if (kb == 0 && !mbar_wait(t_empty, (uint32_t)((k & 1) ^ 1), abort, p.status,
-                                    kWaitLimitNs)) {
+          if (u == 0 && !mbar_wait(t_empty, (uint32_t)((k & 1) ^ 1), abort, p.status,
+                                   kWaitLimitNs)) {
             ok = false;
             break;
           }
-          if (!mbar_wait(ds_full, (uint32_t)(kb & 1), abort, p.status, kWaitLimitNs)) {
+          if (!mbar_wait(&ds_full[b], (uint32_t)(j & 1), abort, p.status, kWaitLimitNs)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t k_s = smem_u32(ring + (s * 2 + 0) * TB);
+          const uint32_t k_s = smem_u32(ring + (s * 2 + 0) * TB) + b * 64 * TileGeom<HD>::kRowBytes;
 #pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk) {
-            const uint32_t a = tmem + kColDP + split_col(kk);
-            const uint64_t b = desc_mnmajor_tile<HD>(k_s, kk);
-            umma_ts(tmem + kColGrad, a, b, idesc_q, (kb > 0 || kk > 0) ? 1u : 0u);
-            umma_ts(tmem + kColGrad, a + 16, b, idesc_q, 1u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t a = tmem + 128 * b + 64 + split_col(kk);
+            const uint64_t bd = desc_mnmajor_tile<HD>(k_s, kk);
+            umma_ts(tmem + kColGrad, a, bd, idesc_q, (u > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tmem + kColGrad, a + 16, bd, idesc_q, 1u);
           }
-          umma_commit(dq_done);
-          umma_commit(&kv_empty[s]);
+          umma_commit(&dq_done[b]);
+          if (b == 1) {
+            umma_commit(&kv_empty[s]);
+            ++e;
+          }
         }
       }
       if (*abort) {
@@ -753,12 +771,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else {
     // Softmax / epilogue: warpgroup kh holds keys 64 kh .. 64 kh + 63 of every
-    // key block for all 128 rows of the query block (thread = row = lane).
+    // key block (sub-blocks 2 kb + kh, in TMEM buffer kh) for all 128 rows of
+    // the query block (thread = row = lane).
     const int kh = warp >> 2;
     const int row = threadIdx.x & (kWg - 1);
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_col = tmem + lane_base + 64 * kh;
-    const uint32_t dp_col = s_col + kColDP;
+    const uint32_t s_col = tmem + lane_base + 128 * kh;
+    const uint32_t dp_col = s_col + 64;
     const float c = p.scale_log2;
     const float dscale = p.scale_log2 * (1.0f / kLog2e);   // head_dim^-1/2
     for (long long k = 0; k < n_local; ++k) {
@@ -781,7 +800,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float m = -INFINITY, l = 0.f, d = 0.f, mdp = 0.f;
 #pragma unroll 1
       for (int kb = 0; kb < kLargeBlocks; ++kb) {
-        mbar_wait(sd_full, (uint32_t)(kb & 1), abort, p.status, kWaitLimitNs);
+        mbar_wait(&sd_full[kh], (uint32_t)(kb & 1), abort, p.status, kWaitLimitNs);
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
@@ -818,7 +837,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           d += d2.x + d2.y;
         }
         tc_fence_before();
-        mbar_arrive(st_free);
+        mbar_arrive(&st_free[kh]);
       }
       // the two halves of each row merge; the block's bound sets its unit
       {
@@ -864,7 +883,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // pass 2: dS into the bins and, scaled, as dQ's operand
 #pragma unroll 1
       for (int kb = 0; kb < kLargeBlocks; ++kb) {
-        mbar_wait(sd_full, (uint32_t)(kb & 1), abort, p.status, kWaitLimitNs);
+        mbar_wait(&sd_full[kh], (uint32_t)(kb & 1), abort, p.status, kWaitLimitNs);
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
@@ -909,13 +928,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(ds_full);
+        mbar_arrive(&ds_full[kh]);
       }
       mbar_arrive(bins_full);
       __syncwarp();
       if (lane == 0) mbar_arrive(qd_empty);   // the bias run is read
-      // epilogue: this half's HD / 2 columns of the dQ row
-      mbar_wait(dq_done, 1u, abort, p.status, kWaitLimitNs);
+      // epilogue: this half's HD / 2 columns of the dQ row, once the item's
+      // last product (sub-block 15, buffer 1) is done
+      mbar_wait(&dq_done[1], 1u, abort, p.status, kWaitLimitNs);
       tc_fence_after();
       {
         constexpr int OC = HD / 2;
@@ -961,10 +981,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* kv_empty = kv_full + 1;
   uint64_t* qd_full = kv_empty + 1;
   uint64_t* qd_empty = qd_full + NS;
-  uint64_t* sd_full = qd_empty + NS;
-  uint64_t* pds_full = sd_full + 1;
-  uint64_t* grad_done = pds_full + 1;
-  uint64_t* t_empty = grad_done + 1;
+  uint64_t* sd_full = qd_empty + NS;   // [2] per TMEM buffer (= softmax warpgroup)
+  uint64_t* pds_full = sd_full + 2;    // [2]
+  uint64_t* grad_done = pds_full + 2;  // [2]
+  uint64_t* t_empty = grad_done + 2;
   uint64_t* drain = t_empty + 1;   // [2]
   uint64_t* never = drain + 2;
   uint32_t* tmem_slot = (uint32_t*)(smem + L.misc);
@@ -976,9 +996,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1 + 8);   // the last S^T / dP^T products and every softmax warp
     for (int i = 0; i < NS; ++i) { mbar_init(&qd_full[i], 1); mbar_init(&qd_empty[i], 1); }
-    mbar_init(sd_full, 1);
-    mbar_init(pds_full, 2 * kWg);
-    mbar_init(grad_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sd_full[i], 1);
+      mbar_init(&pds_full[i], kWg);
+      mbar_init(&grad_done[i], 1);
+    }
     mbar_init(t_empty, 2 * kWg);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
@@ -1032,33 +1054,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   } else if (warp == kBwdMma) {
-    if (lane == 0) {   // S^T = K Q_qb^T and dP^T = V dO_qb^T
-      constexpr uint32_t idesc_s = idesc_bf16(kRows, kRows, 0, 0);
+    if (lane == 0) {   // S^T = K Q_u^T and dP^T = V dO_u^T of 64-query sub-blocks u
+      constexpr uint32_t idesc_s = idesc_bf16(kRows, 64, 0, 0);
       long long e = 0;
       bool ok = true;
       for (long long k = 0; k < n_local && ok; ++k) {
         if (!mbar_wait(kv_full, (uint32_t)(k & 1), abort, p.status, kWaitLimitNs)) break;
         const uint32_t k_s = smem_u32(kvt), v_s = smem_u32(kvt + TB);
-        for (int qb = 0; qb < kLargeBlocks; ++qb, ++e) {
+        for (int u = 0; u < 2 * kLargeBlocks; ++u) {
+          const int b = u & 1, qb = u >> 1;   // buffer (= warpgroup), query block
           const int s = (int)(e % NS);
-          if (!mbar_wait(&qd_full[s], (uint32_t)((e / NS) & 1), abort, p.status,
-                         kWaitLimitNs) ||
-              // the columns hold the previous step's P and dS until its products are done
-              !mbar_wait(grad_done, (uint32_t)((qb & 1) ^ 1), abort, p.status, kWaitLimitNs)) {
+          if ((b == 0 && !mbar_wait(&qd_full[s], (uint32_t)((e / NS) & 1), abort, p.status,
+                                    kWaitLimitNs)) ||
+              // buffer b holds its previous sub-block's P and dS until their products are done
+              !mbar_wait(&grad_done[b], (uint32_t)((qb & 1) ^ 1), abort, p.status,
+                         kWaitLimitNs)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t q_s = smem_u32(ring + (s * 2 + 0) * TB);
-          const uint32_t do_s = smem_u32(ring + (s * 2 + 1) * TB);
+          const uint32_t off = b * 64 * TileGeom<HD>::kRowBytes;
+          const uint32_t q_s = smem_u32(ring + (s * 2 + 0) * TB) + off;
+          const uint32_t do_s = smem_u32(ring + (s * 2 + 1) * TB) + off;
+          const uint32_t d = tmem + 128 * b;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk)
-            umma_ss(tmem, desc_kmajor_tile<HD>(k_s, kk), desc_kmajor_tile<HD>(q_s, kk), idesc_s, kk);
+            umma_ss(d, desc_kmajor_tile<HD>(k_s, kk), desc_kmajor_tile<HD>(q_s, kk), idesc_s, kk);
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk)
-            umma_ss(tmem + kColDP, desc_kmajor_tile<HD>(v_s, kk), desc_kmajor_tile<HD>(do_s, kk),
+            umma_ss(d + 64, desc_kmajor_tile<HD>(v_s, kk), desc_kmajor_tile<HD>(do_s, kk),
                     idesc_s, kk);
-          umma_commit(sd_full);
+          umma_commit(&sd_full[b]);
+          if (b == 1) ++e;
         }
         if (ok) umma_commit(kv_empty);
       }
@@ -1068,38 +1095,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   } else if (warp == kBwdMma2) {
-    if (lane == 0) {   // dV += P^T dO_qb, dK += scale dS^T Q_qb (hi, then lo)
+    if (lane == 0) {   // dV += P^T dO_u, dK += scale dS^T Q_u (hi, then lo), sub-block by sub-block
       constexpr uint32_t idesc_g = idesc_bf16(kRows, HD, 0, 1);
       long long e = 0;
       bool ok = true;
       for (long long k = 0; k < n_local && ok; ++k) {
-        for (int qb = 0; qb < kLargeBlocks; ++qb, ++e) {
+        for (int u = 0; u < 2 * kLargeBlocks; ++u) {
+          const int b = u & 1, qb = u >> 1;
           const int s = (int)(e % NS);
-          if (qb == 0 && !mbar_wait(t_empty, (uint32_t)((k & 1) ^ 1), abort, p.status,
-                                    kWaitLimitNs)) {
+          if (u == 0 && !mbar_wait(t_empty, (uint32_t)((k & 1) ^ 1), abort, p.status,
+                                   kWaitLimitNs)) {
             ok = false;
             break;
           }
-          if (!mbar_wait(pds_full, (uint32_t)(qb & 1), abort, p.status, kWaitLimitNs)) {
+          if (!mbar_wait(&pds_full[b], (uint32_t)(qb & 1), abort, p.status, kWaitLimitNs)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t q_s = smem_u32(ring + (s * 2 + 0) * TB);
-          const uint32_t do_s = smem_u32(ring + (s * 2 + 1) * TB);
+          const uint32_t off = b * 64 * TileGeom<HD>::kRowBytes;
+          const uint32_t q_s = smem_u32(ring + (s * 2 + 0) * TB) + off;
+          const uint32_t do_s = smem_u32(ring + (s * 2 + 1) * TB) + off;
 #pragma unroll
-          for (int kk = 0; kk < kRows / 16; ++kk) {
-            const uint32_t a = tmem + split_col(kk);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t a = tmem + 128 * b + split_col(kk);
             const uint64_t bo = desc_mnmajor_tile<HD>(do_s, kk);
             const uint64_t bq = desc_mnmajor_tile<HD>(q_s, kk);
-            const uint32_t first = (qb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t first = (u > 0 || kk > 0) ? 1u : 0u;
             umma_ts(tmem + kColGrad, a, bo, idesc_g, first);
             umma_ts(tmem + kColGrad, a + 16, bo, idesc_g, 1u);
-            umma_ts(tmem + kColGrad + HD, a + kColDP, bq, idesc_g, first);
-            umma_ts(tmem + kColGrad + HD, a + kColDP + 16, bq, idesc_g, 1u);
+            umma_ts(tmem + kColGrad + HD, a + 64, bq, idesc_g, first);
+            umma_ts(tmem + kColGrad + HD, a + 64 + 16, bq, idesc_g, 1u);
           }
-          umma_commit(grad_done);
-          umma_commit(&qd_empty[s]);
+          umma_commit(&grad_done[b]);
+          if (b == 1) {
+            umma_commit(&qd_empty[s]);
+            ++e;
+          }
         }
       }
       if (*abort) {
@@ -1109,12 +1141,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp < 8) {
     // Softmax / epilogue: thread = key row = lane of the block; warpgroup kh
-    // takes queries 64 kh .. 64 kh + 63 of every query block.
+    // takes queries 64 kh .. 64 kh + 63 of every query block (sub-blocks
+    // 2 qb + kh, in TMEM buffer kh).
     const int kh = warp >> 2;
     const int row = threadIdx.x & (kWg - 1);
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_col = tmem + lane_base + 64 * kh;
-    const uint32_t dp_col = s_col + kColDP;
+    const uint32_t s_col = tmem + lane_base + 128 * kh;
+    const uint32_t dp_col = s_col + 64;
     const float c = p.scale_log2;
     const float dscale = p.scale_log2 * (1.0f / kLog2e);   // head_dim^-1/2
     for (long long k = 0; k < n_local; ++k) {
@@ -1138,7 +1171,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool live = me.valid;   // a pad key: P = 0 in its whole row
 #pragma unroll 1
       for (int qb = 0; qb < kLargeBlocks; ++qb) {
-        mbar_wait(sd_full, (uint32_t)(qb & 1), abort, p.status, kWaitLimitNs);
+        mbar_wait(&sd_full[kh], (uint32_t)(qb & 1), abort, p.status, kWaitLimitNs);
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
@@ -1180,12 +1213,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(pds_full);
+        mbar_arrive(&pds_full[kh]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(kv_empty);   // bias run, statistics and query words read
       // epilogue: this half's HD / 2 columns of the dV and dK rows of this key
-      mbar_wait(grad_done, 1u, abort, p.status, kWaitLimitNs);
+      mbar_wait(&grad_done[1], 1u, abort, p.status, kWaitLimitNs);   // sub-block 15's products
       tc_fence_after();
       {
         constexpr int OC = HD / 2;
