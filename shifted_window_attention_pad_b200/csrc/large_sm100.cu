@@ -475,9 +475,15 @@ constexpr int kBandBins = (kRows / 32 + 31) * 63;     // 2205
 constexpr int kBandPad = (kBandBins + 3) & ~3;        // 2208: whole 16-byte copies
 __host__ __device__ inline int qband0(int qb) { return 4 * qb * 63; }
 __host__ __device__ inline int kband0(int kb) { return (28 - 4 * kb) * 63; }
-constexpr int kBwdWarps = 12;   // two softmax warpgroups, producer, two MMA issuers, fold
-constexpr int kBwdThreads = kBwdWarps * 32;
-constexpr int kBwdProducer = 8, kBwdMma = 9, kBwdMma2 = 10, kBwdFold = 11;
+// Warps: four softmax warpgroups (two per TMEM buffer, each 32 columns of its
+// sub-block), the TMA producer, two MMA issuers and, in the query kernel, the
+// bin fold: 20 and 19 warps, 96 registers a thread.
+constexpr int kBwdSoftWg = 4;
+constexpr int kBwdProducer = kBwdSoftWg * 4, kBwdMma = kBwdProducer + 1,
+              kBwdMma2 = kBwdProducer + 2, kBwdFold = kBwdProducer + 3;
+constexpr int kBwdQThreads = (kBwdSoftWg * 4 + 4) * 32;
+constexpr int kBwdKThreads = (kBwdSoftWg * 4 + 3) * 32;
+constexpr uint32_t kColXch = 384;   // query kernel: the warpgroups' row statistics
 // TMEM: two buffers of 128 columns, one per softmax warpgroup, each a 64-key
 // (query kernel) or 64-query (key kernel) sub-block's S and dP (S^T, dP^T) at
 // 128 b and 128 b + 64; the gradient accumulators from column 256.
@@ -554,7 +560,7 @@ __device__ inline void row_logits(float* x, const float* brow, const uint32_t* c
 }
 
 template <int HD>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdQThreads, 1)
     large_bwdq_kernel(const __grid_constant__ FastParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -569,8 +575,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* bias = (float*)(smem + L.bias);
   int* bins = (int*)(smem + L.bins);
   uint32_t* ci = (uint32_t*)(smem + L.words);
-  float* xch = (float*)(smem + L.xch);   // [kh][m, l, d, max|dP|][row]
-  float* wbd = xch + 2 * 4 * kRows;      // [8] warp bounds, [2][2] (E, finite) per item parity
+  float* wbd = (float*)(smem + L.xch);   // [16] warp bounds, [2][2] (E, finite) per item parity
   uint64_t* bars = (uint64_t*)(smem + L.bars);
   uint64_t* qd_full = bars;
   uint64_t* qd_empty = qd_full + 1;
@@ -592,16 +597,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const long long n_local = local_tiles(p.n_tiles, blockIdx.x, gridDim.x);
   if (threadIdx.x == 0) {
     mbar_init(qd_full, 1);
-    mbar_init(qd_empty, 1 + 8);   // the last S / dP products and every softmax warp
+    mbar_init(qd_empty, 1 + kBwdSoftWg * 4);   // the last S / dP products and every softmax warp
     for (int i = 0; i < NS; ++i) { mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sd_full[i], 1);
-      mbar_init(&st_free[i], kWg);
-      mbar_init(&ds_full[i], kWg);
+      mbar_init(&st_free[i], 2 * kWg);
+      mbar_init(&ds_full[i], 2 * kWg);
       mbar_init(&dq_done[i], 1);
     }
-    mbar_init(t_empty, 2 * kWg);
-    mbar_init(bins_full, 2 * kWg);
+    mbar_init(t_empty, kBwdSoftWg * kWg);
+    mbar_init(bins_full, kBwdSoftWg * kWg);
     mbar_init(bins_empty, 32);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
@@ -612,7 +617,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == kBwdProducer && lane == 0)
     for (int tt = 0; tt < 4; ++tt)
       for (int m = 0; m < kMaxMaps; ++m) prefetch_tmap(&p.maps[tt][m]);
-  for (int i = threadIdx.x; i < kBandPad; i += kBwdThreads) bins[i] = 0;
+  for (int i = threadIdx.x; i < kBandPad; i += kBwdQThreads) bins[i] = 0;
   if (warp == kBwdMma) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -757,7 +762,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const long long wh_item = t / kLargeBlocks;
       const int qb = (int)(t - wh_item * kLargeBlocks);
       const int h = (int)(wh_item - (wh_item / g.heads) * g.heads);
-      const float* eb = wbd + 8 + 2 * (int)(k & 1);
+      const float* eb = wbd + 16 + 2 * (int)(k & 1);
       const int E = (int)eb[0];
       const bool fin = eb[1] != 0.f;
       long long* acc = p.dt_acc + ((size_t)h * bp + qband0(qb)) * kLimbStride;
@@ -770,13 +775,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(bins_empty);
     }
   } else {
-    // Softmax / epilogue: warpgroup kh holds keys 64 kh .. 64 kh + 63 of every
-    // key block (sub-blocks 2 kb + kh, in TMEM buffer kh) for all 128 rows of
-    // the query block (thread = row = lane).
-    const int kh = warp >> 2;
+    // Softmax / epilogue: warpgroup wg holds keys 64 kh + 32 part .. + 31 of
+    // every key block (kh = wg >> 1: sub-blocks 2 kb + kh, in TMEM buffer kh;
+    // part = wg & 1) for all 128 rows of the query block (thread = row = lane).
+    const int wg = warp >> 2, kh = wg >> 1, part = wg & 1;
     const int row = threadIdx.x & (kWg - 1);
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_col = tmem + lane_base + 128 * kh;
+    const uint32_t s_col = tmem + lane_base + 128 * kh + 32 * part;
     const uint32_t dp_col = s_col + 64;
     const float c = p.scale_log2;
     const float dscale = p.scale_log2 * (1.0f / kLog2e);   // head_dim^-1/2
@@ -790,9 +795,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int slot = qb * kRows + row;
       const RowInfo me = plain ? plain_row_info<32>(g, win, slot) : block_row_info(g, win, slot);
       if (!plain)
-        for (int j = kh * kWg + row; j < kLargeKeys; j += 2 * kWg)
+        for (int j = wg * kWg + row; j < kLargeKeys; j += kBwdSoftWg * kWg)
           ci[j] = key_word(block_row_info(g, win, j));
-      if (named_sync_or(1, 2 * kWg, *abort)) break;
+      if (named_sync_or(1, kBwdSoftWg * kWg, *abort)) break;
       if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
       mbar_wait(qd_full, (uint32_t)(k & 1), abort, p.status, kWaitLimitNs);
       const float* brow = bias - qband0(qb);   // indexed by bin
@@ -802,12 +807,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int kb = 0; kb < kLargeBlocks; ++kb) {
         mbar_wait(&sd_full[kh], (uint32_t)(kb & 1), abort, p.status, kWaitLimitNs);
         tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          const int kw = kb * kRows + 64 * kh + 32 * cc;
+        {
+          const int kw = kb * kRows + 64 * kh + 32 * part;
           float x[32];
           __syncwarp();
-          tmem_ld32(s_col + 32 * cc, x);
+          tmem_ld32(s_col, x);
           tmem_wait_ld_regs(x);
           if (plain) row_logits<true>(x, brow, ci, kw, me, c);
           else row_logits<false>(x, brow, ci, kw, me, c);
@@ -823,7 +827,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const float mu = m == -INFINITY ? 0.f : m;
           float dp[32];
           __syncwarp();
-          tmem_ld32(dp_col + 32 * cc, dp);
+          tmem_ld32(dp_col, dp);
           tmem_wait_ld_regs(dp);
           float2 l2 = make_float2(0.f, 0.f), d2 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -839,27 +843,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         mbar_arrive(&st_free[kh]);
       }
-      // the two halves of each row merge; the block's bound sets its unit
+      // the four parts of each row merge (through TMEM columns 384 + 4 wg of
+      // the row's lane); the block's bound sets its unit
       {
-        float* mine = xch + kh * 4 * kRows;
-        mine[row] = m;
-        mine[kRows + row] = l;
-        mine[2 * kRows + row] = d;
-        mine[3 * kRows + row] = mdp;
+        const uint32_t xc = tmem + lane_base + kColXch;
+        tmem_st4(xc + 4 * wg, m, l, d, mdp);
+        tmem_wait_st();
+        tc_fence_before();
+        named_sync(2, kBwdSoftWg * kWg);
+        tc_fence_after();
+        float o[3][4];
+#pragma unroll
+        for (int i = 1; i < 4; ++i) tmem_ld4(xc + 4 * ((wg + i) & 3), o[i - 1]);
+        tmem_wait_ld();
+        float M = m;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) M = fmaxf(M, o[i][0]);
+        const float f0 = m == -INFINITY ? 0.f : ex2(m - M);
+        l *= f0;
+        d *= f0;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+          const float fi = o[i][0] == -INFINITY ? 0.f : ex2(o[i][0] - M);
+          l += o[i][1] * fi;
+          d += o[i][2] * fi;
+          mdp = fmaxf(mdp, o[i][3]);
+        }
+        m = M;
       }
-      named_sync(2, 2 * kWg);
-      const float* oth = xch + (1 - kh) * 4 * kRows;
-      const float mo = oth[row];
-      const float M = fmaxf(m, mo);
-      const float f0 = m == -INFINITY ? 0.f : ex2(m - M);
-      const float f1 = mo == -INFINITY ? 0.f : ex2(mo - M);
-      l = l * f0 + oth[kRows + row] * f1;
-      d = d * f0 + oth[2 * kRows + row] * f1;
-      mdp = fmaxf(mdp, oth[3 * kRows + row]);
+      const float M = m;
       const float Lr = me.valid ? M + __log2f(l) : INFINITY;   // P = 2^(x - L); 0 off real rows
       const float inv = me.valid ? 1.f / l : 0.f;             // max_j P_ij
       const float D = me.valid ? d * inv : 0.f;
-      if (kh == 0)
+      if (wg == 0)
         reinterpret_cast<float2*>(p.lse)[wh_item * kLargeKeys + slot] = make_float2(Lr, D);
       {
         float rb = inv * (mdp + fabsf(D));
@@ -867,16 +883,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float wb = warp_max(rb);
         if (lane == 0) wbd[warp] = wb;
       }
-      named_sync(2, 2 * kWg);
+      named_sync(2, kBwdSoftWg * kWg);
       float bound = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) bound = fmaxf(bound, wbd[i]);
+      for (int i = 0; i < kBwdSoftWg * 4; ++i) bound = fmaxf(bound, wbd[i]);
       const bool fin = bound <= 3.0e38f;
       const int E = tile_exponent(fin ? bound : 0.f);
       const float qs = exp2_int(E);
       if (threadIdx.x == 0) {
-        wbd[8 + 2 * (int)(k & 1)] = (float)E;
-        wbd[9 + 2 * (int)(k & 1)] = fin ? 1.f : 0.f;
+        wbd[16 + 2 * (int)(k & 1)] = (float)E;
+        wbd[17 + 2 * (int)(k & 1)] = fin ? 1.f : 0.f;
       }
       // the bins are free once the fold warp has taken the previous item's
       if (k > 0) mbar_wait(bins_empty, (uint32_t)((k - 1) & 1), abort, p.status, kWaitLimitNs);
@@ -885,13 +901,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int kb = 0; kb < kLargeBlocks; ++kb) {
         mbar_wait(&sd_full[kh], (uint32_t)(kb & 1), abort, p.status, kWaitLimitNs);
         tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          const int kw = kb * kRows + 64 * kh + 32 * cc;
+        {
+          const int kw = kb * kRows + 64 * kh + 32 * part;
           float x[32], ds[32];
           __syncwarp();
-          tmem_ld32(s_col + 32 * cc, x);
-          tmem_ld32(dp_col + 32 * cc, ds);
+          tmem_ld32(s_col, x);
+          tmem_ld32(dp_col, ds);
           tmem_wait_ld_regs(x);
           reg_fence32(ds);
           if (plain) row_logits<true>(x, brow, ci, kw, me, c);
@@ -924,7 +939,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             ds[j] = v.x;
             ds[j + 1] = v.y;
           }
-          split_to_tmem(dp_col + 32 * cc, ds);
+          split_to_tmem(dp_col, ds);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -933,21 +948,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(bins_full);
       __syncwarp();
       if (lane == 0) mbar_arrive(qd_empty);   // the bias run is read
-      // epilogue: this half's HD / 2 columns of the dQ row, once the item's
-      // last product (sub-block 15, buffer 1) is done
+      // epilogue: this warpgroup's HD / 4 columns of the dQ row, once the
+      // item's last product (sub-block 15, buffer 1) is done
       mbar_wait(&dq_done[1], 1u, abort, p.status, kWaitLimitNs);
       tc_fence_after();
       {
-        constexpr int OC = HD / 2;
+        constexpr int OC = HD / 4;
         float o[OC];
         __syncwarp();
-        if constexpr (OC == 32) tmem_ld32(tmem + lane_base + kColGrad + OC * kh, o);
-        else tmem_load_cols<OC>(tmem + lane_base + kColGrad + OC * kh, o);
+        if constexpr (OC == 32) tmem_ld32(tmem + lane_base + kColGrad + OC * wg, o);
+        else tmem_ld16(tmem + lane_base + kColGrad + OC * wg, o);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(t_empty);
         if (me.stored && !*abort)
-          store_row_bf16<OC>((__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD + OC * kh, o,
+          store_row_bf16<OC>((__nv_bfloat16*)p.out0 + (me.token * g.heads + h) * HD + OC * wg, o,
                              1.f);
       }
     }
@@ -961,7 +976,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 template <int HD>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdKThreads, 1)
     large_bwdk_kernel(const __grid_constant__ FastParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -994,14 +1009,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const long long n_local = local_tiles(p.n_tiles, blockIdx.x, gridDim.x);
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(kv_empty, 1 + 8);   // the last S^T / dP^T products and every softmax warp
+    mbar_init(kv_empty, 1 + kBwdSoftWg * 4);   // the last S^T / dP^T products and every softmax warp
     for (int i = 0; i < NS; ++i) { mbar_init(&qd_full[i], 1); mbar_init(&qd_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sd_full[i], 1);
-      mbar_init(&pds_full[i], kWg);
+      mbar_init(&pds_full[i], 2 * kWg);
       mbar_init(&grad_done[i], 1);
     }
-    mbar_init(t_empty, 2 * kWg);
+    mbar_init(t_empty, kBwdSoftWg * kWg);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
     mbar_init(never, 1);
@@ -1139,14 +1154,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_drain(&drain[1], 0, kTestLimitNs * 100);
       }
     }
-  } else if (warp < 8) {
-    // Softmax / epilogue: thread = key row = lane of the block; warpgroup kh
-    // takes queries 64 kh .. 64 kh + 63 of every query block (sub-blocks
-    // 2 qb + kh, in TMEM buffer kh).
-    const int kh = warp >> 2;
+  } else if (warp < kBwdSoftWg * 4) {
+    // Softmax / epilogue: thread = key row = lane of the block; warpgroup wg
+    // takes queries 64 kh + 32 part .. + 31 of every query block (kh = wg >> 1:
+    // sub-blocks 2 qb + kh, in TMEM buffer kh; part = wg & 1).
+    const int wg = warp >> 2, kh = wg >> 1, part = wg & 1;
     const int row = threadIdx.x & (kWg - 1);
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t s_col = tmem + lane_base + 128 * kh;
+    const uint32_t s_col = tmem + lane_base + 128 * kh + 32 * part;
     const uint32_t dp_col = s_col + 64;
     const float c = p.scale_log2;
     const float dscale = p.scale_log2 * (1.0f / kLog2e);   // head_dim^-1/2
@@ -1160,9 +1175,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int slot = kb * kRows + row;
       const RowInfo me = plain ? plain_row_info<32>(g, win, slot) : block_row_info(g, win, slot);
       if (!plain)
-        for (int j = kh * kWg + row; j < kLargeKeys; j += 2 * kWg)
+        for (int j = wg * kWg + row; j < kLargeKeys; j += kBwdSoftWg * kWg)
           qw[j] = key_word(block_row_info(g, win, j));
-      if (named_sync_or(1, 2 * kWg, *abort)) break;
+      if (named_sync_or(1, kBwdSoftWg * kWg, *abort)) break;
       if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
       mbar_wait(kv_full, (uint32_t)(k & 1), abort, p.status, kWaitLimitNs);
       // bias of (query j, this key) = brow[bias_base(j) - key_off]; a query's
@@ -1173,13 +1188,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int qb = 0; qb < kLargeBlocks; ++qb) {
         mbar_wait(&sd_full[kh], (uint32_t)(qb & 1), abort, p.status, kWaitLimitNs);
         tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          const int q0 = qb * kRows + 64 * kh + 32 * cc;   // first query slot of the chunk
+        {
+          const int q0 = qb * kRows + 64 * kh + 32 * part;   // first query slot of the chunk
           float x[32], dp[32];
           __syncwarp();
-          tmem_ld32(s_col + 32 * cc, x);
-          tmem_ld32(dp_col + 32 * cc, dp);
+          tmem_ld32(s_col, x);
+          tmem_ld32(dp_col, dp);
           tmem_wait_ld_regs(x);
           reg_fence32(dp);
           if (plain) {
@@ -1208,8 +1222,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             dp[j] = v.x;
             dp[j + 1] = v.y;
           }
-          split_to_tmem(s_col + 32 * cc, x);
-          split_to_tmem(dp_col + 32 * cc, dp);
+          split_to_tmem(s_col, x);
+          split_to_tmem(dp_col, dp);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -1217,26 +1231,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(kv_empty);   // bias run, statistics and query words read
-      // epilogue: this half's HD / 2 columns of the dV and dK rows of this key
+      // epilogue: this warpgroup's HD / 4 columns of the dV and dK rows of this key
       mbar_wait(&grad_done[1], 1u, abort, p.status, kWaitLimitNs);   // sub-block 15's products
       tc_fence_after();
       {
-        constexpr int OC = HD / 2;
-        const long long roff = (me.token * g.heads + h) * HD + OC * kh;
+        constexpr int OC = HD / 4;
+        const long long roff = (me.token * g.heads + h) * HD + OC * wg;
 #pragma unroll 1
-        for (int part = 0; part < 2; ++part) {
+        for (int gi = 0; gi < 2; ++gi) {
           float o[OC];
-          const uint32_t col = tmem + lane_base + kColGrad + part * HD + OC * kh;
+          const uint32_t col = tmem + lane_base + kColGrad + gi * HD + OC * wg;
           __syncwarp();
           if constexpr (OC == 32) tmem_ld32(col, o);
-          else tmem_load_cols<OC>(col, o);
+          else tmem_ld16(col, o);
           tmem_wait_ld();
-          if (part == 1) {
+          if (gi == 1) {
             tc_fence_before();
             mbar_arrive(t_empty);
           }
           if (me.stored && !*abort)
-            store_row_bf16<OC>((__nv_bfloat16*)(part ? p.out1 : p.out2) + roff, o, 1.f);
+            store_row_bf16<OC>((__nv_bfloat16*)(gi ? p.out1 : p.out2) + roff, o, 1.f);
         }
       }
     }
@@ -1357,13 +1371,13 @@ cudaError_t large_backward(const Geo& g, const void* q, const void* k, const voi
   cudaError_t e = prep_bias(g, table, bias_t, dt_acc, st);
   if (e != cudaSuccess) return e;
   if (g.hd == 128) {
-    e = large_launch(large_bwdq_kernel<128>, p, large_bwd_smem<128, false>(), kBwdThreads, st);
+    e = large_launch(large_bwdq_kernel<128>, p, large_bwd_smem<128, false>(), kBwdQThreads, st);
     if (e == cudaSuccess)
-      e = large_launch(large_bwdk_kernel<128>, p, large_bwd_smem<128, true>(), kBwdThreads, st);
+      e = large_launch(large_bwdk_kernel<128>, p, large_bwd_smem<128, true>(), kBwdKThreads, st);
   } else {
-    e = large_launch(large_bwdq_kernel<64>, p, large_bwd_smem<64, false>(), kBwdThreads, st);
+    e = large_launch(large_bwdq_kernel<64>, p, large_bwd_smem<64, false>(), kBwdQThreads, st);
     if (e == cudaSuccess)
-      e = large_launch(large_bwdk_kernel<64>, p, large_bwd_smem<64, true>(), kBwdThreads, st);
+      e = large_launch(large_bwdk_kernel<64>, p, large_bwd_smem<64, true>(), kBwdKThreads, st);
   }
   if (e != cudaSuccess) return e;
   if (flags & SWIN_FLAG_DBIAS_SUMS) return cudaSuccess;   // the caller finishes the sums
