@@ -1196,24 +1196,48 @@ __global__ void __launch_bounds__(kBwdKThreads, 1)
           tmem_ld32(dp_col, dp);
           tmem_wait_ld_regs(x);
           reg_fence32(dp);
+          // (L, D) of two queries per 16-byte load; eight queries between
+          // compiler barriers, so the loads in flight stay bounded (registers)
+          const float4* st4 = reinterpret_cast<const float4*>(stats + q0);
           if (plain) {
             const float* bq = brow + (q0 / 32) * 63 + q0 % 32;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float2 ld = stats[q0 + j];
-              const float pj = ex2(fmaf(x[j], c, bq[j]) - ld.x);
-              x[j] = pj;
-              dp[j] = pj * (dp[j] - ld.y);
+            for (int j0 = 0; j0 < 32; j0 += 8) {
+#pragma unroll
+              for (int j = j0; j < j0 + 8; j += 2) {
+                const float4 ld = st4[j >> 1];
+                const float2 t = __fadd2_rn(
+                    __ffma2_rn(make_float2(x[j], x[j + 1]), make_float2(c, c),
+                               make_float2(bq[j], bq[j + 1])),
+                    make_float2(-ld.x, -ld.z));
+                const float2 pj = make_float2(ex2(t.x), ex2(t.y));
+                const float2 v = __fmul2_rn(pj, __fadd2_rn(make_float2(dp[j], dp[j + 1]),
+                                                           make_float2(-ld.y, -ld.w)));
+                x[j] = pj.x;
+                x[j + 1] = pj.y;
+                dp[j] = v.x;
+                dp[j + 1] = v.y;
+              }
+              asm volatile("" ::: "memory");
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const uint32_t w = qw[q0 + j];
-              const float2 ld = stats[q0 + j];
-              const bool ok = live && (int)(w >> 16) == me.label;
-              const float pj = ok ? ex2(fmaf(x[j], c, brow[(int)(w & 0xFFFF)]) - ld.x) : 0.f;
-              x[j] = pj;
-              dp[j] = pj * (dp[j] - ld.y);
+            for (int j0 = 0; j0 < 32; j0 += 8) {
+#pragma unroll
+              for (int j = j0; j < j0 + 8; j += 2) {
+                const float4 ld = st4[j >> 1];
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                  const uint32_t w = qw[q0 + j + e2];
+                  const bool ok = live && (int)(w >> 16) == me.label;
+                  const float pj =
+                      ok ? ex2(fmaf(x[j + e2], c, brow[(int)(w & 0xFFFF)]) - (e2 ? ld.z : ld.x))
+                         : 0.f;
+                  x[j + e2] = pj;
+                  dp[j + e2] = pj * (dp[j + e2] - (e2 ? ld.w : ld.y));
+                }
+              }
+              asm volatile("" ::: "memory");
             }
           }
 #pragma unroll
