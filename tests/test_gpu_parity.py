@@ -316,6 +316,29 @@ def test_large_path_parity(case):
         assert e <= BF16_TOL, (case, n, e)
 
 
+def test_large_windows_on_the_table5_grid_two_heads():
+    """Table V's largest window on the 1/12-degree token grid: 256 x 544
+    tokens, 32 x 32 windows, shift 16, 8 heads x 128, the bench workload's
+    launch. The whole problem runs on the GPU; heads 0 and 7 are checked
+    against the oracle in full, and the backward repeats bitwise."""
+    wl = WORKLOADS["table5-large-256x544-8x128-w32"]
+    inp = make_inputs(wl)
+    d = sb.desc_for(wl)
+    assert sb.swin_wattn_path(d) == 4
+    gpu = run_gpu(d, inp, want_lse=False)
+    again = run_gpu(d, inp, want_lse=False)
+    for n in ("o", "dq", "dk", "dv", "dT"):
+        assert torch.equal(gpu[n], again[n]), n
+    for h in (0, 7):
+        sub = {n: inp[n][:, :, :, h:h + 1].contiguous() for n in ("q", "k", "v", "dout")}
+        sub["table"] = inp["table"][:, h:h + 1].contiguous()
+        ds = sb.make_desc(wl.B, wl.H, wl.W, wl.win, wl.shift, 1, wl.head_dim, wl.dtype)
+        g = {n: gpu[n][:, :, :, h:h + 1] for n in ("o", "dq", "dk", "dv")}
+        g["dT"] = gpu["dT"][:, h:h + 1]
+        for n, e in compare(g, run_oracle(ds, sub), "bf16").items():
+            assert e <= BF16_TOL, (h, n, e)
+
+
 @pytest.mark.parametrize("name", ["ragged-90x180-w8", "small-patch-2x512x1088-w8"])
 def test_tiled_path_forced_on_window64_workloads(name):
     """The warp-MMA kernels on the 8 x 8-window workloads the tcgen05 kernels
