@@ -108,10 +108,16 @@ typedef struct swin_wattn_desc {
 } swin_wattn_desc;
 
 /* Kernel family a description runs on:
- *   1 = tcgen05/TMA sm_100a kernels (bf16, 64-token windows, head_dim 32 or 64);
+ *   1 = tcgen05/TMA sm_100a kernels (bf16, 64-token windows, e.g. 8 x 8,
+ *       head_dim 32, 64 or 128);
+ *   3 = tcgen05/TMA kernels for 256-token windows (bf16, e.g. 16 x 16,
+ *       head_dim 32 or 64);
+ *   4 = tcgen05/TMA kernels for 1024-token windows (bf16, 32 x 32, head_dim
+ *       64 or 128, shifts whose 128-token block sub-boxes are whole 8-row
+ *       swizzle atoms, e.g. 16), with an online softmax over 128-token blocks;
  *   2 = warp-level tensor-core kernels, one CTA per (window, head) with the
- *       whole window in shared memory (bf16, windows of up to 256 tokens, e.g.
- *       16 x 16, head_dim 32 or 64);
+ *       whole window in shared memory (bf16, windows of up to 256 tokens the
+ *       families above do not take, e.g. 7 x 7, head_dim 32 or 64);
  *   0 = portable per-token CUDA kernels (everything else, fp32 included).
  * Returns a negative status for an invalid description. Host only, no CUDA
  * call. */
@@ -130,7 +136,7 @@ int swin_wattn_fwd(const swin_wattn_desc* desc, const void* q, const void* k, co
 /* Backward: dq, dk, dv (same layout and dtype as q) and dbias_table, all
  * overwritten, not accumulated. The softmax rows are recomputed from q, k, v
  * and the table; no forward state is needed. On the tensor-core kernels
- * (paths 1 and 2) dbias_table is summed exactly in integers whose unit follows
+ * (paths 1-4) dbias_table is summed exactly in integers whose unit follows
  * the magnitude of each tile's gradients, then rounded once to fp32: repeated
  * calls give identical bits, and the relative error does not depend on the
  * scale of dout. A NaN or infinity reaching a head's gradient makes that

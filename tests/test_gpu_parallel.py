@@ -15,7 +15,8 @@ from shifted_window_attention_pad_b200.workloads import Workload
 pytestmark = pytest.mark.gpu
 
 # (B, H, W, window, shift, heads, head_dim, seed, path)
-CASES = [(3, 36, 44, 8, 4, 5, 64, 51, 1), (2, 40, 52, 16, 8, 3, 64, 52, 3)]
+CASES = [(3, 36, 44, 8, 4, 5, 64, 51, 1), (2, 40, 52, 16, 8, 3, 64, 52, 3),
+         (2, 64, 64, 32, 16, 3, 128, 53, 4)]
 
 
 @pytest.fixture(scope="module", autouse=True)
