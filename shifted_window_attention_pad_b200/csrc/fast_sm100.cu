@@ -220,11 +220,20 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const bool plain = WW > 0 && window_plain(g, win);
       const RowInfo me = plain ? plain_row_info<WW>(g, win, lr) : row_info(g, win, lr);
       uint32_t* ci = colinfo + (wg * 2 + ((k / kNumWg) & 1)) * kRows;
-      ci[row] = key_word(me);
-      if (named_sync_or(1 + wg, kWg, *abort)) break;
+      // A plain window reads no key words, so its two warps need no barrier;
+      // the forward has no other warpgroup-wide barrier, so a warp may leave
+      // on its own when a wait has run out.
+      if (plain && *abort) break;
       if (p.test_timeout) mbar_wait(never, 0, abort, p.status, kTestLimitNs);
       mbar_wait(&s_full[sl], pht, abort, p.status, kWaitLimitNs);
       mbar_wait(&full[s], phs, abort, p.status, kWaitLimitNs);
+      if (!plain) {
+        // key words of the window's rows, published to its two warps only
+        // (written once S is ready: every thread of the warpgroup has then
+        // read the previous words of this buffer, two tiles back)
+        ci[row] = key_word(me);
+        if (named_sync_or(1 + 2 * wg + gw, N, *abort)) break;
+      }
       tc_fence_after();
       float x[N];
       tmem_load_cols<N>(tmem + lane_base + sl * SC + gw * N, x);

@@ -151,3 +151,20 @@ def test_workspace_size_follows_the_documented_layout(L, name):
 def test_strerror_covers_every_status(L):
     for s in range(-5, 1):
         assert sb.swin_wattn_strerror(s) != "unknown status"
+
+
+@pytest.mark.parametrize("win,hd,path", [((16, 16), 64, 3), ((32, 32), 128, 4)])
+def test_row_band_entry_points_take_only_64_token_windows(L, win, hd, path):
+    """A row band needs the 64-token kernels' halo boxes; other families are
+    refused on the host, before any pointer is touched (these are fake,
+    aligned host addresses)."""
+    d = sb.make_desc(1, 64, 96, win, (win[0] // 2, win[1] // 2), 2, hd, "bf16")
+    assert sb.swin_wattn_path(d) == path
+    fake = ctypes.c_void_p(1 << 20)
+    halo = sb.SwinWattnHalo(0, fake, fake, fake, fake, fake, None, fake, fake, fake)
+    rc = L.swin_wattn_fwd_band(ctypes.byref(d), ctypes.byref(halo), fake, fake, fake, fake, fake,
+                               None, fake, ctypes.c_size_t(1 << 30), None)
+    assert rc == -2   # SWIN_ERR_UNSUPPORTED
+    rc = L.swin_wattn_bwd_band(ctypes.byref(d), ctypes.byref(halo), fake, fake, fake, fake, fake,
+                               fake, fake, fake, fake, fake, ctypes.c_size_t(1 << 30), None)
+    assert rc == -2   # SWIN_ERR_UNSUPPORTED

@@ -107,6 +107,7 @@ VALID = [
     (0, Workload("valid-portable", 1, 13, 18, 4, 2, 2, 16, "f32", 73, valid=(11, 15))),
     (1, Workload("valid-1/12-degree-field", 1, 256, 544, 8, 4, 4, 64, "bf16", 74,
                  valid=sb.field_valid_extent(2041, 4320, 8))),
+    (4, Workload("valid-tcgen05-w32", 1, 64, 96, 32, 16, 2, 128, "bf16", 76, valid=(61, 90))),
 ]
 
 
