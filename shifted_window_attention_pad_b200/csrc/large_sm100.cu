@@ -812,10 +812,15 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
         tc_fence_after();
         {
           const int kw = kb * kRows + 64 * kh + 32 * part;
-          float x[32];
+          float x[32], dp[32];
           __syncwarp();
           tmem_ld32(s_col, x);
+          tmem_ld32(dp_col, dp);
           tmem_wait_ld_regs(x);
+          reg_fence32(dp);
+          // S and dP are in registers: the buffer's next products may start
+          tc_fence_before();
+          mbar_arrive(&st_free[kh]);
           if (plain) row_logits<true>(x, brow, ci, kw, me, c);
           else row_logits<false>(x, brow, ci, kw, me, c);
           float cm = -INFINITY;
@@ -828,10 +833,6 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
             m = cm;
           }
           const float mu = m == -INFINITY ? 0.f : m;
-          float dp[32];
-          __syncwarp();
-          tmem_ld32(dp_col, dp);
-          tmem_wait_ld_regs(dp);
           float2 l2 = make_float2(0.f, 0.f), d2 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
@@ -843,8 +844,6 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
           l += l2.x + l2.y;
           d += d2.x + d2.y;
         }
-        tc_fence_before();
-        mbar_arrive(&st_free[kh]);
       }
       // the four parts of each row merge (through TMEM columns 384 + 4 wg of
       // the row's lane); the block's bound sets its unit
