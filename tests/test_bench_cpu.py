@@ -62,3 +62,22 @@ def test_l2_flush_only_for_workloads_smaller_than_twice_l2():
     for name, flush in want.items():
         assert bench.needs_l2_flush(WORKLOADS[name]) == flush, name
     assert bench.input_bytes(WORKLOADS["twelfth-degree-256x544-w8"]) == 4 * 256 * 544 * 16 * 64 * 2
+
+
+def test_roofline_entry_holds_1024_token_windows_to_the_tensor_peak():
+    """32 x 32 windows do N/2 = 512 FLOP per byte, past the ridge of the
+    measured peaks: their backward is held to the bf16 tensor peak in
+    TFLOP/s; every other family to HBM bandwidth in GB/s."""
+    import bench
+    from shifted_window_attention_pad_b200 import WORKLOADS
+    hbm, tf, _ = bench.measured_peaks()
+    assert tf / hbm * 1e3 < 512                      # the ridge in FLOP per byte
+    wl = WORKLOADS["table5-large-256x544-8x128-w32"]
+    assert wl.flops_bwd() == 8 * 1024 * 128 * 256 * 544 * 8
+    e = bench.roofline_entry(4, wl, 5.0, 400.0, hbm, "measured", None, wl.alg_bytes_bwd())
+    assert e["bound"] == "tensor" and e["unit"] == "TFLOP/s" and e["peak"] == tf
+    assert abs(e["achieved"] - wl.flops_bwd() / 5e-3 / 1e12) < 1e-9
+    assert abs(e["frac"] - e["achieved"] / tf) < 1e-12
+    wl8 = WORKLOADS["twelfth-degree-256x544-w8"]
+    e = bench.roofline_entry(1, wl8, 0.75, 2660.0, hbm, "measured", None, wl8.alg_bytes_bwd())
+    assert e["bound"] == "hbm" and e["unit"] == "GB/s" and e["achieved"] == 2660.0
