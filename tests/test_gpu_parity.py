@@ -289,7 +289,7 @@ def test_wide_path_parity(case):
 # (B, H, W, window, shift, heads, head_dim, seed): both seams at head_dim 128
 # and 64, a padded grid, no shift, batch 2, a row shift whose seam splits a
 # 128-token block (window row 18 of 32), the largest model's window at the
-# 1/12-degree grid's width
+# 1/12-degree grid's width, a grid smaller than one window
 LARGE = [
     (1, 64, 96, (32, 32), (16, 16), 2, 128, 91),
     (1, 40, 72, (32, 32), (16, 16), 1, 64, 92),
@@ -297,6 +297,7 @@ LARGE = [
     (2, 64, 64, (32, 32), (16, 16), 1, 128, 94),
     (1, 64, 96, (32, 32), (14, 16), 1, 64, 95),
     (1, 32, 544, (32, 32), (16, 16), 1, 128, 96),
+    (1, 20, 24, (32, 32), (16, 16), 2, 64, 97),
 ]
 
 
