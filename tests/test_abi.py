@@ -168,3 +168,22 @@ def test_row_band_entry_points_take_only_64_token_windows(L, win, hd, path):
     rc = L.swin_wattn_bwd_band(ctypes.byref(d), ctypes.byref(halo), fake, fake, fake, fake, fake,
                                fake, fake, fake, fake, fake, ctypes.c_size_t(1 << 30), None)
     assert rc == -2   # SWIN_ERR_UNSUPPORTED
+
+
+def test_1024_token_workspace_adds_the_rows_statistics(L):
+    """Path 4's workspace: the header, the bias table [heads][bins rounded up
+    to 4] fp32, the exact bias-gradient sums (10 int64 words per head and
+    bin), then L and D (float2) of every query of every window and head, each
+    part rounded up to 256 bytes; the sums sit where swin_wattn_dbias_sums
+    says."""
+    a256 = lambda x: (x + 255) // 256 * 256
+    for (H, W, heads, hd) in [(64, 96, 2, 128), (256, 544, 8, 128), (20, 24, 3, 64)]:
+        d = sb.make_desc(1, H, W, (32, 32), (16, 16), heads, hd, "bf16")
+        assert sb.swin_wattn_path(d) == 4
+        bp = (63 * 63 + 3) // 4 * 4
+        n_win = (-(-H // 32)) * (-(-W // 32))
+        want = 256 + a256(heads * bp * 4) + a256(heads * bp * 80) + a256(n_win * heads * 1024 * 8)
+        assert sb.swin_wattn_workspace_size(d) == want
+        off, nbytes = ctypes.c_size_t(0), ctypes.c_size_t(0)
+        assert L.swin_wattn_dbias_sums(ctypes.byref(d), ctypes.byref(off), ctypes.byref(nbytes)) == 0
+        assert off.value == 256 + a256(heads * bp * 4) and nbytes.value == heads * bp * 80
