@@ -951,7 +951,13 @@ __global__ void __launch_bounds__(kBwdQThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(qd_empty);   // the bias run is read
       // epilogue: this warpgroup's HD / 4 columns of the dQ row, once the
-      // item's last product (sub-block 15, buffer 1) is done
+      // item's last product (sub-block 15, buffer 1) is done. A parity wait
+      // only names a phase when the barrier is at most one phase behind it:
+      // this buffer's own barrier is (its last sub-block's S and dP were
+      // issued after the one before had completed), and its last products
+      // completing brings buffer 1's there as well (products complete in
+      // issue order), so buffer 0's warpgroups wait on their own first.
+      mbar_wait(&dq_done[kh], 1u, abort, p.status, kWaitLimitNs);
       mbar_wait(&dq_done[1], 1u, abort, p.status, kWaitLimitNs);
       tc_fence_after();
       {
@@ -1258,7 +1264,11 @@ __global__ void __launch_bounds__(kBwdKThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(kv_empty);   // bias run, statistics and query words read
       // epilogue: this warpgroup's HD / 4 columns of the dV and dK rows of this key
-      mbar_wait(&grad_done[1], 1u, abort, p.status, kWaitLimitNs);   // sub-block 15's products
+      // sub-block 15's products (buffer 1); buffer 0's warpgroups first wait
+      // for their own last products, which leaves buffer 1's barrier at most
+      // one phase behind the one the parity names (as in the query kernel)
+      mbar_wait(&grad_done[kh], 1u, abort, p.status, kWaitLimitNs);
+      mbar_wait(&grad_done[1], 1u, abort, p.status, kWaitLimitNs);
       tc_fence_after();
       {
         constexpr int OC = HD / 4;
