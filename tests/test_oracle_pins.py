@@ -145,7 +145,7 @@ def _sdpa_heads(qt, kt, vt, mask=None):
     return F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask)
 
 
-@pytest.mark.parametrize("H,W", [(6, 5), (4, 8), (3, 3)])
+@pytest.mark.parametrize("H,W", [(6, 5), (4, 8), (3, 3), (32, 32)])
 def test_one_window_no_shift_zero_bias_equals_sdpa(H, W):
     heads, hd = 2, 8
     s, q, k, v, T, do = problem(1, H, W, (H, W), 0, heads, hd, seed=11)
@@ -170,7 +170,7 @@ def test_one_window_with_padding_equals_sdpa_over_valid_tokens():
     np.testing.assert_allclose(o[0], ref, rtol=0, atol=1e-12)
 
 
-@pytest.mark.parametrize("H,W,win", [(6, 5, (6, 5)), (5, 7, 8)])
+@pytest.mark.parametrize("H,W,win", [(6, 5, (6, 5)), (5, 7, 8), (32, 32, 32), (20, 27, 32)])
 def test_one_window_backward_equals_autograd(H, W, win):
     heads, hd = 2, 5
     s, q, k, v, T, do = problem(1, H, W, win, 0, heads, hd, seed=13)
